@@ -1,0 +1,248 @@
+"""CPU oracle for the RPTQ data path -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py`` may import this package.  The product path (``post_activation_quantization_b200``)
+never imports it and fails loudly when its CUDA library is missing.
+
+The arithmetic lives in ``rptq_oracle.c`` (plain single-threaded C, fp64 unless a step fixes
+fp32, built with ``-ffp-contract=off``); this module only marshals numpy arrays into it.
+Inputs in fp16/bf16 are widened to fp32 here, which is exact.
+
+Sources (page title + part), the same as in the C file:
+  [RPTQ-art]  "基于重排序的新量化方法RPTQ：实现大型语言模型的 3 比特量化": Fig. 1 caption, the text
+              after Fig. 2 (calibration, KMeans, reorder, per-cluster s/z), the text after Fig. 3
+              (LayerNorm emits reordered activations), the results paragraph (K/V quantization).
+  [Basics]    quantization-basics article (gitcode.csdn.net), sections 一, 1.1, 1.3, 1.4.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "rptq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library in place (gcc, -O2 -ffp-contract=off)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+             "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = ctypes.CDLL(_LIB)
+    return _lib
+
+
+def _p(a: np.ndarray | None):
+    if a is None:
+        return None
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _f32(x) -> np.ndarray:
+    """Exact widening of an fp16/bf16/fp32 array (numpy or torch CPU tensor) to fp32."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return np.ascontiguousarray(x.detach().to("cpu", torch.float32).numpy())
+    except ImportError:  # pragma: no cover
+        pass
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_DBL = ctypes.c_double
+
+
+def minmax(x, ch_max=None, ch_min=None):
+    """Per-channel (max, min) of x [T, C].  With ch_max/ch_min given, folds into them."""
+    x = _f32(x)
+    T, C = x.shape
+    acc = ch_max is not None
+    mx = np.array(ch_max, dtype=np.float32) if acc else np.empty(C, np.float32)
+    mn = np.array(ch_min, dtype=np.float32) if acc else np.empty(C, np.float32)
+    _load().orc_minmax(_p(x), _I64(T), _INT(C), _p(mx), _p(mn), _INT(int(acc)))
+    return mx, mn
+
+
+def layernorm(x, gamma, beta, eps=1e-5):
+    """LayerNorm in fp64; returns (y64, y32) in the ORIGINAL channel order."""
+    x = _f32(x)
+    T, C = x.shape
+    g, b = _f32(gamma), _f32(beta)
+    y64 = np.empty((T, C), np.float64)
+    y32 = np.empty((T, C), np.float32)
+    _load().orc_layernorm(_p(x), _I64(T), _INT(C), _p(g), _p(b), _DBL(eps), _p(y64), _p(y32))
+    return y64, y32
+
+
+def minmax_ln(x, gamma, beta, eps=1e-5, ch_max=None, ch_min=None):
+    """Per-channel (max, min) of the fp32-rounded LayerNorm output of x."""
+    x = _f32(x)
+    T, C = x.shape
+    acc = ch_max is not None
+    mx = np.array(ch_max, dtype=np.float32) if acc else np.empty(C, np.float32)
+    mn = np.array(ch_min, dtype=np.float32) if acc else np.empty(C, np.float32)
+    _load().orc_minmax_ln(_p(x), _I64(T), _INT(C), _p(_f32(gamma)), _p(_f32(beta)), _DBL(eps),
+                          _p(mx), _p(mn), _INT(int(acc)))
+    return mx, mn
+
+
+def kmeans_init(ch_max, ch_min, g):
+    mx, mn = _f32(ch_max), _f32(ch_min)
+    cent = np.empty((g, 2), np.float64)
+    rc = _load().orc_kmeans_init(_p(mx), _p(mn), _INT(mx.size), _INT(g), _p(cent))
+    if rc != 0:
+        raise ValueError("kmeans_init: need 1 <= g <= C")
+    return cent
+
+
+def kmeans_assign(ch_max, ch_min, cent, labels=None):
+    mx, mn = _f32(ch_max), _f32(ch_min)
+    cent = np.ascontiguousarray(cent, dtype=np.float64)
+    lab = np.full(mx.size, -1, np.int32) if labels is None else _i32(labels).copy()
+    changed = _load().orc_kmeans_assign(_p(mx), _p(mn), _INT(mx.size), _INT(cent.shape[0]),
+                                        _p(cent), _p(lab))
+    return lab, changed
+
+
+def kmeans_update(ch_max, ch_min, labels, cent):
+    mx, mn = _f32(ch_max), _f32(ch_min)
+    out = np.array(cent, dtype=np.float64, copy=True)
+    _load().orc_kmeans_update(_p(mx), _p(mn), _INT(mx.size), _INT(out.shape[0]), _p(_i32(labels)),
+                              _p(out))
+    return out
+
+
+def kmeans(ch_max, ch_min, g, iters):
+    """Deterministic Lloyd KMeans; returns (labels int32[C], centroids fp64[g, 2])."""
+    mx, mn = _f32(ch_max), _f32(ch_min)
+    C = mx.size
+    labels = np.empty(C, np.int32)
+    cent = np.empty((g, 2), np.float64)
+    rc = _load().orc_kmeans(_p(mx), _p(mn), _INT(C), _INT(g), _INT(iters), _p(labels), _p(cent))
+    if rc != 0:
+        raise ValueError("kmeans: need 1 <= g <= C and iters >= 0")
+    return labels, cent
+
+
+def reorder(labels, g):
+    """Stable counting sort by cluster: returns (R, col_cluster, offsets)."""
+    lab = _i32(labels)
+    C = lab.size
+    R = np.empty(C, np.int32)
+    cc = np.empty(C, np.int32)
+    off = np.empty(g + 1, np.int32)
+    _load().orc_reorder(_p(lab), _INT(C), _INT(g), _p(R), _p(cc), _p(off))
+    return R, cc, off
+
+
+def cluster_params(ch_max, ch_min, labels, g, bits):
+    """Per-cluster fp32 scale and int32 zero point."""
+    mx, mn = _f32(ch_max), _f32(ch_min)
+    s = np.empty(g, np.float32)
+    z = np.empty(g, np.int32)
+    _load().orc_cluster_params(_p(mx), _p(mn), _p(_i32(labels)), _INT(mx.size), _INT(g),
+                               _INT(bits), _p(s), _p(z))
+    return s, z
+
+
+def quantize(y, col_cluster, s, z, bits):
+    """Unpacked codes (uint8) of y [rows, C], column j in cluster col_cluster[j]."""
+    y = _f32(y)
+    rows, C = y.shape
+    q = np.empty((rows, C), np.uint8)
+    _load().orc_quantize(_p(y), _I64(rows), _INT(C), _p(_i32(col_cluster)), _p(_f32(s)),
+                         _p(_i32(z)), _INT(bits), _p(q))
+    return q
+
+
+def pack(q, bits):
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    rows, C = q.shape
+    out = np.empty((rows, C * bits // 8), np.uint8)
+    _load().orc_pack(_p(q), _I64(rows), _INT(C), _INT(bits), _p(out))
+    return out
+
+
+def unpack(packed, C, bits):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    rows = packed.shape[0]
+    q = np.empty((rows, C), np.uint8)
+    _load().orc_unpack(_p(packed), _I64(rows), _INT(C), _INT(bits), _p(q))
+    return q
+
+
+def dequant(q, col_cluster, s, z):
+    """fp32 values s*(q - z) of unpacked codes q [rows, C]."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    rows, C = q.shape
+    out = np.empty((rows, C), np.float32)
+    _load().orc_dequant(_p(q), _I64(rows), _INT(C), _p(_i32(col_cluster)), _p(_f32(s)),
+                        _p(_i32(z)), _p(out))
+    return out
+
+
+def ln_reorder_quant(x, gamma, beta, R, col_cluster, s, z, bits, eps=1e-5, want_codes=True,
+                     want_ln=False):
+    """Unfused definition: LN -> gather(R) -> quantize -> pack.
+
+    Returns (packed or None, ln32 or None, ln64 or None); ln outputs are in stored order.
+    """
+    x = _f32(x)
+    T, C = x.shape
+    packed = np.empty((T, C * bits // 8), np.uint8) if want_codes else None
+    ln32 = np.empty((T, C), np.float32) if want_ln else None
+    ln64 = np.empty((T, C), np.float64) if want_ln else None
+    _load().orc_ln_reorder_quant(_p(x), _I64(T), _INT(C), _p(_f32(gamma)), _p(_f32(beta)),
+                                 _DBL(eps), _p(_i32(R)), _p(_i32(col_cluster)), _p(_f32(s)),
+                                 _p(_i32(z)), _INT(bits), _p(packed), _p(ln32), _p(ln64))
+    return packed, ln32, ln64
+
+
+def kv_quant(kv, col_cluster, s, z, bits):
+    """Packed codes of a [B, H, S, D] tensor, channel c = h*D + d, layout kept."""
+    kv = _f32(kv)
+    B, H, S, D = kv.shape
+    out = np.empty((B, H, S, D * bits // 8), np.uint8)
+    _load().orc_kv_quant(_p(kv), _I64(B), _INT(H), _I64(S), _INT(D), _p(_i32(col_cluster)),
+                         _p(_f32(s)), _p(_i32(z)), _INT(bits), _p(out))
+    return out
+
+
+def kv_dequant(packed, D, col_cluster, s, z, bits):
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    B, H, S, _ = packed.shape
+    out = np.empty((B, H, S, D), np.float32)
+    _load().orc_kv_dequant(_p(packed), _I64(B), _INT(H), _I64(S), _INT(D), _p(_i32(col_cluster)),
+                           _p(_f32(s)), _p(_i32(z)), _INT(bits), _p(out))
+    return out
+
+
+def calibrate(ch_max, ch_min, g, iters, bits):
+    """The whole offline chain on given statistics: KMeans -> reorder -> cluster params."""
+    labels, cent = kmeans(ch_max, ch_min, g, iters)
+    R, cc, off = reorder(labels, g)
+    s, z = cluster_params(ch_max, ch_min, labels, g, bits)
+    return dict(labels=labels, centroids=cent, R=R, col_cluster=cc, offsets=off, scale=s, zero=z)
