@@ -1,0 +1,215 @@
+/*
+ * rptq.h -- C ABI of librptq.so: the RPTQ data path on NVIDIA B200 (sm_100a).
+ *
+ * RPTQ (reorder-based post-training quantization) quantizes LLM activations per cluster of
+ * channels.  Sources, cited by page title and the part of the page:
+ *  [RPTQ-art]  "基于重排序的新量化方法RPTQ：实现大型语言模型的 3 比特量化":
+ *              Fig. 1 caption (one (max, min) point per activation channel); the text after
+ *              Fig. 2 (calibrate per-channel max/min, KMeans into g clusters, reorder so that a
+ *              cluster's channels are adjacent, one scale s and zero point z per cluster); the
+ *              text after Fig. 3 (LayerNorm changed to emit the reordered activations, so no
+ *              explicit reorder runs); the results paragraph (K/V cache quantized alone:
+ *              W4A4KV, W4A3KV, W3A3KV) and the closing memory paragraph.
+ *  [Houmo-art] RPTQ / PB-LLM article, section "RPTQ：量化激活通道的新思路" (3-bit activations;
+ *              reorder removed by operator fusion).
+ *  [Basics]    quantization-basics article (gitcode.csdn.net), section 一 (scale = float
+ *              range / integer range), 1.1 (static ranges, outliers clamped), 1.3 (zero point,
+ *              dequantization S(Wq - Z)), 1.4 (granularity).
+ *
+ * Conventions for every entry point
+ *  - Tensor arguments are DEVICE pointers on the current CUDA device, owned by the caller,
+ *    never freed or retained by the library.  Tensors are dense, row-major, and their base
+ *    addresses must be 16-byte aligned (what cudaMalloc and torch allocations give).
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and is
+ *    asynchronous: outputs are valid once the stream has been synchronised.
+ *  - Arguments are validated on the host before anything is launched; an invalid call
+ *    returns a negative status and launches nothing.  No C++ exception crosses the ABI.
+ *  - Kernels never trap.  Conditions only the device can see (a cluster id outside [0, g), an
+ *    R entry outside [0, C), a bounded wait that ran out) set a sticky device error word and
+ *    the kernel carries on with safe values; read and clear it with rptq_device_error().
+ *  - Calls that touch the same output buffers must not overlap on the GPU.
+ *
+ * Notation: T tokens, C channels, g clusters, b = bits (3 or 4), qmax = 2^b - 1.
+ *
+ * Packed code layout (the pages only name 3- and 4-bit codes; this is the library's layout):
+ *   a row of C codes takes C*b/8 bytes (C must be a multiple of 8);
+ *   b = 4: code 2i -> low nibble of byte i, code 2i+1 -> high nibble;
+ *   b = 3: codes 8m..8m+7 -> bytes 3m..3m+2; code 8m+k at bits [3k, 3k+3) of the
+ *          little-endian 24-bit word byte0 | byte1 << 8 | byte2 << 16.
+ */
+#ifndef RPTQ_H_
+#define RPTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so that this header needs no CUDA header. */
+typedef struct CUstream_st *rptq_stream_t;
+
+/* Status codes. */
+#define RPTQ_OK 0
+#define RPTQ_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size or range */
+#define RPTQ_ERR_UNSUPPORTED (-2) /* bits not 3/4, C not a multiple of 8, C too large, dtype */
+#define RPTQ_ERR_WORKSPACE (-3)   /* workspace pointer null or smaller than required */
+#define RPTQ_ERR_CUDA (-4)        /* a CUDA runtime call or a launch failed */
+#define RPTQ_ERR_DEVICE (-5)      /* the device error word was set (see rptq_device_error) */
+
+/* Element types. */
+#define RPTQ_F32 0
+#define RPTQ_F16 1
+#define RPTQ_BF16 2
+
+/* Code layouts for rptq_dequant. */
+#define RPTQ_LAYOUT_ROWS 0 /* [rows, C], column j in cluster col_cluster[j] */
+#define RPTQ_LAYOUT_BHSD 1 /* [B, H, S, D] packed along D, channel c = h*D + d */
+
+/* Largest channel count C (and H*D) any entry point accepts. */
+#define RPTQ_MAX_CHANNELS 16384
+/* Largest cluster count g. */
+#define RPTQ_MAX_CLUSTERS 1024
+
+/* Human-readable text of a status code (static storage, never NULL). */
+const char *rptq_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int rptq_version(void);
+
+/*
+ * Device error word.  Waits for `stream` to finish, stores the sticky device error word of
+ * the current device in *code (0 = none; otherwise a bit set of RPTQ_DEVERR_* values) and
+ * clears it.  Returns RPTQ_OK, or RPTQ_ERR_CUDA if the synchronisation or copy failed.
+ */
+#define RPTQ_DEVERR_CLUSTER_ID 1 /* a cluster id was outside [0, g); cluster 0 was used */
+#define RPTQ_DEVERR_REORDER 2    /* an R entry was outside [0, C) */
+#define RPTQ_DEVERR_TIMEOUT 4    /* a bounded wait on an asynchronous copy ran out */
+int rptq_device_error(rptq_stream_t stream, int *code);
+
+/*
+ * Calibration statistics: per-channel maximum and minimum over T tokens.
+ * [RPTQ-art] text after Fig. 2 and Fig. 1 caption.  The statistic is taken on the tensor
+ * that will be quantized: with gamma != NULL it is LayerNorm(x) (the activation path),
+ * otherwise x itself (the K/V path).
+ *   x        [T, C] of `dtype` (RPTQ_F32 / RPTQ_F16 / RPTQ_BF16).
+ *   gamma, beta  fp32 [C] in the original channel order, or both NULL.
+ *   eps      LayerNorm epsilon (added to the biased variance); ignored without gamma.
+ *   ch_max, ch_min  fp32 [C] outputs.  accumulate = 0 overwrites them; accumulate = 1 folds
+ *            this batch into the values already there (calibrate in chunks).
+ * In raw mode (gamma == NULL) the results are exact (bit-identical to a CPU max/min).
+ * LayerNorm mode computes the normalisation in fp32 (single-pass moments with an exact
+ * two-pass fallback for rows whose mean is large against their spread).
+ * T == 0 is valid (no work; with accumulate = 0 the outputs become -inf / +inf).
+ */
+int rptq_calib_minmax(const void *x, int dtype, int64_t T, int C, const float *gamma,
+                      const float *beta, float eps, float *ch_max, float *ch_min,
+                      int accumulate, rptq_stream_t stream);
+
+/*
+ * Calibration statistics of a K or V cache in its attention layout: kv is [B, H, S, D] of
+ * `dtype`, channel c = h*D + d, and the max / min of every channel are taken over the B*S
+ * tokens (exact, like raw-mode rptq_calib_minmax).  ch_max, ch_min: fp32 [H*D].
+ * accumulate as in rptq_calib_minmax.  D must be a multiple of 8, D <= 2048, H*D <=
+ * RPTQ_MAX_CHANNELS.  [RPTQ-art] results paragraph (K/V cache quantized per cluster) with the
+ * calibration of the text after Fig. 2.
+ */
+int rptq_kv_calib_minmax(const void *kv, int dtype, int B, int H, int64_t S, int D, float *ch_max,
+                         float *ch_min, int accumulate, rptq_stream_t stream);
+
+/* Workspace bytes rptq_kmeans needs for C points and g clusters (0 for invalid sizes). */
+size_t rptq_kmeans_workspace_size(int C, int g);
+
+/*
+ * KMeans on the C points (ch_max[c], ch_min[c]), then the reorder index and the per-cluster
+ * quantization parameters.  [RPTQ-art] text after Fig. 2 (KMeans on the (max, min) points,
+ * same-cluster channels placed together, per-cluster s and z); [Basics] sections 一, 1.3.
+ * Fixed readings (deterministic, identical on every run):
+ *   - points are (double)ch_max[c], (double)ch_min[c];
+ *   - init: channels sorted by (max, min, index) ascending; centroid k = point at sorted
+ *     position floor((2k+1) C / (2g));
+ *   - `iters` rounds of (assign, update) then a final assign; assign = argmin of the fp64
+ *     squared distance dx*dx + dy*dy (no fused multiply-add), ties to the lowest k;
+ *     update = mean of the members; an empty cluster keeps its centroid.  The loop stops
+ *     early once an assignment repeats the previous one (provably the same result);
+ *   - R: stable counting sort of the channels by label (clusters in label order, channels
+ *     ascending inside each cluster);
+ *   - cluster range M_k = max of members' ch_max, m_k = min of members' ch_min;
+ *     scale s_k = (M_k - m_k) / qmax and zero z_k = rint(-m_k / s_k), fp32 IEEE divides,
+ *     round-half-to-even, z not clamped; M_k == m_k gives s_k = max(|m_k|, |M_k|) / qmax
+ *     (1 / qmax if both are 0); an empty cluster gets s = 1, z = 0.
+ * Inputs: 1 <= g <= min(C, RPTQ_MAX_CLUSTERS), 1 <= C <= RPTQ_MAX_CHANNELS, iters >= 0,
+ * bits in {3, 4}, finite statistics.
+ * Outputs (device): labels int32[C]; centroids fp64[g][2] as (max, min); R int32[C]
+ * (R[j] = channel stored at column j); col_cluster int32[C] (= labels[R[j]], non-decreasing);
+ * offsets int32[g+1] (first stored column of each cluster, offsets[g] = C); scale fp32[g];
+ * zero int32[g].
+ * workspace: device buffer of at least rptq_kmeans_workspace_size(C, g) bytes, owned by the
+ * caller; its contents need no initialisation and are garbage afterwards.
+ */
+int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iters, int bits,
+                int32_t *labels, double *centroids, int32_t *R, int32_t *col_cluster,
+                int32_t *offsets, float *scale, int32_t *zero, void *workspace,
+                size_t workspace_bytes, rptq_stream_t stream);
+
+/*
+ * Reorder-fused LayerNorm with per-cluster quantization: the runtime activation path.
+ * [RPTQ-art] text after Fig. 3 (the LayerNorm itself emits channels in cluster order, so no
+ * reordered copy of x is ever stored); text after Fig. 2 (per-cluster s, z); [Houmo-art]
+ * (reorder fused away, 3-bit activations); [Basics] 1.1 (static range: out-of-range values
+ * clamp), 1.3 (q = round(y / s) + z).
+ * For every token t, with y = LayerNorm(x[t]) over the C channels in the ORIGINAL order
+ * (mean, biased variance, eps, gamma, beta):
+ *   stored column j holds channel R[j]; k = col_cluster[j];
+ *   code[t][j] = clamp(rint(y[R[j]] / scale[k]) + zero[k], 0, qmax)  (half-to-even),
+ *   ln_out[t][j] = y[R[j]] rounded to `dtype`.
+ *   x            [T, C] of `dtype`.
+ *   gamma, beta  fp32 [C], original channel order.
+ *   R, col_cluster  int32 [C] from rptq_kmeans.  R must be a permutation of [0, C): entries
+ *                outside [0, C) are reported and skipped; repeated entries are not detected.
+ *   scale, zero  fp32 [g], int32 [g]; g is the length of these tables.
+ *   codes        uint8 [T, C*bits/8] packed codes in stored order, or NULL.
+ *   ln_out       [T, C] of `dtype`, stored order, or NULL.  At least one of codes / ln_out.
+ * Codes are computed in fp32 and may differ from an exact-arithmetic reference by one step
+ * where y / scale lies within fp32 rounding of a half-integer.
+ */
+int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const float *gamma,
+                          const float *beta, float eps, const int32_t *R,
+                          const int32_t *col_cluster, const float *scale, const int32_t *zero,
+                          int g, int bits, uint8_t *codes, void *ln_out, rptq_stream_t stream);
+
+/*
+ * K/V cache quantization with per-cluster parameters ([RPTQ-art] results paragraph:
+ * W4A4KV / W4A3KV / W3A3KV quantize the key and value caches alone).
+ * k, v: [B, H, S, D] of `dtype` (either may be NULL, not both); channel c = h*D + d.
+ * cluster_k / cluster_v: int32 [H*D] cluster id of each channel in its NATURAL order (the
+ * `labels` output of rptq_kmeans run on that tensor's statistics); the cache layout is kept,
+ * so no reorder applies.  scale_*, zero_*: fp32 / int32 [g].
+ *   code = clamp(rint(x / s) + z, 0, qmax), packed along D:
+ *   k_codes / v_codes uint8 [B, H, S, D*bits/8].
+ * D must be a multiple of 8 and H*D <= RPTQ_MAX_CHANNELS.
+ */
+int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t S, int D,
+                  const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
+                  const int32_t *cluster_v, const float *scale_v, const int32_t *zero_v, int g,
+                  int bits, uint8_t *k_codes, uint8_t *v_codes, rptq_stream_t stream);
+
+/*
+ * Dequantization, [Basics] section 1.3: value = s_k * (q - z_k), computed in fp32 (one
+ * rounding) and rounded to out_dtype.
+ *   layout RPTQ_LAYOUT_ROWS: codes [n0, n1*bits/8] with n0 = rows, n1 = C; cluster[j] is the
+ *          cluster of column j (col_cluster from rptq_kmeans); S and D are ignored.
+ *   layout RPTQ_LAYOUT_BHSD: codes [n0, n1, S, D*bits/8] with n0 = B, n1 = H; cluster[c] is
+ *          the cluster of channel c = h*D + d.
+ *   out: same shape with unpacked values of out_dtype.
+ */
+int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,
+                 const int32_t *cluster, const float *scale, const int32_t *zero, int g,
+                 int bits, void *out, int out_dtype, rptq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RPTQ_H_ */

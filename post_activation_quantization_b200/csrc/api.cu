@@ -1,0 +1,237 @@
+// api.cu -- the extern "C" entry points of librptq.so (declared in include/rptq.h).
+//
+// Every entry point validates its arguments on the host, then enqueues kernels on the
+// caller's stream and returns without synchronising.  Nothing here allocates device memory:
+// the only library-owned device storage is the sticky error word below.
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace rptq {
+
+// Sticky device error word (one per device that loads the library).
+__device__ int g_device_error;
+
+namespace {
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+    bool ready = false;
+    int num_sms = 0;
+    int max_smem = 0;
+    int *err = nullptr;
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Per-device facts, looked up once per device with that device current.
+int dev_info(DevInfo *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RPTQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DevInfo &d = g_dev[dev];
+    if (!d.ready) {
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return RPTQ_ERR_CUDA;
+        if (cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+            return RPTQ_ERR_CUDA;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return RPTQ_ERR_CUDA;
+        d.err = static_cast<int *>(p);
+        d.ready = true;
+    }
+    *out = d;
+    return RPTQ_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool dtype_ok(int d) { return d == RPTQ_F32 || d == RPTQ_F16 || d == RPTQ_BF16; }
+int esize(int d) { return d == RPTQ_F32 ? 4 : 2; }
+
+int cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return RPTQ_OK;
+    cudaGetLastError();  // clear a sticky launch-configuration error of this thread
+    return RPTQ_ERR_CUDA;
+}
+}  // namespace
+}  // namespace rptq
+
+using namespace rptq;
+
+extern "C" {
+
+const char *rptq_status_string(int status)
+{
+    switch (status) {
+    case RPTQ_OK: return "ok";
+    case RPTQ_ERR_INVALID_ARG: return "invalid argument";
+    case RPTQ_ERR_UNSUPPORTED: return "unsupported shape, bit width or type";
+    case RPTQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case RPTQ_ERR_CUDA: return "CUDA error";
+    case RPTQ_ERR_DEVICE: return "device-side error flag set";
+    default: return "unknown status";
+    }
+}
+
+int rptq_version(void) { return 100; }
+
+int rptq_device_error(rptq_stream_t stream, int *code)
+{
+    if (!code) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    int v = 0;
+    if (cudaMemcpy(&v, d.err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return cuda_status(cudaErrorUnknown);
+    const int zero = 0;
+    if (cudaMemcpy(d.err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return cuda_status(cudaErrorUnknown);
+    *code = v;
+    return RPTQ_OK;
+}
+
+int rptq_calib_minmax(const void *x, int dtype, int64_t T, int C, const float *gamma,
+                      const float *beta, float eps, float *ch_max, float *ch_min, int accumulate,
+                      rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (T < 0 || !ch_max || !ch_min || (accumulate != 0 && accumulate != 1)) return RPTQ_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !aligned16(x))) return RPTQ_ERR_INVALID_ARG;
+    if ((gamma == nullptr) != (beta == nullptr)) return RPTQ_ERR_INVALID_ARG;
+    if (gamma && !(eps >= 0.0f)) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    CalibArgs a{x, dtype, T, C, gamma, beta, eps, ch_max, ch_min, accumulate, d.err,
+                (cudaStream_t)stream, d.num_sms, d.max_smem};
+    return cuda_status(launch_calib(a));
+}
+
+int rptq_kv_calib_minmax(const void *kv, int dtype, int B, int H, int64_t S, int D, float *ch_max,
+                         float *ch_min, int accumulate, rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (D <= 0 || D % 8 != 0 || D > 2048 || H <= 0 || (int64_t)H * D > RPTQ_MAX_CHANNELS)
+        return RPTQ_ERR_UNSUPPORTED;
+    if (B < 0 || S < 0 || !ch_max || !ch_min || (accumulate != 0 && accumulate != 1))
+        return RPTQ_ERR_INVALID_ARG;
+    if (B > 0 && S > 0 && (!kv || !aligned16(kv))) return RPTQ_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    KvCalibArgs a{kv, dtype, B, H, S, D, ch_max, ch_min, accumulate, (cudaStream_t)stream, d.num_sms};
+    return cuda_status(launch_kv_calib(a));
+}
+
+size_t rptq_kmeans_workspace_size(int C, int g)
+{
+    if (C <= 0 || g <= 0 || g > C || C > RPTQ_MAX_CHANNELS || g > RPTQ_MAX_CLUSTERS) return 0;
+    return kmeans_ws_bytes(C, g);
+}
+
+int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iters, int bits,
+                int32_t *labels, double *centroids, int32_t *R, int32_t *col_cluster,
+                int32_t *offsets, float *scale, int32_t *zero, void *workspace,
+                size_t workspace_bytes, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (g <= 0 || g > C || g > RPTQ_MAX_CLUSTERS || iters < 0) return RPTQ_ERR_INVALID_ARG;
+    if (!ch_max || !ch_min || !labels || !centroids || !R || !col_cluster || !offsets || !scale ||
+        !zero)
+        return RPTQ_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < kmeans_ws_bytes(C, g)) return RPTQ_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RPTQ_ERR_WORKSPACE;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if (km_final_smem(C, g) + 16 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    KmArgs a{ch_max, ch_min, C, g, iters, bits, labels, centroids, R, col_cluster, offsets,
+             scale, zero, workspace, (cudaStream_t)stream, d.num_sms};
+    return cuda_status(launch_kmeans(a));
+}
+
+int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const float *gamma,
+                          const float *beta, float eps, const int32_t *R,
+                          const int32_t *col_cluster, const float *scale, const int32_t *zero,
+                          int g, int bits, uint8_t *codes, void *ln_out, rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (T < 0 || g <= 0 || g > C || !(eps >= 0.0f)) return RPTQ_ERR_INVALID_ARG;
+    if (!codes && !ln_out) return RPTQ_ERR_INVALID_ARG;
+    if (!gamma || !beta || !R || !col_cluster || !scale || !zero) return RPTQ_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !aligned16(x))) return RPTQ_ERR_INVALID_ARG;
+    if (codes && !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
+    if (ln_out && !aligned16(ln_out)) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if ((size_t)C * 5 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    LnQuantArgs a{x, dtype, T, C, gamma, beta, eps, R, col_cluster, scale, zero, g, bits, codes,
+                  ln_out, d.err, (cudaStream_t)stream, d.num_sms, d.max_smem};
+    return cuda_status(launch_ln_quant(a, 0));
+}
+
+int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t S, int D,
+                  const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
+                  const int32_t *cluster_v, const float *scale_v, const int32_t *zero_v, int g,
+                  int bits, uint8_t *k_codes, uint8_t *v_codes, rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (D <= 0 || D % 8 != 0 || D > 2048 || H <= 0 || (int64_t)H * D > RPTQ_MAX_CHANNELS)
+        return RPTQ_ERR_UNSUPPORTED;
+    if (B < 0 || S < 0 || g <= 0) return RPTQ_ERR_INVALID_ARG;
+    if (!k && !v) return RPTQ_ERR_INVALID_ARG;
+    const bool work = B > 0 && S > 0;
+    if (k && (!cluster_k || !scale_k || !zero_k || !k_codes || !aligned16(k_codes) ||
+              (work && !aligned16(k))))
+        return RPTQ_ERR_INVALID_ARG;
+    if (v && (!cluster_v || !scale_v || !zero_v || !v_codes || !aligned16(v_codes) ||
+              (work && !aligned16(v))))
+        return RPTQ_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    KvArgs a{k, v, dtype, B, H, S, D, cluster_k, scale_k, zero_k, cluster_v, scale_v, zero_v, g,
+             bits, k_codes, v_codes, d.err, (cudaStream_t)stream};
+    return cuda_status(launch_kv_quant(a));
+}
+
+int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,
+                 const int32_t *cluster, const float *scale, const int32_t *zero, int g,
+                 int bits, void *out, int out_dtype, rptq_stream_t stream)
+{
+    if (!dtype_ok(out_dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (layout != RPTQ_LAYOUT_ROWS && layout != RPTQ_LAYOUT_BHSD) return RPTQ_ERR_INVALID_ARG;
+    if (n0 < 0 || n1 <= 0 || g <= 0) return RPTQ_ERR_INVALID_ARG;
+    if (!codes || !cluster || !scale || !zero || !out) return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(codes) || !aligned16(out)) return RPTQ_ERR_INVALID_ARG;
+    if (layout == RPTQ_LAYOUT_ROWS) {
+        if (n1 % 8 != 0 || n1 > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    } else {
+        if (D <= 0 || D % 8 != 0 || D > 2048 || (int64_t)n1 * D > RPTQ_MAX_CHANNELS)
+            return RPTQ_ERR_UNSUPPORTED;
+        if (S < 0 || S > 0x7fffffffLL || n0 * n1 > 0x7fffffffLL) return RPTQ_ERR_INVALID_ARG;
+    }
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    DequantArgs a{codes, layout, n0, n1, S, D, cluster, scale, zero, g, bits, out, out_dtype,
+                  d.err, (cudaStream_t)stream, d.num_sms};
+    return cuda_status(launch_dequant(a));
+}
+
+}  // extern "C"

@@ -1,0 +1,484 @@
+// calib.cu -- calibration statistics: per-channel max and min over calibration tokens.
+//
+// RPTQ article (基于重排序的新量化方法RPTQ…), text after Fig. 2 (run calibration data through
+// the model and record each activation channel's max and min) and the Fig. 1 caption (one
+// (max, min) point per channel).  The statistic is taken on the tensor that is later
+// quantized: LayerNorm(x) for the activation path, the raw tensor for the K/V path.
+//
+// Raw mode: a CTA owns 32 chunk columns (512 bytes of every row, one 16-byte chunk per lane)
+// and a contiguous row range; its eight warps stride over the rows, keep running max/min in
+// registers (packed half2/bfloat162 max/min for 16-bit inputs, which are exact), combine
+// through shared memory and fold into the outputs with integer atomics (exact and
+// order-independent, so the result equals a sequential CPU max/min bit for bit).
+//
+// LayerNorm mode: the row pipeline of row_pipeline.cuh (bulk-copied token rows, fp32
+// LayerNorm statistics).  For every owned channel a thread keeps the running max and min of
+// the normalised value t = (x - mean) * rstd over its quads; the affine part y = t*gamma+beta is
+// monotone in t, so max y = fmaf(max t, gamma, beta) for gamma >= 0 (and the min of t for
+// gamma < 0) is the same value as taking the max of the per-token fmaf results.
+#include <algorithm>
+
+#include "launch.h"
+#include "row_pipeline.cuh"
+
+namespace rptq {
+
+__global__ void calib_init_kernel(float *ch_max, float *ch_min, int C)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c < C) {
+        ch_max[c] = -INFINITY;
+        ch_min[c] = INFINITY;
+    }
+}
+
+// ---- raw mode ------------------------------------------------------------------------------
+template <typename T> struct RawAcc;
+template <> struct RawAcc<float> {
+    float mx[4], mn[4];
+    __device__ void init()
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            mx[i] = -INFINITY;
+            mn[i] = INFINITY;
+        }
+    }
+    __device__ void add(const uint4 &v)
+    {
+        const float f[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                            __uint_as_float(v.w)};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            mx[i] = fmaxf(mx[i], f[i]);
+            mn[i] = fminf(mn[i], f[i]);
+        }
+    }
+    __device__ float get_max(int e) const { return mx[e]; }
+    __device__ float get_min(int e) const { return mn[e]; }
+};
+template <typename H2> struct RawAcc16 {
+    H2 mx[4], mn[4];
+    __device__ void add(const uint4 &v)
+    {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const H2 h = *reinterpret_cast<const H2 *>(&w[i]);
+            mx[i] = __hmax2(mx[i], h);
+            mn[i] = __hmin2(mn[i], h);
+        }
+    }
+};
+template <> struct RawAcc<__nv_bfloat16> : RawAcc16<__nv_bfloat162> {
+    __device__ void init()
+    {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(-INFINITY, -INFINITY);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(INFINITY, INFINITY);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            mx[i] = lo;
+            mn[i] = hi;
+        }
+    }
+    __device__ float get_max(int e) const
+    {
+        return (e & 1) ? __high2float(mx[e >> 1]) : __low2float(mx[e >> 1]);
+    }
+    __device__ float get_min(int e) const
+    {
+        return (e & 1) ? __high2float(mn[e >> 1]) : __low2float(mn[e >> 1]);
+    }
+};
+template <> struct RawAcc<__half> : RawAcc16<__half2> {
+    __device__ void init()
+    {
+        const __half2 lo = __floats2half2_rn(-INFINITY, -INFINITY);
+        const __half2 hi = __floats2half2_rn(INFINITY, INFINITY);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            mx[i] = lo;
+            mn[i] = hi;
+        }
+    }
+    __device__ float get_max(int e) const
+    {
+        return (e & 1) ? __high2float(mx[e >> 1]) : __low2float(mx[e >> 1]);
+    }
+    __device__ float get_min(int e) const
+    {
+        return (e & 1) ? __high2float(mn[e >> 1]) : __low2float(mn[e >> 1]);
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    calib_raw_kernel(const T *__restrict__ x, int64_t T_, int C, int64_t rows_per_cta,
+                     float *ch_max, float *ch_min)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int NCH = C / VEC;
+    const int ch = blockIdx.x * 32 + lane;
+    const int64_t r0 = (int64_t)blockIdx.y * rows_per_cta;
+    const int64_t r1 = r0 + rows_per_cta < T_ ? r0 + rows_per_cta : T_;
+    RawAcc<T> acc;
+    acc.init();
+    if (ch < NCH) {
+        const uint4 *base = reinterpret_cast<const uint4 *>(x) + ch;
+        int64_t r = r0 + warp;
+        // four independent rows in flight per thread
+        for (; r + 24 < r1; r += 32) {
+            const uint4 a = ldg_stream(base + (r + 0) * NCH);
+            const uint4 b = ldg_stream(base + (r + 8) * NCH);
+            const uint4 c = ldg_stream(base + (r + 16) * NCH);
+            const uint4 d = ldg_stream(base + (r + 24) * NCH);
+            acc.add(a);
+            acc.add(b);
+            acc.add(c);
+            acc.add(d);
+        }
+        for (; r < r1; r += 8) acc.add(ldg_stream(base + r * NCH));
+    }
+    __shared__ float smx[8][32 * 8], smn[8][32 * 8];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        smx[warp][lane * VEC + e] = acc.get_max(e);
+        smn[warp][lane * VEC + e] = acc.get_min(e);
+    }
+    __syncthreads();
+    // 32 lanes x VEC channels = 32*VEC columns; thread i < 32*VEC folds column i of the 8 warps
+    const int i = threadIdx.x;
+    if (i < 32 * VEC) {
+        const int c = (blockIdx.x * 32) * VEC + i;
+        if (c < C) {
+            float m = smx[0][i], n = smn[0][i];
+#pragma unroll
+            for (int w = 1; w < 8; ++w) {
+                m = fmaxf(m, smx[w][i]);
+                n = fminf(n, smn[w][i]);
+            }
+            if (r1 > r0) {
+                atomic_max_f32(ch_max + c, m);
+                atomic_min_f32(ch_min + c, n);
+            }
+        }
+    }
+}
+
+// ---- K/V layout: [B, H, S, D], channel c = h*D + d, statistics over the B*S tokens ------------
+// A CTA takes one (b, h) pair and a slice of S; each thread owns 8 consecutive d of one row
+// group and strides over the rows; a shared-memory fold over the row groups and integer atomics
+// finish the exact max/min.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    kv_calib_kernel(const T *__restrict__ x, int H, int64_t S, int D, int64_t s_per_cta, float *ch_max,
+                    float *ch_min)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int NLD = 8 / VEC;
+    const int bh = blockIdx.x, h = bh % H;
+    const int TPR = D / 8, RPI = blockDim.x / TPR;
+    const int tl = threadIdx.x % TPR, rr = threadIdx.x / TPR;
+    const int64_t s0 = (int64_t)blockIdx.y * s_per_cta;
+    const int64_t s1 = s0 + s_per_cta < S ? s0 + s_per_cta : S;
+    RawAcc<T> acc[NLD];
+#pragma unroll
+    for (int l = 0; l < NLD; ++l) acc[l].init();
+    if (rr < RPI) {
+        const T *base = x + (int64_t)bh * S * D + tl * 8;
+        int64_t s = s0 + rr;
+        for (; s + 3 * RPI < s1; s += 4 * RPI) {
+            uint4 a[4][NLD];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int l = 0; l < NLD; ++l) a[u][l] = ldg_stream(base + (s + u * RPI) * D + l * VEC);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int l = 0; l < NLD; ++l) acc[l].add(a[u][l]);
+        }
+        for (; s < s1; s += RPI)
+#pragma unroll
+            for (int l = 0; l < NLD; ++l) acc[l].add(ldg_stream(base + s * D + l * VEC));
+    }
+    __shared__ float kmx[256 * 8], kmn[256 * 8];
+    if (rr < RPI)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            kmx[rr * D + tl * 8 + i] = acc[i / VEC].get_max(i % VEC);
+            kmn[rr * D + tl * 8 + i] = acc[i / VEC].get_min(i % VEC);
+        }
+    __syncthreads();
+    if (s1 <= s0) return;
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        float m = kmx[d], n = kmn[d];
+        for (int r = 1; r < RPI; ++r) {
+            m = fmaxf(m, kmx[r * D + d]);
+            n = fminf(n, kmn[r * D + d]);
+        }
+        atomic_max_f32(ch_max + h * D + d, m);
+        atomic_min_f32(ch_min + h * D + d, n);
+    }
+}
+
+// ---- LayerNorm mode ------------------------------------------------------------------------
+template <typename T, int CPT>
+__global__ void __launch_bounds__(512, 1)
+    calib_ln_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                    const float *__restrict__ beta, float eps, float *ch_max, float *ch_min, int NS,
+                    int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, NT = blockDim.x;
+    const int NCH = C / VEC;
+    const uint32_t rowbytes = (uint32_t)C * sizeof(T);
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, 2 * 8 * 32 * 4);
+    float *red = reinterpret_cast<float *>(smem + L.extra_off);
+    float *red2 = red + 8 * 32;
+    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
+    pipe.start();
+    __syncthreads();
+
+    float tmax[CPT][VEC], tmin[CPT][VEC];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            tmax[k][e] = -INFINITY;
+            tmin[k][e] = INFINITY;
+        }
+    int64_t lq = 0;
+    for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
+        const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
+        uint4 xr[4][CPT];
+        pipe.load(lq, nrows, xr);
+        float rstd[4], nmr[4];
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
+#pragma unroll
+        for (int k = 0; k < CPT; ++k)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r >= nrows) break;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
+                    tmax[k][e] = fmaxf(tmax[k][e], t);
+                    tmin[k][e] = fminf(tmin[k][e], t);
+                }
+            }
+    }
+    if (lq == 0) return;  // this CTA saw no rows
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        const int ch = tid + k * NT;
+        if (ch >= NCH) continue;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const int c = ch * VEC + e;
+            const float gm = gamma[c], bt = beta[c];
+            const float hi = fmaf(gm >= 0.f ? tmax[k][e] : tmin[k][e], gm, bt);
+            const float lo = fmaf(gm >= 0.f ? tmin[k][e] : tmax[k][e], gm, bt);
+            atomic_max_f32(ch_max + c, hi);
+            atomic_min_f32(ch_min + c, lo);
+        }
+    }
+}
+
+__device__ __forceinline__ float to_float(float v) { return v; }
+__device__ __forceinline__ float to_float(__half v) { return __half2float(v); }
+__device__ __forceinline__ float to_float(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// LayerNorm mode, general shapes (any C % 8 == 0 the quad kernel cannot hold in registers):
+// one row at a time in shared memory as fp32, two-pass statistics, running max/min of the
+// normalised value per channel in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256)
+    calib_ln_simple_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                           const float *__restrict__ beta, float eps, float *ch_max, float *ch_min)
+{
+    extern __shared__ __align__(16) float csm[];
+    float *xs = csm, *tmx = csm + C, *tmn = csm + 2 * (size_t)C;
+    __shared__ float red[8 * 8];
+    const int tid = threadIdx.x, NT = blockDim.x;
+    for (int c = tid; c < C; c += NT) {
+        tmx[c] = -INFINITY;
+        tmn[c] = INFINITY;
+    }
+    for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
+        const T *xr = x + t * (int64_t)C;
+        float s = 0.f;
+        for (int c = tid; c < C; c += NT) {
+            const float v = to_float(xr[c]);
+            xs[c] = v;
+            s += v;
+        }
+        float v8[8] = {s, 0, 0, 0, 0, 0, 0, 0};
+        cta_sum8(v8, red);
+        const float mean = v8[0] / (float)C;
+        float ss = 0.f;
+        for (int c = tid; c < C; c += NT) {
+            const float d = xs[c] - mean;
+            ss = fmaf(d, d, ss);
+        }
+        float w8[8] = {ss, 0, 0, 0, 0, 0, 0, 0};
+        __syncthreads();  // red is reused
+        cta_sum8(w8, red);
+        const float rstd = rsqrtf(w8[0] / (float)C + eps);
+        const float nmr = -mean * rstd;
+        for (int c = tid; c < C; c += NT) {
+            const float tv = fmaf(xs[c], rstd, nmr);
+            tmx[c] = fmaxf(tmx[c], tv);
+            tmn[c] = fminf(tmn[c], tv);
+        }
+        __syncthreads();  // xs and red are rewritten by the next row
+    }
+    if ((int64_t)blockIdx.x >= T_) return;
+    for (int c = tid; c < C; c += NT) {
+        const float gm = gamma[c], bt = beta[c];
+        atomic_max_f32(ch_max + c, fmaf(gm >= 0.f ? tmx[c] : tmn[c], gm, bt));
+        atomic_min_f32(ch_min + c, fmaf(gm >= 0.f ? tmn[c] : tmx[c], gm, bt));
+    }
+}
+
+
+// ---- host launchers ---------------------------------------------------------------------------
+
+template <typename T>
+static cudaError_t launch_raw_t(const CalibArgs &a)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int NCH = a.C / VEC;
+    const int gx = (NCH + 31) / 32;
+    // about 8 CTAs of 256 threads per SM in total, each with at least 64 rows
+    int64_t gy = std::max<int64_t>(1, ((int64_t)a.num_sms * 8 + gx - 1) / gx);
+    gy = std::min<int64_t>(gy, std::max<int64_t>(1, a.T / 64));
+    gy = std::min<int64_t>(gy, 65535);
+    const int64_t rows_per_cta = (a.T + gy - 1) / gy;
+    gy = (a.T + rows_per_cta - 1) / rows_per_cta;
+    calib_raw_kernel<T><<<dim3(gx, (unsigned)gy), 256, 0, a.stream>>>((const T *)a.x, a.T, a.C,
+                                                                       rows_per_cta, a.ch_max, a.ch_min);
+    return cudaGetLastError();
+}
+
+template <typename T, int CPT>
+static cudaError_t launch_ln_t(const CalibArgs &a, int NT, int NS)
+{
+    const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, 2 * 8 * 32 * 4);
+    auto kern = calib_ln_kernel<T, CPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, L.total);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t quads = (a.T + 3) / 4;
+    const int64_t grid = std::min<int64_t>(quads, (int64_t)per_sm * a.num_sms);
+    kern<<<(unsigned)grid, NT, L.total, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps,
+                                                    a.ch_max, a.ch_min, NS, a.err);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_ln_simple(const CalibArgs &a)
+{
+    const size_t smem = (size_t)a.C * 12;
+    if (smem > (size_t)a.max_smem) return cudaErrorInvalidValue;
+    auto kern = calib_ln_simple_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t grid = std::min<int64_t>(a.T, (int64_t)per_sm * a.num_sms);
+    kern<<<(unsigned)grid, 256, smem, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps,
+                                                  a.ch_max, a.ch_min);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_ln_d(const CalibArgs &a)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int NCH = a.C / VEC;
+    int cpt = 0, nt = 0;
+    for (int k = 1; k <= 4; ++k) {
+        const int n = ((NCH + k - 1) / k + 31) / 32 * 32;
+        if (n <= 512) {
+            cpt = k;
+            nt = n;
+            break;
+        }
+    }
+    const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
+    int ns = 0;
+    for (int s = 8; s >= 4 && cpt; --s)
+        if (quad_smem_layout(s, rowbytes, 2 * 8 * 32 * 4).total <= (size_t)a.max_smem) {
+            ns = s;
+            break;
+        }
+    if (!cpt || !ns) return launch_ln_simple<T>(a);
+    switch (cpt) {
+    case 1: return launch_ln_t<T, 1>(a, nt, ns);
+    case 2: return launch_ln_t<T, 2>(a, nt, ns);
+    case 3: return launch_ln_t<T, 3>(a, nt, ns);
+    default: return launch_ln_t<T, 4>(a, nt, ns);
+    }
+}
+
+cudaError_t launch_calib(const CalibArgs &a)
+{
+    if (!a.accumulate) {
+        calib_init_kernel<<<(a.C + 255) / 256, 256, 0, a.stream>>>(a.ch_max, a.ch_min, a.C);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (a.T == 0) return cudaSuccess;
+    if (a.gamma) {
+        switch (a.dtype) {
+        case RPTQ_F32: return launch_ln_d<float>(a);
+        case RPTQ_F16: return launch_ln_d<__half>(a);
+        default: return launch_ln_d<__nv_bfloat16>(a);
+        }
+    }
+    switch (a.dtype) {
+    case RPTQ_F32: return launch_raw_t<float>(a);
+    case RPTQ_F16: return launch_raw_t<__half>(a);
+    default: return launch_raw_t<__nv_bfloat16>(a);
+    }
+}
+
+template <typename T>
+static cudaError_t launch_kv_calib_t(const KvCalibArgs &a)
+{
+    const int nbh = a.B * a.H;
+    int64_t gy = std::max<int64_t>(1, ((int64_t)a.num_sms * 6 + nbh - 1) / nbh);
+    gy = std::min<int64_t>(gy, std::max<int64_t>(1, a.S / 64));
+    gy = std::min<int64_t>(gy, 65535);
+    const int64_t per = (a.S + gy - 1) / gy;
+    gy = (a.S + per - 1) / per;
+    kv_calib_kernel<T><<<dim3((unsigned)nbh, (unsigned)gy), 256, 0, a.stream>>>((const T *)a.x, a.H, a.S, a.D,
+                                                                                per, a.ch_max, a.ch_min);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kv_calib(const KvCalibArgs &a)
+{
+    if (!a.accumulate) {
+        calib_init_kernel<<<(a.H * a.D + 255) / 256, 256, 0, a.stream>>>(a.ch_max, a.ch_min, a.H * a.D);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (a.B == 0 || a.S == 0) return cudaSuccess;
+    switch (a.dtype) {
+    case RPTQ_F32: return launch_kv_calib_t<float>(a);
+    case RPTQ_F16: return launch_kv_calib_t<__half>(a);
+    default: return launch_kv_calib_t<__nv_bfloat16>(a);
+    }
+}
+
+}  // namespace rptq

@@ -1,0 +1,114 @@
+// launch.h -- argument bundles and host launchers shared by api.cu and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rptq {
+
+struct LnQuantArgs {
+    const void *x;
+    int dtype;
+    int64_t T;
+    int C;
+    const float *gamma, *beta;
+    float eps;
+    const int32_t *R, *col_cluster;
+    const float *scale;
+    const int32_t *zero;
+    int g, bits;
+    uint8_t *codes;
+    void *ln_out;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+    int max_smem;
+};
+
+struct CalibArgs {
+    const void *x;
+    int dtype;
+    int64_t T;
+    int C;
+    const float *gamma, *beta;
+    float eps;
+    float *ch_max, *ch_min;
+    int accumulate;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+    int max_smem;
+};
+
+struct KvCalibArgs {
+    const void *x;
+    int dtype, B, H;
+    int64_t S;
+    int D;
+    float *ch_max, *ch_min;
+    int accumulate;
+    cudaStream_t stream;
+    int num_sms;
+};
+
+struct KvArgs {
+    const void *k, *v;
+    int dtype, B, H;
+    int64_t S;
+    int D;
+    const int32_t *ck;
+    const float *sk;
+    const int32_t *zk;
+    const int32_t *cv;
+    const float *sv;
+    const int32_t *zv;
+    int g, bits;
+    uint8_t *kq, *vq;
+    int *err;
+    cudaStream_t stream;
+};
+
+struct DequantArgs {
+    const uint8_t *codes;
+    int layout;
+    int64_t n0;
+    int n1;
+    int64_t S;
+    int D;
+    const int32_t *cluster;
+    const float *scale;
+    const int32_t *zero;
+    int g, bits;
+    void *out;
+    int out_dtype;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+};
+
+struct KmArgs {
+    const float *mx, *mn;
+    int C, g, iters, bits;
+    int32_t *labels;
+    double *cent;
+    int32_t *R, *col_cluster, *offsets;
+    float *scale;
+    int32_t *zero;
+    void *ws;
+    cudaStream_t stream;
+    int num_sms;
+};
+
+// force_simple = 1 routes codes-only calls to the general kernel (used by tests of that path)
+cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple);
+bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS);
+cudaError_t launch_calib(const CalibArgs &a);
+cudaError_t launch_kv_calib(const KvCalibArgs &a);
+cudaError_t launch_kv_quant(const KvArgs &a);
+cudaError_t launch_dequant(const DequantArgs &a);
+cudaError_t launch_kmeans(const KmArgs &a);
+size_t kmeans_ws_bytes(int C, int g);
+size_t km_final_smem(int C, int g);
+
+}  // namespace rptq

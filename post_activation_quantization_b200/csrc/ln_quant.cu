@@ -1,0 +1,371 @@
+// ln_quant.cu -- reorder-fused LayerNorm + per-cluster asymmetric quantization.
+//
+// RPTQ article (基于重排序的新量化方法RPTQ…), text after Fig. 3: the LayerNorm is changed so
+// that it emits activations already in cluster order, so no reordered copy of the activation
+// tensor is ever stored; text after Fig. 2: one scale s and zero point z per cluster.
+// Quantization-basics article, sections 1.1 (static range, clamp) and 1.3 (q = round(y/s)+z).
+//
+// Fast kernel (codes only, C % 32 == 0): see row_pipeline.cuh for the row staging.  Per quad
+// of four tokens a thread holds its chunks of x in registers, computes the LayerNorm
+// statistics, and for each of its channels c turns the four tokens' values into four codes
+//     u = sat(((x - mean) * rstd) * A_c + B_c),  code = rint(u * qmax)
+// with A_c = gamma_c / (s_k * qmax), B_c = (beta_c / s_k + z_k) / qmax, k the cluster of c
+// (this is clamp(rint(y/s_k) + z_k, 0, qmax) with y the LayerNorm output, in fp32).  The four
+// codes form one 32-bit word that is stored at the channel's STORED position R^-1(c) in a
+// shared code buffer: the reorder happens in that single shared-memory store, and because the
+// word carries four tokens a random position costs a quarter of a byte-wise scatter.  After a
+// barrier each thread reads 32 consecutive stored positions (4 tokens each), packs them into
+// 3- or 4-bit codes in registers and writes whole words of the packed rows.
+//
+// Simple kernel (any C % 8 == 0, dense LayerNorm output and/or codes): one CTA per token row,
+// the row in shared memory as fp32, a two-pass LayerNorm, a gather through R per stored
+// column, the quantizer written as clamp(rint(y / s) + z) with an IEEE divide.
+#include <algorithm>
+
+#include "launch.h"
+#include "row_pipeline.cuh"
+
+namespace rptq {
+
+// ------------------------------------------------------------------------------------------
+template <typename T, int BITS, int CPT>
+__global__ void __launch_bounds__(512, 1)
+    ln_quant_fast_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                         const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
+                         const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                         const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int NS,
+                         int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr float QMAX = (float)((1 << BITS) - 1);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, NT = blockDim.x;
+    const int NCH = C / VEC;
+    const uint32_t rowbytes = (uint32_t)C * sizeof(T);
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, (size_t)C * 4 + (size_t)C * 2 + 2 * 8 * 32 * 4);
+    uint8_t *codebuf = smem + L.extra_off;                                   // 4*C bytes
+    uint16_t *postab = reinterpret_cast<uint16_t *>(codebuf + (size_t)C * 4);  // 2*C bytes
+    float *red = reinterpret_cast<float *>(postab + C);                      // 8*32 floats
+    float *red2 = red + 8 * 32;
+
+    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
+    pipe.start();
+
+    // ---- per-channel tables: stored position (code-buffer offset) and affine coefficients
+    for (int c = tid; c < C; c += NT) postab[c] = 0;
+    __syncthreads();
+    for (int j = tid; j < C; j += NT) {
+        const int c = R[j];
+        if (c >= 0 && c < C)
+            postab[c] = (uint16_t)codebuf_offset((uint32_t)j);
+        else
+            raise_error(err, RPTQ_DEVERR_REORDER);
+    }
+    __syncthreads();
+    float pA[CPT][VEC], pB[CPT][VEC];
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        const int ch = tid + k * NT;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            pA[k][e] = 0.f;
+            pB[k][e] = 0.f;
+            if (ch < NCH) {
+                const int c = ch * VEC + e;
+                const int j = (int)codebuf_index(postab[c]);
+                int kc = col_cluster[j];
+                if (kc < 0 || kc >= g) {
+                    raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+                    kc = 0;
+                }
+                const double s = (double)scale[kc];
+                pA[k][e] = (float)((double)gamma[c] / (s * (double)QMAX));
+                pB[k][e] = (float)(((double)beta[c] / s + (double)zero[kc]) / (double)QMAX);
+            }
+        }
+    }
+
+    const uint32_t codebuf_s = smem_u32(codebuf);
+    const int64_t pitch = (int64_t)C * BITS / 8;
+    const int NU = C >> 5;  // 32-position pack units
+    int64_t lq = 0;
+    for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
+        const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
+        uint4 xr[4][CPT];
+        pipe.load(lq, nrows, xr);
+        float rstd[4], nmr[4];
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
+
+        // ---- codes of four tokens per channel -> one word at the channel's stored position
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            const int ch = tid + k * NT;
+            if (ch >= NCH) continue;
+            uint16_t pos[VEC];
+            if constexpr (VEC == 8) {
+                const uint4 p = *reinterpret_cast<const uint4 *>(postab + ch * 8);
+                const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) pos[e] = (uint16_t)(pw[e >> 1] >> (16 * (e & 1)));
+            } else {
+                const uint2 p = *reinterpret_cast<const uint2 *>(postab + ch * 4);
+                const uint32_t pw[2] = {p.x, p.y};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pos[e] = (uint16_t)(pw[e >> 1] >> (16 * (e & 1)));
+            }
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                uint32_t b[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
+                    const float u = fma_sat(t, pA[k][e], pB[k][e]);
+                    b[r] = __float_as_uint(fmaf(u, QMAX, MAGIC_RINT));
+                }
+                const uint32_t word = prmt(prmt(b[0], b[1], 0x0040), prmt(b[2], b[3], 0x0040), 0x5410);
+                asm volatile("st.shared.u32 [%0], %1;" ::"r"(codebuf_s + pos[e]), "r"(word) : "memory");
+            }
+        }
+        __syncthreads();
+
+        // ---- pack 32 stored positions x 4 tokens per thread, write whole words
+        for (int u = tid; u < NU; u += NT) {
+            uint32_t w[32];
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t slot = 8u * u + (kk ^ (u & 7));
+                const uint4 q = *reinterpret_cast<const uint4 *>(codebuf + (slot << 4));
+                w[4 * kk + 0] = q.x;
+                w[4 * kk + 1] = q.y;
+                w[4 * kk + 2] = q.z;
+                w[4 * kk + 3] = q.w;
+            }
+            uint32_t o[4][4];  // [group m][token r]
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                if constexpr (BITS == 4)
+                    pack8x4_a4(w + 8 * m, o[m]);
+                else
+                    pack8x4_a3(w + 8 * m, o[m]);
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                if (r >= nrows) break;
+                uint8_t *dst = codes + (4 * gq + r) * pitch;
+                if constexpr (BITS == 4) {
+                    *reinterpret_cast<uint4 *>(dst + 16 * (int64_t)u) =
+                        make_uint4(o[0][r], o[1][r], o[2][r], o[3][r]);
+                } else {
+                    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst + 12 * (int64_t)u);
+                    d32[0] = o[0][r] | (o[1][r] << 24);
+                    d32[1] = (o[1][r] >> 8) | (o[2][r] << 16);
+                    d32[2] = (o[2][r] >> 16) | (o[3][r] << 8);
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v)
+{
+    return __bfloat162float(v);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v)
+{
+    return __float2bfloat16_rn(v);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+    ln_quant_simple_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                           const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
+                           const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                           const int32_t *__restrict__ zero, int g, int bits, uint8_t *__restrict__ codes,
+                           T *__restrict__ ln_out, int *err)
+{
+    extern __shared__ __align__(16) uint8_t smem[];
+    float *xs = reinterpret_cast<float *>(smem);              // C floats
+    uint8_t *qb = smem + (size_t)C * 4;                        // C bytes
+    __shared__ float red[8 * 8];
+    const int tid = threadIdx.x, NT = blockDim.x;
+    const int qmax = (1 << bits) - 1;
+    const int64_t pitch = (int64_t)C * bits / 8;
+    for (int64_t t = blockIdx.x; t < T_; t += gridDim.x) {
+        const T *xr = x + t * (int64_t)C;
+        float s = 0.f;
+        for (int c = tid; c < C; c += NT) {
+            const float v = to_f32<T>(xr[c]);
+            xs[c] = v;
+            s += v;
+        }
+        float v8[8] = {s, 0, 0, 0, 0, 0, 0, 0};
+        cta_sum8(v8, red);
+        const float mean = v8[0] / (float)C;
+        float ss = 0.f;
+        for (int c = tid; c < C; c += NT) {
+            const float d = xs[c] - mean;
+            ss = fmaf(d, d, ss);
+        }
+        float w8[8] = {ss, 0, 0, 0, 0, 0, 0, 0};
+        __syncthreads();  // red is reused
+        cta_sum8(w8, red);
+        const float rstd = rsqrtf(w8[0] / (float)C + eps);
+        const float nmr = -mean * rstd;
+        for (int j = tid; j < C; j += NT) {
+            int c = R[j];
+            if (c < 0 || c >= C) {
+                raise_error(err, RPTQ_DEVERR_REORDER);
+                c = 0;
+            }
+            int k = col_cluster[j];
+            if (k < 0 || k >= g) {
+                raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+                k = 0;
+            }
+            const float y = fmaf(fmaf(xs[c], rstd, nmr), gamma[c], beta[c]);
+            if (ln_out) ln_out[t * (int64_t)C + j] = from_f32<T>(y);
+            if (codes) {
+                const float q = rintf(__fdiv_rn(y, scale[k])) + (float)zero[k];
+                qb[j] = (uint8_t)fminf(fmaxf(q, 0.f), (float)qmax);
+            }
+        }
+        __syncthreads();
+        if (codes) {
+            uint8_t *dst = codes + t * pitch;
+            for (int grp = tid; grp < C / 8; grp += NT) {
+                const uint8_t *q = qb + 8 * grp;
+                if (bits == 4) {
+                    uint32_t wv = 0;
+                    for (int i = 0; i < 8; ++i) wv |= (uint32_t)(q[i] & 15) << (4 * i);
+                    *reinterpret_cast<uint32_t *>(dst + 4 * grp) = wv;
+                } else {
+                    uint32_t wv = 0;
+                    for (int i = 0; i < 8; ++i) wv |= (uint32_t)(q[i] & 7) << (3 * i);
+                    dst[3 * grp + 0] = (uint8_t)wv;
+                    dst[3 * grp + 1] = (uint8_t)(wv >> 8);
+                    dst[3 * grp + 2] = (uint8_t)(wv >> 16);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host launchers
+// ------------------------------------------------------------------------------------------
+
+template <typename T, int BITS, int CPT>
+static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS)
+{
+    const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, (size_t)a.C * 4 + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
+    auto kern = ln_quant_fast_kernel<T, BITS, CPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, L.total);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t quads = (a.T + 3) / 4;
+    const int64_t grid = std::min<int64_t>(quads, (int64_t)per_sm * a.num_sms);
+    kern<<<(unsigned)grid, NT, L.total, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps,
+                                                    a.R, a.col_cluster, a.scale, a.zero, a.g,
+                                                    a.codes, NS, a.err);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS>
+static cudaError_t launch_fast_b(const LnQuantArgs &a, int CPT, int NT, int NS)
+{
+    switch (CPT) {
+    case 1: return launch_fast_t<T, BITS, 1>(a, NT, NS);
+    case 2: return launch_fast_t<T, BITS, 2>(a, NT, NS);
+    case 3: return launch_fast_t<T, BITS, 3>(a, NT, NS);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename T>
+static cudaError_t launch_fast_d(const LnQuantArgs &a, int CPT, int NT, int NS)
+{
+    return a.bits == 4 ? launch_fast_b<T, 4>(a, CPT, NT, NS) : launch_fast_b<T, 3>(a, CPT, NT, NS);
+}
+
+// Plan of the fast kernel for (C, dtype): threads, chunks per thread and ring depth;
+// returns false when the shape needs the simple kernel.
+bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS)
+{
+    if (C % 32 != 0) return false;
+    const int VEC = 16 / esize;
+    const int NCH = C / VEC;
+    int cpt = 0, nt = 0;
+    for (int k = 1; k <= 3; ++k) {
+        const int n = ((NCH + k - 1) / k + 31) / 32 * 32;
+        if (n <= 512) {
+            cpt = k;
+            nt = n;
+            break;
+        }
+    }
+    if (!cpt) return false;
+    const uint32_t rowbytes = (uint32_t)C * esize;
+    for (int ns = 8; ns >= 4; --ns) {
+        const QuadSmem L = quad_smem_layout(ns, rowbytes, (size_t)C * 4 + (size_t)C * 2 + 2 * 8 * 32 * 4);
+        if (L.total <= (size_t)max_smem) {
+            *CPT = cpt;
+            *NT = nt;
+            *NS = ns;
+            return true;
+        }
+    }
+    return false;
+}
+
+template <typename T>
+static cudaError_t launch_simple_t(const LnQuantArgs &a)
+{
+    const size_t smem = (size_t)a.C * 5;
+    auto kern = ln_quant_simple_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t grid = std::min<int64_t>(a.T, (int64_t)per_sm * a.num_sms);
+    kern<<<(unsigned)grid, 256, smem, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps, a.R,
+                                                  a.col_cluster, a.scale, a.zero, a.g, a.bits, a.codes,
+                                                  (T *)a.ln_out, a.err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple)
+{
+    if (a.T == 0) return cudaSuccess;
+    const int esize = a.dtype == RPTQ_F32 ? 4 : 2;
+    int CPT = 0, NT = 0, NS = 0;
+    const bool fast = !force_simple && a.ln_out == nullptr && a.codes != nullptr &&
+                      ln_quant_fast_plan(a.C, esize, a.max_smem, &CPT, &NT, &NS);
+    if (fast) {
+        switch (a.dtype) {
+        case RPTQ_F32: return launch_fast_d<float>(a, CPT, NT, NS);
+        case RPTQ_F16: return launch_fast_d<__half>(a, CPT, NT, NS);
+        default: return launch_fast_d<__nv_bfloat16>(a, CPT, NT, NS);
+        }
+    }
+    switch (a.dtype) {
+    case RPTQ_F32: return launch_simple_t<float>(a);
+    case RPTQ_F16: return launch_simple_t<__half>(a);
+    default: return launch_simple_t<__nv_bfloat16>(a);
+    }
+}
+
+}  // namespace rptq

@@ -1,0 +1,165 @@
+// row_pipeline.cuh -- token-row staging and LayerNorm statistics shared by the fused
+// LN-reorder-quant kernel and the LayerNorm-mode calibration kernel.
+//
+// A CTA owns a fixed set of 16-byte chunks of the channel axis (chunk tid + k*NT, k < CPT) and
+// walks token rows four at a time ("quads": rows 4q .. 4q+3 of its grid-stride sequence).
+// Rows arrive in a ring of NS shared-memory slots through bulk asynchronous copies (one copy
+// per row, issued by thread 0, completion on one mbarrier per slot; never multicast).  Each
+// quad is read once into registers; right after the first CTA-wide reduction the four slots
+// are refilled with the rows NS positions ahead, so the copies overlap the rest of the quad.
+//
+// LayerNorm statistics (standard LayerNorm of OPT-style models: mean and biased variance over
+// the C channels): single-pass fp32 sums of x and x^2, reduced in a fixed order; a quad with a
+// row whose squared mean exceeds its variance (where the single-pass form loses accuracy) is
+// recomputed with the two-pass form sum((x - mean)^2).
+#pragma once
+
+#include "common.cuh"
+
+namespace rptq {
+
+template <typename T, int CPT>
+struct QuadRows {
+    static constexpr int VEC = Elem<T>::VEC;
+
+    const T *x;
+    int64_t T_;
+    int C, NCH, NS;
+    uint32_t rowbytes;
+    uint8_t *ring;      // NS * rowbytes, 128-byte aligned
+    uint32_t bar0;      // shared address of NS consecutive 8-byte mbarriers
+    int *err;
+
+    __device__ __forceinline__ int64_t row_of(int64_t local) const
+    {
+        // local row i -> quad i/4 of this CTA's grid-stride sequence, row i%4 of that quad
+        const int64_t q = (int64_t)blockIdx.x + (local >> 2) * (int64_t)gridDim.x;
+        return 4 * q + (local & 3);
+    }
+    // thread 0 only
+    __device__ __forceinline__ void issue(int64_t local) const
+    {
+        const int64_t row = row_of(local);
+        if (row >= T_) return;
+        const int slot = (int)(local % NS);
+        const uint32_t bar = bar0 + 8u * slot;
+        mbar_expect_tx(bar, rowbytes);
+        bulk_g2s(smem_u32(ring + (size_t)slot * rowbytes), x + row * (int64_t)C, rowbytes, bar);
+    }
+    // thread 0: barriers + first NS rows.  Caller must __syncthreads() before any wait.
+    __device__ __forceinline__ void start() const
+    {
+        if (threadIdx.x == 0) {
+            for (int s = 0; s < NS; ++s) mbar_init(bar0 + 8u * s, 1);
+            fence_mbar_init();
+            for (int s = 0; s < NS; ++s) issue(s);
+        }
+    }
+    // Wait for quad lq (rows < nrows valid) and copy this thread's chunks into registers.
+    __device__ __forceinline__ void load(int64_t lq, int nrows, uint4 (&xr)[4][CPT]) const
+    {
+        const int tid = threadIdx.x, NT = blockDim.x;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int64_t local = 4 * lq + r;
+            const int slot = (int)(local % NS);
+            if (r < nrows) mbar_wait_bounded(bar0 + 8u * slot, (uint32_t)((local / NS) & 1), err);
+            const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)slot * rowbytes);
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) {
+                const int ch = tid + k * NT;
+                xr[r][k] = (r < nrows && ch < NCH) ? src[ch] : make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    // thread 0 after the first reduction of quad lq: refill its four slots.
+    __device__ __forceinline__ void refill(int64_t lq) const
+    {
+        if (threadIdx.x == 0) {
+            fence_proxy_async_smem();
+#pragma unroll
+            for (int r = 0; r < 4; ++r) issue(4 * lq + NS + r);
+        }
+    }
+};
+
+// LayerNorm statistics of the four rows in xr.  Returns rstd[r] and nmr[r] = -mean*rstd so that
+// the normalised value is fmaf(x, rstd, nmr).  `red`, `red2`: 8*(NT/32) floats each.
+// Calls refill() between its first barrier and any later one.
+template <typename T, int CPT, typename Pipe>
+__device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int NCH, float eps,
+                                           float *red, float *red2, const Pipe &pipe, int64_t lq,
+                                           float (&rstd)[4], float (&nmr)[4])
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int tid = threadIdx.x, NT = blockDim.x;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        if (tid + k * NT < NCH) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const float xv = Elem<T>::get(xr[r][k], e);
+                    v[r] += xv;
+                    v[4 + r] = fmaf(xv, xv, v[4 + r]);
+                }
+        }
+    }
+    cta_sum8(v, red);  // every thread is past its reads of this quad's ring slots
+    pipe.refill(lq);
+    const float invC = 1.0f / (float)C;
+    float mean[4], var[4];
+    bool ill = false;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        mean[r] = v[r] * invC;
+        var[r] = v[4 + r] * invC - mean[r] * mean[r];
+        ill |= !(mean[r] * mean[r] <= var[r]);
+    }
+    if (ill) {  // same decision in every thread (identical reduced values)
+        float w[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) w[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            if (tid + k * NT < NCH) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        const float d = Elem<T>::get(xr[r][k], e) - mean[r];
+                        w[r] = fmaf(d, d, w[r]);
+                    }
+            }
+        }
+        cta_sum8(w, red2);
+#pragma unroll
+        for (int r = 0; r < 4; ++r) var[r] = w[r] * invC;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        rstd[r] = rsqrtf(fmaxf(var[r], 0.f) + eps);
+        nmr[r] = -mean[r] * rstd[r];
+    }
+}
+
+// Dynamic shared memory of a quad pipeline: ring + extra bytes, with 128-byte alignment.
+struct QuadSmem {
+    size_t ring_off, extra_off, bar_off, total;
+};
+__host__ __device__ inline QuadSmem quad_smem_layout(int NS, uint32_t rowbytes, size_t extra)
+{
+    QuadSmem s;
+    auto up = [](size_t v) { return (v + 127) & ~(size_t)127; };
+    s.ring_off = 0;
+    s.extra_off = up((size_t)NS * rowbytes);
+    s.bar_off = up(s.extra_off + extra);
+    s.total = s.bar_off + 8 * (size_t)NS;
+    return s;
+}
+
+}  // namespace rptq

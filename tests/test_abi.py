@@ -1,0 +1,84 @@
+"""The C-ABI library loads on a machine without a GPU and exports every entry point that
+include/rptq.h declares; host-side argument validation needs no GPU either."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "rptq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rptq_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def rlib():
+    from post_activation_quantization_b200 import build, rptq
+    build.build()
+    return rptq.lib()
+
+
+def test_every_declared_symbol_is_exported(rlib):
+    from post_activation_quantization_b200 import rptq
+    names = _declared_functions()
+    assert "rptq_ln_reorder_quant" in names and len(names) >= 9
+    for n in names:
+        assert hasattr(rlib, n), n
+    assert set(names) == set(rptq.SIGNATURES)
+
+
+def test_status_strings_and_version(rlib):
+    assert rlib.rptq_version() == 100
+    assert rlib.rptq_status_string(0) == b"ok"
+    for st in (-1, -2, -3, -4, -5):
+        assert rlib.rptq_status_string(st) != b"unknown status"
+
+
+def test_workspace_size_rules(rlib):
+    assert rlib.rptq_kmeans_workspace_size(12288, 64) > 0
+    assert rlib.rptq_kmeans_workspace_size(8, 9) == 0      # g > C
+    assert rlib.rptq_kmeans_workspace_size(0, 1) == 0
+    assert rlib.rptq_kmeans_workspace_size(20000, 8) == 0  # C over the maximum
+
+
+def test_host_validation_rejects_before_any_launch(rlib):
+    """Invalid calls are refused on the host (no CUDA context is touched)."""
+    P = ctypes.c_void_p
+    fake = P(16 * 1024)  # never dereferenced: validation fails first
+    # bits not in {3, 4}
+    assert rlib.rptq_ln_reorder_quant(fake, 2, 4, 64, fake, fake, 1e-5, fake, fake, fake, fake, 8, 5,
+                                      fake, None, None) == -2
+    # C not a multiple of 8
+    assert rlib.rptq_ln_reorder_quant(fake, 2, 4, 60, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
+                                      fake, None, None) == -2
+    # neither codes nor ln_out
+    assert rlib.rptq_ln_reorder_quant(fake, 2, 4, 64, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
+                                      None, None, None) == -1
+    # misaligned x
+    assert rlib.rptq_ln_reorder_quant(P(16 * 1024 + 2), 2, 4, 64, fake, fake, 1e-5, fake, fake, fake,
+                                      fake, 8, 3, fake, None, None) == -1
+    # unsupported dtype
+    assert rlib.rptq_calib_minmax(fake, 7, 4, 64, None, None, 1e-5, fake, fake, 0, None) == -2
+    # gamma without beta
+    assert rlib.rptq_calib_minmax(fake, 2, 4, 64, fake, None, 1e-5, fake, fake, 0, None) == -1
+    # kmeans: g > C, bad bits, missing workspace
+    assert rlib.rptq_kmeans(fake, fake, 8, 9, 1, 3, fake, fake, fake, fake, fake, fake, fake, fake,
+                            1 << 20, None) == -1
+    assert rlib.rptq_kmeans(fake, fake, 64, 8, 1, 2, fake, fake, fake, fake, fake, fake, fake, fake,
+                            1 << 20, None) == -2
+    assert rlib.rptq_kmeans(fake, fake, 64, 8, 1, 3, fake, fake, fake, fake, fake, fake, fake, None,
+                            1 << 20, None) == -3
+    assert rlib.rptq_kmeans(fake, fake, 64, 8, 1, 3, fake, fake, fake, fake, fake, fake, fake, fake,
+                            16, None) == -3
+    # kv: D not a multiple of 8, neither k nor v
+    assert rlib.rptq_kv_quant(fake, fake, 1, 1, 2, 4, 12, fake, fake, fake, fake, fake, fake, 4, 3,
+                              fake, fake, None) == -2
+    assert rlib.rptq_kv_quant(None, None, 1, 1, 2, 4, 16, fake, fake, fake, fake, fake, fake, 4, 3,
+                              fake, fake, None) == -1
+    # dequant: bad layout
+    assert rlib.rptq_dequant(fake, 5, 4, 64, 0, 0, fake, fake, fake, 8, 3, fake, 0, None) == -1
+    assert rlib.rptq_device_error(None, None) == -1
