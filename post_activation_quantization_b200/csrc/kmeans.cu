@@ -357,3 +357,93 @@ cudaError_t launch_kmeans(const KmArgs &a)
 }
 
 }  // namespace rptq
+
+// ==========================================================================================
+// Allocation-free KMeans entry point.
+//
+// Some callers cannot allocate device memory once they are running: a plugin inside a host
+// application that owns every byte of GPU memory through its own pool, or a serving loop that
+// forbids cudaMalloc / cudaFree after start-up because they can synchronise the device and
+// stall other work.  rptq_kmeans_noalloc gives them the KMeans + reorder + (s, z) call without
+// a caller-provided workspace: its scratch is the fixed array below, which every GPU that
+// loads this library holds until the process exits.
+//
+// Limits and sharing rules (also stated in include/rptq.h):
+//   - the scratch holds RPTQ_KMEANS_NOALLOC_SCRATCH_BYTES (1 MiB, include/rptq.h); a (C, g) whose workspace
+//     would be larger is refused with RPTQ_ERR_UNSUPPORTED (every C <= 16384 fits for g <= 512);
+//   - all calls on one device share the array and it keeps the previous call's contents; the
+//     launch sequence clears the parts that must start at zero (rank counters, control words)
+//     and overwrites the rest before reading it, so stale contents never leak into results;
+//   - two calls whose kernels overlap on the GPU (different streams, no ordering) race on the
+//     array and may give wrong results: order them on one stream or with events;
+//   - the first call on a device looks up the array's device address and the device's
+//     properties with that device current; make that first call before any stream capture.
+// ==========================================================================================
+#include <mutex>
+
+static __device__ __align__(256) unsigned char g_kmeans_scratch[RPTQ_KMEANS_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+struct NoAllocDev {
+    bool ready = false;
+    void *scratch = nullptr;  // device address of g_kmeans_scratch on this device
+    int num_sms = 0;
+    int max_smem = 0;
+};
+NoAllocDev g_noalloc_dev[64];
+std::mutex g_noalloc_mu;
+
+// One-time set-up per device, run with that device current.
+int noalloc_setup(NoAllocDev *out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RPTQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    NoAllocDev &d = g_noalloc_dev[dev];
+    if (!d.ready) {
+        void *p = nullptr;
+        // In host code g_kmeans_scratch names a host-side stand-in; this returns the address
+        // of the array in the current device's memory, the only address a kernel may be given.
+        if (cudaGetSymbolAddress(&p, g_kmeans_scratch) != cudaSuccess) {
+            cudaGetLastError();
+            return RPTQ_ERR_CUDA;
+        }
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess) {
+            cudaGetLastError();
+            return RPTQ_ERR_CUDA;
+        }
+        d.scratch = p;
+        d.ready = true;
+    }
+    *out = d;
+    return RPTQ_OK;
+}
+}  // namespace
+
+extern "C" int rptq_kmeans_noalloc(const float *ch_max, const float *ch_min, int C, int g,
+                                   int iters, int bits, int32_t *labels, double *centroids,
+                                   int32_t *R, int32_t *col_cluster, int32_t *offsets,
+                                   float *scale, int32_t *zero, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (g <= 0 || g > C || g > RPTQ_MAX_CLUSTERS || iters < 0) return RPTQ_ERR_INVALID_ARG;
+    if (!ch_max || !ch_min || !labels || !centroids || !R || !col_cluster || !offsets || !scale ||
+        !zero)
+        return RPTQ_ERR_INVALID_ARG;
+    if (rptq::kmeans_ws_bytes(C, g) > RPTQ_KMEANS_NOALLOC_SCRATCH_BYTES) return RPTQ_ERR_UNSUPPORTED;
+    NoAllocDev d;
+    const int st = noalloc_setup(&d);
+    if (st != RPTQ_OK) return st;
+    if (rptq::km_final_smem(C, g) + 16 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    rptq::KmArgs a{ch_max, ch_min, C, g, iters, bits, labels, centroids, R, col_cluster, offsets,
+                   scale, zero, d.scratch, (cudaStream_t)stream, d.num_sms};
+    const cudaError_t e = rptq::launch_kmeans(a);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return RPTQ_ERR_CUDA;
+    }
+    return RPTQ_OK;
+}

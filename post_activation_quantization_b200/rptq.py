@@ -45,6 +45,7 @@ SIGNATURES = {
     "rptq_kv_calib_minmax": (_I, [_P, _I, _I, _I, _I64, _I, _P, _P, _I, _P]),
     "rptq_kmeans_workspace_size": (_SZ, [_I, _I]),
     "rptq_kmeans": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "rptq_kmeans_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "rptq_ln_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_quant": (_I, [_P, _P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
@@ -165,6 +166,19 @@ def rptq_kmeans(ch_max: torch.Tensor, ch_min: torch.Tensor, g: int, iters: int, 
                            _ptr(out["offsets"]), _ptr(out["scale"]), _ptr(out["zero"]),
                            _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "rptq_kmeans")
+    return out
+
+
+def rptq_kmeans_noalloc(ch_max: torch.Tensor, ch_min: torch.Tensor, g: int, iters: int, bits: int,
+                        out: dict, stream=None) -> dict:
+    """rptq_kmeans without a workspace (the library's fixed device scratch is used); `out` holds
+    caller-allocated output tensors with the keys rptq_kmeans returns."""
+    C = ch_max.numel()
+    st = lib().rptq_kmeans_noalloc(_ptr(ch_max), _ptr(ch_min), C, g, iters, bits, _ptr(out["labels"]),
+                                   _ptr(out["centroids"]), _ptr(out["R"]), _ptr(out["col_cluster"]),
+                                   _ptr(out["offsets"]), _ptr(out["scale"]), _ptr(out["zero"]),
+                                   _stream(stream))
+    _check(st, "rptq_kmeans_noalloc")
     return out
 
 
