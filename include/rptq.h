@@ -70,7 +70,7 @@ typedef struct CUstream_st *rptq_stream_t;
 /* Largest channel count C (and H*D) any entry point accepts. */
 #define RPTQ_MAX_CHANNELS 16384
 /* Largest cluster count g. */
-#define RPTQ_MAX_CLUSTERS 1024
+#define RPTQ_MAX_CLUSTERS 512
 
 /* Human-readable text of a status code (static storage, never NULL). */
 const char *rptq_status_string(int status);
@@ -161,7 +161,7 @@ int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iter
  * memory while running (a plugin whose host owns all GPU memory, a serving loop that forbids
  * cudaMalloc / cudaFree after start-up); the call itself allocates nothing.
  *   - (C, g) needing more than 1 MiB of scratch is refused with RPTQ_ERR_UNSUPPORTED (every
- *     C <= RPTQ_MAX_CHANNELS fits for g <= 512);
+ *     C <= RPTQ_MAX_CHANNELS fits for g <= 256);
  *   - all calls on a device share the scratch: calls whose kernels may overlap on the GPU
  *     race and can give wrong results, so order them (one stream, or events);
  *   - the scratch keeps the last call's contents; each call re-initialises what it reads;

@@ -47,6 +47,15 @@ int dev_info(DevInfo *out)
     return RPTQ_OK;
 }
 
+}  // namespace
+
+int *device_error_word()
+{
+    DevInfo d;
+    return dev_info(&d) == RPTQ_OK ? d.err : nullptr;
+}
+
+namespace {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool dtype_ok(int d) { return d == RPTQ_F32 || d == RPTQ_F16 || d == RPTQ_BF16; }
 int esize(int d) { return d == RPTQ_F32 ? 4 : 2; }
@@ -153,9 +162,9 @@ int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iter
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
-    if (km_final_smem(C, g) + 16 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    if (km_final_batch(C, g, d.max_smem) < 1) return RPTQ_ERR_UNSUPPORTED;
     KmArgs a{ch_max, ch_min, C, g, iters, bits, labels, centroids, R, col_cluster, offsets,
-             scale, zero, workspace, (cudaStream_t)stream, d.num_sms};
+             scale, zero, workspace, (cudaStream_t)stream, d.num_sms, d.max_smem, d.err};
     return cuda_status(launch_kmeans(a));
 }
 

@@ -81,6 +81,65 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
     return d;
 }
 
+// ---- two fp32 lanes in one 64-bit register pair (sm_100 packed fp32 arithmetic) ---------
+// fma/add/mul on .f32x2 round each lane exactly like the scalar instruction (IEEE, nearest).
+struct f32x2 {
+    unsigned long long v;
+};
+__device__ __forceinline__ f32x2 mk2(float lo, float hi)
+{
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float lo2(f32x2 a)
+{
+    float l, h;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(l), "=f"(h) : "l"(a.v));
+    return l;
+}
+__device__ __forceinline__ float hi2(f32x2 a)
+{
+    float l, h;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(l), "=f"(h) : "l"(a.v));
+    return h;
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
+{
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+    return r;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
+{
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
+{
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+    return r;
+}
+// Elements 2p, 2p+1 of a 16-byte chunk as one fp32 pair (exact widening).
+template <typename T> __device__ __forceinline__ f32x2 pair_of(const uint4 &v, int p);
+template <> __device__ __forceinline__ f32x2 pair_of<__nv_bfloat16>(const uint4 &v, int p)
+{
+    const uint32_t w = (&v.x)[p];
+    return mk2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <> __device__ __forceinline__ f32x2 pair_of<__half>(const uint4 &v, int p)
+{
+    const uint32_t w = (&v.x)[p];
+    const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    return mk2(f.x, f.y);
+}
+template <> __device__ __forceinline__ f32x2 pair_of<float>(const uint4 &v, int p)
+{
+    return mk2(__uint_as_float((&v.x)[2 * p]), __uint_as_float((&v.x)[2 * p + 1]));
+}
+
 // Order-independent float max/min through integer atomics (exact; finite inputs).
 __device__ __forceinline__ void atomic_max_f32(float *addr, float v)
 {
@@ -129,13 +188,15 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+// One suspending try: the thread sleeps in hardware until the phase completes or a system
+// time limit passes (no busy polling that would take issue slots from working warps).
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(1000000u)
         : "memory");
     return ok != 0;
 }
@@ -149,16 +210,13 @@ __device__ __forceinline__ uint64_t global_ns()
 // RPTQ_DEVERR_TIMEOUT and returns false (the caller then uses whatever is in the buffer).
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int *err)
 {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = global_ns();
-    for (uint32_t spin = 1;; ++spin) {
-        if (mbar_test(bar, parity)) return true;
-        if ((spin & 63u) == 0) {
-            if (global_ns() - t0 > 2000000000ull) {
-                raise_error(err, RPTQ_DEVERR_TIMEOUT);
-                return false;
-            }
-            __nanosleep(64);
+    for (;;) {
+        if (mbar_try(bar, parity)) return true;
+        if (global_ns() - t0 > 2000000000ull) {
+            raise_error(err, RPTQ_DEVERR_TIMEOUT);
+            return false;
         }
     }
 }

@@ -138,25 +138,33 @@ __global__ void __launch_bounds__(256, 2)
     const uint8_t *cbase = codes + (int64_t)tl * (DPT * BITS / 8);
     T *obase = out + p0;
     if (exact) {
-        int64_t r = r0;
-        uint32_t grp[NGRP];
-        if (r < r1) load_groups<BITS, DPT>(cbase + r * pitch, grp);
-        for (; r < r1; r += rstep) {
-            uint32_t nxt[NGRP];
-            const int64_t rn = r + rstep;
-            if (rn < r1) load_groups<BITS, DPT>(cbase + rn * pitch, nxt);  // next row in flight
+        constexpr int U = 4;  // rows of codes in flight per thread
+        for (int64_t rb = r0; rb < r1; rb += (int64_t)U * rstep) {
+            uint32_t grp[U][NGRP];
 #pragma unroll
-            for (int c8 = 0; c8 < NGRP; ++c8) {
-                float v[8];
+            for (int u = 0; u < U; ++u) {
+                const int64_t r = rb + (int64_t)u * rstep;
+                if (r < r1)
+                    load_groups<BITS, DPT>(cbase + r * pitch, grp[u]);
+                else
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t q = (grp[c8] >> (BITS * i)) & QMASK;
-                    v[i] = sc[8 * c8 + i] * (__uint_as_float(0x4B000000u | q) - zf[8 * c8 + i]);
-                }
-                Store<T>::template put<8>(obase + r * width + 8 * c8, v);
+                    for (int i = 0; i < NGRP; ++i) grp[u][i] = 0;
             }
 #pragma unroll
-            for (int i = 0; i < NGRP; ++i) grp[i] = nxt[i];
+            for (int u = 0; u < U; ++u) {
+                const int64_t r = rb + (int64_t)u * rstep;
+                if (r >= r1) break;
+#pragma unroll
+                for (int c8 = 0; c8 < NGRP; ++c8) {
+                    float v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const uint32_t q = (grp[u][c8] >> (BITS * i)) & QMASK;
+                        v[i] = sc[8 * c8 + i] * (__uint_as_float(0x4B000000u | q) - zf[8 * c8 + i]);
+                    }
+                    Store<T>::template put<8>(obase + r * width + 8 * c8, v);
+                }
+            }
         }
     } else {  // some |z| too large for the exact float form: integer subtraction, then convert
         for (int64_t r = r0; r < r1; r += rstep) {

@@ -29,7 +29,7 @@ __device__ __forceinline__ float div_rn(float x, float s, float r)
     return fmaf(res, r, q0);
 }
 
-template <typename T, int BITS>
+template <typename T, int BITS, int DPT>
 __global__ void __launch_bounds__(256)
     kv_quant_kernel(const T *__restrict__ k, const T *__restrict__ v, int H, int64_t S, int D,
                     const int32_t *__restrict__ ck, const float *__restrict__ sk,
@@ -38,9 +38,11 @@ __global__ void __launch_bounds__(256)
                     uint8_t *__restrict__ kq, uint8_t *__restrict__ vq, int *err)
 {
     constexpr int VEC = Elem<T>::VEC;
-    constexpr int NLD = 8 / VEC;  // 16-byte loads per 8 channels
+    constexpr int NLD = DPT / VEC;  // 16-byte loads per row and thread
+    constexpr int NG = DPT / 8;     // packed 8-code groups per row and thread
     constexpr int QMAX = (1 << BITS) - 1;
     constexpr uint32_t MAGIC_BITS = 0x4B400000u;
+    constexpr int U = 4;            // rows whose loads are in flight together
     const bool is_v = blockIdx.y == 1;
     const T *src = is_v ? v : k;
     uint8_t *dst = is_v ? vq : kq;
@@ -51,118 +53,124 @@ __global__ void __launch_bounds__(256)
 
     const int bh = blockIdx.x;  // b*H + h
     const int h = bh % H;
-    const int TPR = D / 8;      // threads per row, 8 channels each
+    const int TPR = D / DPT;    // threads per row
     const int RPI = blockDim.x / TPR;
     const int tl = threadIdx.x % TPR, rr = threadIdx.x / TPR;
-    const bool active = rr < RPI;
-    const int d0 = tl * 8;
+    if (rr >= RPI) return;
+    const int d0 = tl * DPT;
 
-    // per-channel divisor, its reciprocal and the code-domain clamp [-z, qmax - z]
-    float s8[8], r8[8], lo8[8], hi8[8];
-    uint32_t bias = 0;  // sum_i (MAGIC_BITS - z_i) << (BITS*i): removes the rounding constant
+    // per-channel divisor s (negated), its reciprocal r, and the code-domain clamp [-z, qmax - z]
+    f32x2 ns2[DPT / 2], r2[DPT / 2];
+    float lo_[DPT], hi_[DPT];
+    uint32_t bias[NG];  // sum_i (MAGIC_BITS - z_i) << (BITS*i): removes the rounding constant
     bool small_z = true;  // |z| < 2^21 keeps q + 1.5*2^23 inside one binade (exact rounding)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        int kc = active ? cl[h * D + d0 + i] : 0;
-        if (kc < 0 || kc >= g) {
-            raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
-            kc = 0;
+    for (int gi = 0; gi < NG; ++gi) bias[gi] = 0;
+#pragma unroll
+    for (int i = 0; i < DPT; i += 2) {
+        float sv2[2], rv2[2];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            int kc = cl[h * D + d0 + i + h2];
+            if (kc < 0 || kc >= g) {
+                raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+                kc = 0;
+            }
+            sv2[h2] = sc[kc];
+            rv2[h2] = __frcp_rn(sv2[h2]);
+            const int z = zp[kc];
+            lo_[i + h2] = (float)(-z);
+            hi_[i + h2] = (float)(QMAX - z);
+            bias[(i + h2) / 8] += (MAGIC_BITS - (uint32_t)z) << (BITS * ((i + h2) % 8));
+            small_z &= (z > -(1 << 21)) && (z < (1 << 21));
         }
-        s8[i] = sc[kc];
-        r8[i] = __frcp_rn(s8[i]);
-        const int z = zp[kc];
-        lo8[i] = (float)(-z);
-        hi8[i] = (float)(QMAX - z);
-        bias += (MAGIC_BITS - (uint32_t)z) << (BITS * i);
-        small_z &= (z > -(1 << 21)) && (z < (1 << 21));
+        ns2[i / 2] = mk2(-sv2[0], -sv2[1]);
+        r2[i / 2] = mk2(rv2[0], rv2[1]);
     }
+    const f32x2 magic2 = mk2(MAGIC_RINT, MAGIC_RINT);
     const int64_t pitch = (int64_t)D * BITS / 8;
     const T *base = src + (int64_t)bh * S * D + d0;
-    uint8_t *obase = dst + (int64_t)bh * S * pitch;
-    // A warp covers whole consecutive rows (or a run of one row) when TPR divides 32 or 32
-    // divides TPR: its 3-byte groups then form one contiguous run that lanes store as words.
-    const bool contiguous = (32 % TPR == 0) || (TPR % 32 == 0);
-    const int lane = threadIdx.x & 31;
+    uint8_t *obase = dst + (int64_t)bh * S * pitch + (int64_t)tl * (DPT * BITS / 8);
 
-    const int64_t iters = active ? (S - rr + RPI - 1) / RPI : 0;
-    const int64_t trips = (S + RPI - 1) / RPI;  // the same for every lane (shuffles below)
-    constexpr int U = 4;                         // rows whose loads are in flight together
-    for (int64_t it0 = 0; it0 < trips; it0 += U) {
+    for (int64_t s0 = rr; s0 < S; s0 += (int64_t)U * RPI) {
         uint4 xb[U][NLD];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t s_row = rr + (it0 + u) * RPI;
-            const bool valid = it0 + u < iters && s_row < S;
+            const int64_t row = s0 + (int64_t)u * RPI;
 #pragma unroll
             for (int l = 0; l < NLD; ++l)
-                xb[u][l] = valid ? ldg_stream(base + s_row * D + l * VEC) : make_uint4(0, 0, 0, 0);
+                xb[u][l] = row < S ? ldg_stream(base + row * D + l * VEC) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-        if (it0 + u >= trips) break;
-        const int64_t it = it0 + u;
-        const int64_t s_row = rr + it * RPI;
-        const bool valid = it < iters && s_row < S;
-        const uint4 *xv = xb[u];
-        uint32_t grp;  // codes of the 8 channels, packed
-        if (small_z) {
-            uint32_t acc = 0;
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = s0 + (int64_t)u * RPI;
+            if (row >= S) break;
+            uint32_t grp[NG];
+            if (small_z) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float xf = Elem<T>::get(xv[i / VEC], i % VEC);
-                float q = div_rn(xf, s8[i], r8[i]);
-                q = fminf(fmaxf(q, lo8[i]), hi8[i]);  // clamp(rint(q) + z) == rint(clamp(q)) + z
-                acc += __float_as_uint(q + MAGIC_RINT) << (BITS * i);
-            }
-            grp = acc - bias;
-        } else {  // a huge zero point: integer rounding and clamping
-            grp = 0;
-            for (int i = 0; i < 8; ++i) {
-                const float xf = Elem<T>::get(xv[i / VEC], i % VEC);
-                const float q = rintf(div_rn(xf, s8[i], r8[i]));
-                const float c = fminf(fmaxf(q, lo8[i]), hi8[i]) - lo8[i];
-                grp |= (uint32_t)c << (BITS * i);
-            }
-        }
-        uint8_t *o = obase + s_row * pitch + (int64_t)tl * BITS;  // this thread's group
-        if constexpr (BITS == 4) {
-            if (valid) *reinterpret_cast<uint32_t *>(o) = grp;
-        } else if (contiguous) {
-            // The warp's groups form one run starting at lane 0's group; its valid lanes are a
-            // prefix of the warp (rows beyond S come last).  Lane w < 24 writes bytes [4w, 4w+4)
-            // of the run: a whole word when the run start is 4-byte aligned and the word is
-            // complete, single bytes otherwise.
-            const unsigned long long a0 = __shfl_sync(FULL, reinterpret_cast<unsigned long long>(o), 0);
-            const int nbytes = 3 * __popc(__ballot_sync(FULL, valid));
-            const int w = lane, a = (4 * w) / 3, off = (4 * w) % 3;
-            const uint32_t ga = __shfl_sync(FULL, grp, a < 32 ? a : 31);
-            const uint32_t gb = __shfl_sync(FULL, grp, a + 1 < 32 ? a + 1 : 31);
-            const uint32_t lo = (ga & 0xffffffu) | (gb << 24), hi = (gb & 0xffffffu) >> 8;
-            const uint32_t word = __funnelshift_r(lo, hi, 8 * off);
-            uint8_t *run = reinterpret_cast<uint8_t *>(a0);
-            if (w < 24 && 4 * w < nbytes) {
-                if ((a0 & 3ull) == 0 && 4 * w + 4 <= nbytes) {
-                    *reinterpret_cast<uint32_t *>(run + 4 * w) = word;
-                } else {
-                    for (int b = 0; b < 4 && 4 * w + b < nbytes; ++b) run[4 * w + b] = (uint8_t)(word >> (8 * b));
+                for (int gi = 0; gi < NG; ++gi) {
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        const int i = gi * 8 + j;
+                        // correctly rounded x/s for two channels (reciprocal + one correction)
+                        const f32x2 x2 = pair_of<T>(xb[u][i / VEC], (i % VEC) / 2);
+                        const f32x2 q0 = mul2(x2, r2[i / 2]);
+                        const f32x2 q1 = fma2(fma2(q0, ns2[i / 2], x2), r2[i / 2], q0);
+                        // clamp(rint(q) + z) == rint(clamp(q, -z, qmax - z)) + z
+                        const f32x2 qc = mk2(fminf(fmaxf(lo2(q1), lo_[i]), hi_[i]),
+                                             fminf(fmaxf(hi2(q1), lo_[i + 1]), hi_[i + 1]));
+                        const f32x2 b2 = add2(qc, magic2);
+                        acc += __float_as_uint(lo2(b2)) << (BITS * j);
+                        acc += __float_as_uint(hi2(b2)) << (BITS * (j + 1));
+                    }
+                    grp[gi] = acc - bias[gi];
+                }
+            } else {  // a huge zero point: integer rounding and clamping
+#pragma unroll
+                for (int gi = 0; gi < NG; ++gi) {
+                    uint32_t acc = 0;
+                    for (int j = 0; j < 8; ++j) {
+                        const int i = gi * 8 + j;
+                        const float xf = Elem<T>::get(xb[u][i / VEC], i % VEC);
+                        const float si = (i & 1) ? -hi2(ns2[i / 2]) : -lo2(ns2[i / 2]);
+                        const float ri = (i & 1) ? hi2(r2[i / 2]) : lo2(r2[i / 2]);
+                        const float q = rintf(div_rn(xf, si, ri));
+                        const float c = fminf(fmaxf(q, lo_[i]), hi_[i]) - lo_[i];
+                        acc |= (uint32_t)c << (BITS * j);
+                    }
+                    grp[gi] = acc;
                 }
             }
-        } else if (valid) {
-            o[0] = (uint8_t)grp;
-            o[1] = (uint8_t)(grp >> 8);
-            o[2] = (uint8_t)(grp >> 16);
+            uint8_t *o = obase + row * pitch;
+            if constexpr (BITS == 4) {
+                if constexpr (NG == 2)
+                    *reinterpret_cast<uint2 *>(o) = make_uint2(grp[0], grp[1]);
+                else
+                    *reinterpret_cast<uint32_t *>(o) = grp[0];
+            } else {
+                if constexpr (NG == 2) {  // 6 bytes at an even offset: three 2-byte stores
+                    uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
+                    o16[0] = (uint16_t)grp[0];
+                    o16[1] = (uint16_t)((grp[0] >> 16) | (grp[1] << 8));
+                    o16[2] = (uint16_t)(grp[1] >> 8);
+                } else {
+                    o[0] = (uint8_t)grp[0];
+                    o[1] = (uint8_t)(grp[0] >> 8);
+                    o[2] = (uint8_t)(grp[0] >> 16);
+                }
+            }
         }
-    }
     }
 }
 
-template <typename T, int BITS>
-static cudaError_t launch_kv_b(const KvArgs &a)
+template <typename T, int BITS, int DPT>
+static cudaError_t launch_kv_t(const KvArgs &a)
 {
-    // D <= 2048 (checked by the caller) keeps threads-per-row D / 8 <= 256
+    // D <= 2048 (checked by the caller) keeps threads-per-row D / DPT <= 256
     const int threads = 256;
     const dim3 grid((unsigned)(a.B * a.H), 2);
-    kv_quant_kernel<T, BITS><<<grid, threads, 0, a.stream>>>(
+    kv_quant_kernel<T, BITS, DPT><<<grid, threads, 0, a.stream>>>(
         (const T *)a.k, (const T *)a.v, a.H, a.S, a.D, a.ck, a.sk, a.zk, a.cv, a.sv, a.zv, a.g, a.kq,
         a.vq, a.err);
     return cudaGetLastError();
@@ -171,7 +179,8 @@ static cudaError_t launch_kv_b(const KvArgs &a)
 template <typename T>
 static cudaError_t launch_kv_d(const KvArgs &a)
 {
-    return a.bits == 4 ? launch_kv_b<T, 4>(a) : launch_kv_b<T, 3>(a);
+    if (a.D % 16 == 0) return a.bits == 4 ? launch_kv_t<T, 4, 16>(a) : launch_kv_t<T, 3, 16>(a);
+    return a.bits == 4 ? launch_kv_t<T, 4, 8>(a) : launch_kv_t<T, 3, 8>(a);
 }
 
 cudaError_t launch_kv_quant(const KvArgs &a)

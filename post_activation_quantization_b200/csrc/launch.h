@@ -98,6 +98,8 @@ struct KmArgs {
     void *ws;
     cudaStream_t stream;
     int num_sms;
+    int max_smem;
+    int *err;
 };
 
 // force_simple = 1 routes codes-only calls to the general kernel (used by tests of that path)
@@ -109,6 +111,8 @@ cudaError_t launch_kv_quant(const KvArgs &a);
 cudaError_t launch_dequant(const DequantArgs &a);
 cudaError_t launch_kmeans(const KmArgs &a);
 size_t kmeans_ws_bytes(int C, int g);
-size_t km_final_smem(int C, int g);
+int km_final_batch(int C, int g, int max_smem);
+// the sticky device error word of the current device (nullptr if it cannot be looked up)
+int *device_error_word();
 
 }  // namespace rptq

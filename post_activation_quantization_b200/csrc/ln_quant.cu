@@ -85,7 +85,6 @@ __global__ void __launch_bounds__(512, 1)
         }
     }
 
-    const uint32_t codebuf_s = smem_u32(codebuf);
     const int64_t pitch = (int64_t)C * BITS / 8;
     const int NU = C >> 5;  // 32-position pack units
     int64_t lq = 0;
@@ -101,17 +100,13 @@ __global__ void __launch_bounds__(512, 1)
         for (int k = 0; k < CPT; ++k) {
             const int ch = tid + k * NT;
             if (ch >= NCH) continue;
-            uint16_t pos[VEC];
+            uint32_t pw[VEC / 2];  // stored positions of the chunk's channels, two u16 per word
             if constexpr (VEC == 8) {
                 const uint4 p = *reinterpret_cast<const uint4 *>(postab + ch * 8);
-                const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
-#pragma unroll
-                for (int e = 0; e < 8; ++e) pos[e] = (uint16_t)(pw[e >> 1] >> (16 * (e & 1)));
+                pw[0] = p.x, pw[1] = p.y, pw[2] = p.z, pw[3] = p.w;
             } else {
                 const uint2 p = *reinterpret_cast<const uint2 *>(postab + ch * 4);
-                const uint32_t pw[2] = {p.x, p.y};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) pos[e] = (uint16_t)(pw[e >> 1] >> (16 * (e & 1)));
+                pw[0] = p.x, pw[1] = p.y;
             }
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
@@ -123,7 +118,8 @@ __global__ void __launch_bounds__(512, 1)
                     b[r] = __float_as_uint(fmaf(u, QMAX, MAGIC_RINT));
                 }
                 const uint32_t word = prmt(prmt(b[0], b[1], 0x0040), prmt(b[2], b[3], 0x0040), 0x5410);
-                asm volatile("st.shared.u32 [%0], %1;" ::"r"(codebuf_s + pos[e]), "r"(word) : "memory");
+                const uint32_t pos = (e & 1) ? (pw[e >> 1] >> 16) : (pw[e >> 1] & 0xffffu);
+                *reinterpret_cast<uint32_t *>(codebuf + pos) = word;
             }
         }
         __syncthreads();

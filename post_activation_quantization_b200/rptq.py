@@ -25,7 +25,7 @@ RPTQ_F32, RPTQ_F16, RPTQ_BF16 = 0, 1, 2
 RPTQ_LAYOUT_ROWS, RPTQ_LAYOUT_BHSD = 0, 1
 RPTQ_DEVERR_CLUSTER_ID, RPTQ_DEVERR_REORDER, RPTQ_DEVERR_TIMEOUT = 1, 2, 4
 RPTQ_MAX_CHANNELS = 16384
-RPTQ_MAX_CLUSTERS = 1024
+RPTQ_MAX_CLUSTERS = 512
 
 _DT = {torch.float32: RPTQ_F32, torch.float16: RPTQ_F16, torch.bfloat16: RPTQ_BF16}
 _TD = {v: k for k, v in _DT.items()}
