@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
-        pipe.load(lq, nrows, xr);
+        pipe.load(nrows, xr);
         float rstd[4], nmr[4];
         quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
 #pragma unroll
@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(512, 1)
                     tmin[k][e] = fminf(tmin[k][e], t);
                 }
             }
+        pipe.advance();
     }
     if (lq == 0) return;  // this CTA saw no rows
 #pragma unroll

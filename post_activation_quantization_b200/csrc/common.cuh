@@ -82,46 +82,14 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 }
 
 // ---- two fp32 lanes in one 64-bit register pair (sm_100 packed fp32 arithmetic) ---------
-// fma/add/mul on .f32x2 round each lane exactly like the scalar instruction (IEEE, nearest).
-struct f32x2 {
-    unsigned long long v;
-};
-__device__ __forceinline__ f32x2 mk2(float lo, float hi)
-{
-    f32x2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float lo2(f32x2 a)
-{
-    float l, h;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(l), "=f"(h) : "l"(a.v));
-    return l;
-}
-__device__ __forceinline__ float hi2(f32x2 a)
-{
-    float l, h;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(l), "=f"(h) : "l"(a.v));
-    return h;
-}
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
-{
-    f32x2 r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r.v) : "l"(a.v), "l"(b.v), "l"(c.v));
-    return r;
-}
-__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
-{
-    f32x2 r;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
-    return r;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
-{
-    f32x2 r;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
-    return r;
-}
+// __ffma2_rn / __fadd2_rn / __fmul2_rn round each lane exactly like the scalar operation.
+using f32x2 = float2;
+__device__ __forceinline__ f32x2 mk2(float lo, float hi) { return make_float2(lo, hi); }
+__device__ __forceinline__ float lo2(f32x2 a) { return a.x; }
+__device__ __forceinline__ float hi2(f32x2 a) { return a.y; }
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) { return __fmul2_rn(a, b); }
 // Elements 2p, 2p+1 of a 16-byte chunk as one fp32 pair (exact widening).
 template <typename T> __device__ __forceinline__ f32x2 pair_of(const uint4 &v, int p);
 template <> __device__ __forceinline__ f32x2 pair_of<__nv_bfloat16>(const uint4 &v, int p)
@@ -305,8 +273,9 @@ __device__ __forceinline__ void pack8x4_a3(const uint32_t *w, uint32_t (&o)[4])
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         // byte lanes hold 6-bit fields f0..f3; gather them to f0 | f1<<6 | f2<<12 | f3<<18
+        // u = f0 + f1 2^6 + (f2 + f3 2^6) 2^16; move the upper 12-bit field down by 4 bits
         const uint32_t u = prmt(t[r], 0u, 0x4240) + (prmt(t[r], 0u, 0x4341) << 6);
-        o[r] = (u & 0xfffu) | ((u >> 4) & 0xfff000u);
+        o[r] = u - (u >> 16) * 61440u;
     }
 }
 

@@ -5,7 +5,11 @@
 // tensor is ever stored; text after Fig. 2: one scale s and zero point z per cluster.
 // Quantization-basics article, sections 1.1 (static range, clamp) and 1.3 (q = round(y/s)+z).
 //
-// Fast kernel (codes only, C % 32 == 0): see row_pipeline.cuh for the row staging.  Per quad
+// Fast kernel (codes only, C % 32 == 0): see row_pipeline.cuh for the row staging.  When shared
+// memory cannot hold eight ring rows next to a separate code buffer (large C), the code buffer of
+// a quad lives in that quad's own four ring slots, which are free once the rows sit in registers;
+// they are refilled after the pack, and the eight-row ring still keeps a whole quad in flight.
+// Per quad
 // of four tokens a thread holds its chunks of x in registers, computes the LayerNorm
 // statistics, and for each of its channels c turns the four tokens' values into four codes
 //     u = sat(((x - mean) * rstd) * A_c + B_c),  code = rint(u * qmax)
@@ -34,7 +38,7 @@ __global__ void __launch_bounds__(512, 1)
                          const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
                          const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
                          const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int NS,
-                         int *err)
+                         int alias, int *err)
 {
     constexpr int VEC = Elem<T>::VEC;
     constexpr float QMAX = (float)((1 << BITS) - 1);
@@ -42,9 +46,10 @@ __global__ void __launch_bounds__(512, 1)
     const int tid = threadIdx.x, NT = blockDim.x;
     const int NCH = C / VEC;
     const uint32_t rowbytes = (uint32_t)C * sizeof(T);
-    const QuadSmem L = quad_smem_layout(NS, rowbytes, (size_t)C * 4 + (size_t)C * 2 + 2 * 8 * 32 * 4);
-    uint8_t *codebuf = smem + L.extra_off;                                   // 4*C bytes
-    uint16_t *postab = reinterpret_cast<uint16_t *>(codebuf + (size_t)C * 4);  // 2*C bytes
+    const size_t cb_bytes = alias ? 0 : (size_t)C * 4;
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, cb_bytes + (size_t)C * 2 + 2 * 8 * 32 * 4);
+    uint8_t *codebuf = smem + L.extra_off;                                    // 4*C bytes (own)
+    uint16_t *postab = reinterpret_cast<uint16_t *>(smem + L.extra_off + cb_bytes);  // 2*C bytes
     float *red = reinterpret_cast<float *>(postab + C);                      // 8*32 floats
     float *red2 = red + 8 * 32;
 
@@ -91,9 +96,10 @@ __global__ void __launch_bounds__(512, 1)
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
-        pipe.load(lq, nrows, xr);
+        pipe.load(nrows, xr);
         float rstd[4], nmr[4];
-        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, !alias);
+        if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
 
         // ---- codes of four tokens per channel -> one word at the channel's stored position
 #pragma unroll
@@ -159,6 +165,11 @@ __global__ void __launch_bounds__(512, 1)
                 }
             }
         }
+        if (alias) {  // the quad's slots held its codes until now
+            __syncthreads();
+            pipe.refill(lq);
+        }
+        pipe.advance();
     }
 }
 
@@ -259,10 +270,10 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------------------------------
 
 template <typename T, int BITS, int CPT>
-static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS)
+static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias)
 {
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
-    const QuadSmem L = quad_smem_layout(NS, rowbytes, (size_t)a.C * 4 + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, (alias ? 0 : (size_t)a.C * 4) + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
     auto kern = ln_quant_fast_kernel<T, BITS, CPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     if (e != cudaSuccess) return e;
@@ -274,30 +285,30 @@ static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS)
     const int64_t grid = std::min<int64_t>(quads, (int64_t)per_sm * a.num_sms);
     kern<<<(unsigned)grid, NT, L.total, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps,
                                                     a.R, a.col_cluster, a.scale, a.zero, a.g,
-                                                    a.codes, NS, a.err);
+                                                    a.codes, NS, alias, a.err);
     return cudaGetLastError();
 }
 
 template <typename T, int BITS>
-static cudaError_t launch_fast_b(const LnQuantArgs &a, int CPT, int NT, int NS)
+static cudaError_t launch_fast_b(const LnQuantArgs &a, int CPT, int NT, int NS, int alias)
 {
     switch (CPT) {
-    case 1: return launch_fast_t<T, BITS, 1>(a, NT, NS);
-    case 2: return launch_fast_t<T, BITS, 2>(a, NT, NS);
-    case 3: return launch_fast_t<T, BITS, 3>(a, NT, NS);
+    case 1: return launch_fast_t<T, BITS, 1>(a, NT, NS, alias);
+    case 2: return launch_fast_t<T, BITS, 2>(a, NT, NS, alias);
+    case 3: return launch_fast_t<T, BITS, 3>(a, NT, NS, alias);
     default: return cudaErrorInvalidValue;
     }
 }
 
 template <typename T>
-static cudaError_t launch_fast_d(const LnQuantArgs &a, int CPT, int NT, int NS)
+static cudaError_t launch_fast_d(const LnQuantArgs &a, int CPT, int NT, int NS, int alias)
 {
-    return a.bits == 4 ? launch_fast_b<T, 4>(a, CPT, NT, NS) : launch_fast_b<T, 3>(a, CPT, NT, NS);
+    return a.bits == 4 ? launch_fast_b<T, 4>(a, CPT, NT, NS, alias) : launch_fast_b<T, 3>(a, CPT, NT, NS, alias);
 }
 
 // Plan of the fast kernel for (C, dtype): threads, chunks per thread and ring depth;
 // returns false when the shape needs the simple kernel.
-bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS)
+bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS, int *alias)
 {
     if (C % 32 != 0) return false;
     const int VEC = 16 / esize;
@@ -313,16 +324,28 @@ bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *
     }
     if (!cpt) return false;
     const uint32_t rowbytes = (uint32_t)C * esize;
-    for (int ns = 8; ns >= 4; --ns) {
-        const QuadSmem L = quad_smem_layout(ns, rowbytes, (size_t)C * 4 + (size_t)C * 2 + 2 * 8 * 32 * 4);
-        if (L.total <= (size_t)max_smem) {
-            *CPT = cpt;
-            *NT = nt;
-            *NS = ns;
-            return true;
-        }
+    const size_t tables = (size_t)C * 2 + 2 * 8 * 32 * 4;
+    auto fits = [&](int ns, bool al) {
+        return quad_smem_layout(ns, rowbytes, (al ? 0 : (size_t)C * 4) + tables).total <= (size_t)max_smem;
+    };
+    // preference: 8 ring rows with a separate code buffer, then 8 rows with the code buffer in
+    // the quad's own slots, then fewer rows
+    int ns = 0, al = 0;
+    if (fits(8, false)) {
+        ns = 8;
+    } else if (fits(8, true)) {
+        ns = 8;
+        al = 1;
+    } else {
+        for (int n = 7; n >= 4 && !ns; --n)
+            if (fits(n, false)) ns = n;
     }
-    return false;
+    if (!ns) return false;
+    *CPT = cpt;
+    *NT = nt;
+    *NS = ns;
+    *alias = al;
+    return true;
 }
 
 template <typename T>
@@ -347,14 +370,14 @@ cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple)
 {
     if (a.T == 0) return cudaSuccess;
     const int esize = a.dtype == RPTQ_F32 ? 4 : 2;
-    int CPT = 0, NT = 0, NS = 0;
+    int CPT = 0, NT = 0, NS = 0, alias = 0;
     const bool fast = !force_simple && a.ln_out == nullptr && a.codes != nullptr &&
-                      ln_quant_fast_plan(a.C, esize, a.max_smem, &CPT, &NT, &NS);
+                      ln_quant_fast_plan(a.C, esize, a.max_smem, &CPT, &NT, &NS, &alias);
     if (fast) {
         switch (a.dtype) {
-        case RPTQ_F32: return launch_fast_d<float>(a, CPT, NT, NS);
-        case RPTQ_F16: return launch_fast_d<__half>(a, CPT, NT, NS);
-        default: return launch_fast_d<__nv_bfloat16>(a, CPT, NT, NS);
+        case RPTQ_F32: return launch_fast_d<float>(a, CPT, NT, NS, alias);
+        case RPTQ_F16: return launch_fast_d<__half>(a, CPT, NT, NS, alias);
+        default: return launch_fast_d<__nv_bfloat16>(a, CPT, NT, NS, alias);
         }
     }
     switch (a.dtype) {

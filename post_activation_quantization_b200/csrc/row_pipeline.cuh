@@ -29,6 +29,9 @@ struct QuadRows {
     uint8_t *ring;      // NS * rowbytes, 128-byte aligned
     uint32_t bar0;      // shared address of NS consecutive 8-byte mbarriers
     int *err;
+    // ring position of the current quad's first row, kept incrementally (no divisions):
+    // slot = (4 lq) mod NS and phase parity = ((4 lq) / NS) mod 2
+    uint32_t slot = 0, phase = 0;
 
     __device__ __forceinline__ int64_t row_of(int64_t local) const
     {
@@ -36,15 +39,14 @@ struct QuadRows {
         const int64_t q = (int64_t)blockIdx.x + (local >> 2) * (int64_t)gridDim.x;
         return 4 * q + (local & 3);
     }
-    // thread 0 only
-    __device__ __forceinline__ void issue(int64_t local) const
+    // thread 0 only: local row `local` into ring slot `s`
+    __device__ __forceinline__ void issue(int64_t local, uint32_t s) const
     {
         const int64_t row = row_of(local);
         if (row >= T_) return;
-        const int slot = (int)(local % NS);
-        const uint32_t bar = bar0 + 8u * slot;
+        const uint32_t bar = bar0 + 8u * s;
         mbar_expect_tx(bar, rowbytes);
-        bulk_g2s(smem_u32(ring + (size_t)slot * rowbytes), x + row * (int64_t)C, rowbytes, bar);
+        bulk_g2s(smem_u32(ring + (size_t)s * rowbytes), x + row * (int64_t)C, rowbytes, bar);
     }
     // thread 0: barriers + first NS rows.  Caller must __syncthreads() before any wait.
     __device__ __forceinline__ void start() const
@@ -52,19 +54,29 @@ struct QuadRows {
         if (threadIdx.x == 0) {
             for (int s = 0; s < NS; ++s) mbar_init(bar0 + 8u * s, 1);
             fence_mbar_init();
-            for (int s = 0; s < NS; ++s) issue(s);
+            for (int s = 0; s < NS; ++s) issue(s, (uint32_t)s);
         }
     }
-    // Wait for quad lq (rows < nrows valid) and copy this thread's chunks into registers.
-    __device__ __forceinline__ void load(int64_t lq, int nrows, uint4 (&xr)[4][CPT]) const
+    // ring slot and phase parity of row r (< 4) of the current quad
+    __device__ __forceinline__ void where(int r, uint32_t &s, uint32_t &ph) const
+    {
+        s = slot + r;
+        ph = phase;
+        if (s >= (uint32_t)NS) {
+            s -= NS;
+            ph ^= 1u;
+        }
+    }
+    // Wait for the current quad (rows < nrows valid) and copy this thread's chunks into registers.
+    __device__ __forceinline__ void load(int nrows, uint4 (&xr)[4][CPT]) const
     {
         const int tid = threadIdx.x, NT = blockDim.x;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int64_t local = 4 * lq + r;
-            const int slot = (int)(local % NS);
-            if (r < nrows) mbar_wait_bounded(bar0 + 8u * slot, (uint32_t)((local / NS) & 1), err);
-            const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)slot * rowbytes);
+            uint32_t s, ph;
+            where(r, s, ph);
+            if (r < nrows) mbar_wait_bounded(bar0 + 8u * s, ph, err);
+            const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)s * rowbytes);
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
                 const int ch = tid + k * NT;
@@ -72,24 +84,38 @@ struct QuadRows {
             }
         }
     }
-    // thread 0 after the first reduction of quad lq: refill its four slots.
+    // thread 0 after the quad's last read of its slots: refill them with the rows NS ahead
     __device__ __forceinline__ void refill(int64_t lq) const
     {
         if (threadIdx.x == 0) {
             fence_proxy_async_smem();
 #pragma unroll
-            for (int r = 0; r < 4; ++r) issue(4 * lq + NS + r);
+            for (int r = 0; r < 4; ++r) {
+                uint32_t s, ph;
+                where(r, s, ph);
+                issue(4 * lq + NS + r, s);  // the same slot, NS rows later
+            }
+        }
+    }
+    // all threads, at the end of every quad
+    __device__ __forceinline__ void advance()
+    {
+        slot += 4;
+        if (slot >= (uint32_t)NS) {
+            slot -= NS;
+            phase ^= 1u;
         }
     }
 };
 
 // LayerNorm statistics of the four rows in xr.  Returns rstd[r] and nmr[r] = -mean*rstd so that
 // the normalised value is fmaf(x, rstd, nmr).  `red`, `red2`: 8*(NT/32) floats each.
-// Calls refill() between its first barrier and any later one.
+// With refill_now, calls refill() between its first barrier and any later one (the caller
+// refills later when it still uses the quad's ring slots).
 template <typename T, int CPT, typename Pipe>
 __device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int NCH, float eps,
                                            float *red, float *red2, const Pipe &pipe, int64_t lq,
-                                           float (&rstd)[4], float (&nmr)[4])
+                                           float (&rstd)[4], float (&nmr)[4], bool refill_now = true)
 {
     constexpr int VEC = Elem<T>::VEC;
     const int tid = threadIdx.x, NT = blockDim.x;
@@ -110,7 +136,7 @@ __device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int
         }
     }
     cta_sum8(v, red);  // every thread is past its reads of this quad's ring slots
-    pipe.refill(lq);
+    if (refill_now) pipe.refill(lq);
     const float invC = 1.0f / (float)C;
     float mean[4], var[4];
     bool ill = false;
