@@ -57,6 +57,41 @@ template <> struct Elem<__half> {
     }
 };
 
+// Moments of a 16-byte chunk: s += sum(x), q += sum(x^2).  16-bit inputs use the sm_100
+// mixed-precision add/fma (16-bit sources, fp32 accumulator, one rounding; identical to widening
+// first), so no separate conversion instruction is spent on them.
+template <typename T> __device__ __forceinline__ void chunk_moments(const uint4 &v, float &s, float &q);
+template <> __device__ __forceinline__ void chunk_moments<float>(const uint4 &v, float &s, float &q)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float f = __uint_as_float(w[i]);
+        s += f;
+        q = fmaf(f, f, q);
+    }
+}
+template <> __device__ __forceinline__ void chunk_moments<__nv_bfloat16>(const uint4 &v, float &s, float &q)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.bf16 %0, lo, %0;\n"
+            " add.rn.f32.bf16 %0, hi, %0;\n fma.rn.f32.bf16 %1, lo, lo, %1;\n fma.rn.f32.bf16 %1, hi, hi, %1;\n}"
+            : "+f"(s), "+f"(q)
+            : "r"(w[i]));
+}
+template <> __device__ __forceinline__ void chunk_moments<__half>(const uint4 &v, float &s, float &q)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %2;\n add.rn.f32.f16 %0, lo, %0;\n"
+            " add.rn.f32.f16 %0, hi, %0;\n fma.rn.f32.f16 %1, lo, lo, %1;\n fma.rn.f32.f16 %1, hi, hi, %1;\n}"
+            : "+f"(s), "+f"(q)
+            : "r"(w[i]));
+}
+
 // Streaming 16-byte global load that does not allocate in L1.
 __device__ __forceinline__ uint4 ldg_stream(const void *p)
 {

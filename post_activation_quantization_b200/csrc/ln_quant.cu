@@ -32,7 +32,7 @@
 namespace rptq {
 
 // ------------------------------------------------------------------------------------------
-template <typename T, int BITS, int CPT>
+template <typename T, int BITS, int CPT, bool EXACT>
 __global__ void __launch_bounds__(512, 1)
     ln_quant_fast_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
                          const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
@@ -96,16 +96,22 @@ __global__ void __launch_bounds__(512, 1)
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
-        pipe.load(nrows, xr);
+        if (EXACT && nrows == 4)  // every chunk of every row is inside the tensor
+            pipe.load_full(xr);
+        else
+            pipe.load(nrows, xr);
         float rstd[4], nmr[4];
         quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, !alias);
         if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
 
         // ---- codes of four tokens per channel -> one word at the channel's stored position
+        const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
+        const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
+        const f32x2 qm2 = mk2(QMAX, QMAX), mg2 = mk2(MAGIC_RINT, MAGIC_RINT);
 #pragma unroll
         for (int k = 0; k < CPT; ++k) {
             const int ch = tid + k * NT;
-            if (ch >= NCH) continue;
+            if (!EXACT && ch >= NCH) continue;
             uint32_t pw[VEC / 2];  // stored positions of the chunk's channels, two u16 per word
             if constexpr (VEC == 8) {
                 const uint4 p = *reinterpret_cast<const uint4 *>(postab + ch * 8);
@@ -116,14 +122,17 @@ __global__ void __launch_bounds__(512, 1)
             }
 #pragma unroll
             for (int e = 0; e < VEC; ++e) {
-                uint32_t b[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
-                    const float u = fma_sat(t, pA[k][e], pB[k][e]);
-                    b[r] = __float_as_uint(fmaf(u, QMAX, MAGIC_RINT));
-                }
-                const uint32_t word = prmt(prmt(b[0], b[1], 0x0040), prmt(b[2], b[3], 0x0040), 0x5410);
+                // normalised values of channel e for tokens (0,1) and (2,3), two lanes at a time
+                const f32x2 t01 = fma2(mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e)), rs01, nm01);
+                const f32x2 t23 = fma2(mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e)), rs23, nm23);
+                const float A = pA[k][e], Bc = pB[k][e];
+                // u = sat(y / (s qmax) + z / qmax); code = rint(u qmax) (the 1.5*2^23 rounding add)
+                const f32x2 u01 = mk2(fma_sat(lo2(t01), A, Bc), fma_sat(hi2(t01), A, Bc));
+                const f32x2 u23 = mk2(fma_sat(lo2(t23), A, Bc), fma_sat(hi2(t23), A, Bc));
+                const f32x2 b01 = fma2(u01, qm2, mg2), b23 = fma2(u23, qm2, mg2);
+                const uint32_t word = prmt(prmt(__float_as_uint(lo2(b01)), __float_as_uint(hi2(b01)), 0x0040),
+                                           prmt(__float_as_uint(lo2(b23)), __float_as_uint(hi2(b23)), 0x0040),
+                                           0x5410);
                 const uint32_t pos = (e & 1) ? (pw[e >> 1] >> 16) : (pw[e >> 1] & 0xffffu);
                 *reinterpret_cast<uint32_t *>(codebuf + pos) = word;
             }
@@ -132,33 +141,32 @@ __global__ void __launch_bounds__(512, 1)
 
         // ---- pack 32 stored positions x 4 tokens per thread, write whole words
         for (int u = tid; u < NU; u += NT) {
-            uint32_t w[32];
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t slot = 8u * u + (kk ^ (u & 7));
-                const uint4 q = *reinterpret_cast<const uint4 *>(codebuf + (slot << 4));
-                w[4 * kk + 0] = q.x;
-                w[4 * kk + 1] = q.y;
-                w[4 * kk + 2] = q.z;
-                w[4 * kk + 3] = q.w;
-            }
-            uint32_t o[4][4];  // [group m][token r]
+            uint32_t o[4][4];  // [group m of 8 positions][token r]
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                if constexpr (BITS == 4)
-                    pack8x4_a4(w + 8 * m, o[m]);
-                else
-                    pack8x4_a3(w + 8 * m, o[m]);
-            }
+                uint32_t w[8];
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t slot = 8u * u + ((2 * m + h) ^ (u & 7));
+                    const uint4 q = *reinterpret_cast<const uint4 *>(codebuf + (slot << 4));
+                    w[4 * h + 0] = q.x;
+                    w[4 * h + 1] = q.y;
+                    w[4 * h + 2] = q.z;
+                    w[4 * h + 3] = q.w;
+                }
+                if constexpr (BITS == 4)
+                    pack8x4_a4(w, o[m]);
+                else
+                    pack8x4_a3(w, o[m]);
+            }
+            uint8_t *dst = codes + 4 * gq * pitch + (BITS == 4 ? 16 : 12) * (int64_t)u;
+#pragma unroll
+            for (int r = 0; r < 4; ++r, dst += pitch) {
                 if (r >= nrows) break;
-                uint8_t *dst = codes + (4 * gq + r) * pitch;
                 if constexpr (BITS == 4) {
-                    *reinterpret_cast<uint4 *>(dst + 16 * (int64_t)u) =
-                        make_uint4(o[0][r], o[1][r], o[2][r], o[3][r]);
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0][r], o[1][r], o[2][r], o[3][r]);
                 } else {
-                    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst + 12 * (int64_t)u);
+                    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
                     d32[0] = o[0][r] | (o[1][r] << 24);
                     d32[1] = (o[1][r] >> 8) | (o[2][r] << 16);
                     d32[2] = (o[2][r] >> 16) | (o[3][r] << 8);
@@ -274,7 +282,8 @@ static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias
 {
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
     const QuadSmem L = quad_smem_layout(NS, rowbytes, (alias ? 0 : (size_t)a.C * 4) + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
-    auto kern = ln_quant_fast_kernel<T, BITS, CPT>;
+    const bool exact = (a.C / (int)Elem<T>::VEC) == CPT * NT;  // chunks split evenly over threads
+    auto kern = exact ? ln_quant_fast_kernel<T, BITS, CPT, true> : ln_quant_fast_kernel<T, BITS, CPT, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

@@ -84,6 +84,20 @@ struct QuadRows {
             }
         }
     }
+    // The same for a full quad whose chunks are all inside the row (no predicates).
+    __device__ __forceinline__ void load_full(uint4 (&xr)[4][CPT]) const
+    {
+        const int tid = threadIdx.x, NT = blockDim.x;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            uint32_t s, ph;
+            where(r, s, ph);
+            mbar_wait_bounded(bar0 + 8u * s, ph, err);
+            const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)s * rowbytes) + tid;
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) xr[r][k] = src[k * NT];
+        }
+    }
     // thread 0 after the quad's last read of its slots: refill them with the rows NS ahead
     __device__ __forceinline__ void refill(int64_t lq) const
     {
@@ -122,19 +136,11 @@ __device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    // chunks beyond the row were loaded as zeros and add nothing
 #pragma unroll
-    for (int k = 0; k < CPT; ++k) {
-        if (tid + k * NT < NCH) {
+    for (int k = 0; k < CPT; ++k)
 #pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    const float xv = Elem<T>::get(xr[r][k], e);
-                    v[r] += xv;
-                    v[4 + r] = fmaf(xv, xv, v[4 + r]);
-                }
-        }
-    }
+        for (int r = 0; r < 4; ++r) chunk_moments<T>(xr[r][k], v[r], v[4 + r]);
     cta_sum8(v, red);  // every thread is past its reads of this quad's ring slots
     if (refill_now) pipe.refill(lq);
     const float invC = 1.0f / (float)C;
