@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import hashlib
 import io
 import json
@@ -105,16 +106,18 @@ class Step:
                     scale=torch.empty(g, dtype=torch.float32, device=d),
                     zero=torch.empty(g, dtype=torch.int32, device=d))
 
-    # (name, algorithmic bytes per launch, launches of our kernels per call)
+    # (name, algorithmic bytes per call, launches of our kernels per call).  A calibration call
+    # without `accumulate` is an init launch + the reduction; a KMeans call is four launches
+    # (prep, rank, the cooperative Lloyd kernel, the final sort / scale kernel).
     def stages(self):
         w, k = self.w, self.kvw
         n = w.T * w.C
         st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2),
-              ("kmeans_act", 0, 4 + w.iters),
+              ("kmeans_act", 0, 4),
               ("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
         if k:
             st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4),
-                   ("kmeans_kv", 0, 2 * (4 + k.iters)),
+                   ("kmeans_kv", 0, 2 * 4),
                    ("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
         st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
         if k:
@@ -237,7 +240,7 @@ def run_rptq(args):
     if ws > 1:
         torch.distributed.barrier()
     rptq.lib()
-    w = W.WORKLOADS[args.workload]
+    w = scaled_workload(args)
     step = Step(w, rank, dev)
     stages = step.stages()
     for _ in range(args.warmup):
@@ -308,6 +311,20 @@ def run_rptq(args):
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+
+
+def scaled_workload(args) -> W.Workload:
+    """The named workload; with --token-scale f < 1 its token counts (T, calibration tokens,
+    K/V sequence length) shrink by f -- a smaller case of the same kernels for ncu captures,
+    never the configuration a bench number is quoted on."""
+    w = W.WORKLOADS[args.workload]
+    f = args.token_scale
+    if f == 1.0:
+        return w
+    kv = w.kv and dataclasses.replace(w.kv, S=max(1, int(w.kv.S * f)))
+    return dataclasses.replace(w, T=max(4, int(w.T * f)) if w.T else 0,
+                               T_cal=max(4, int(w.T_cal * f)) if w.T_cal else 0, kv=kv,
+                               name=f"{w.name} (tokens x{f:g}, profiling case)")
 
 
 def workload_config(w):
@@ -475,11 +492,13 @@ def main():
     ap.add_argument("--impl", choices=["rptq", "reference"], default="rptq")
     ap.add_argument("--workload", choices=W.ORDER, default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--cpu-frac", type=float, default=1 / 4,
+    ap.add_argument("--cpu-frac", type=float, default=1 / 2,
                     help="fraction of the tokens the CPU oracle processes for its baseline")
     ap.add_argument("--ref-frac", type=float, default=1 / 32,
                     help="fraction of the tokens per step of the --impl reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--token-scale", type=float, default=1.0,
+                    help="shrink the token counts (a small case for ncu captures; not a bench config)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
