@@ -156,19 +156,20 @@ int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iter
 /*
  * Allocation-free variant of rptq_kmeans (the pages have no counterpart: this is a library
  * convenience).  Same arguments, outputs and results as rptq_kmeans, without the workspace:
- * the scratch is a fixed 1 MiB array inside the library's device image, which every GPU that
+ * the scratch is a fixed 2 MiB array inside the library's device image, which every GPU that
  * loads the library holds until the process exits.  For callers that cannot allocate device
  * memory while running (a plugin whose host owns all GPU memory, a serving loop that forbids
  * cudaMalloc / cudaFree after start-up); the call itself allocates nothing.
- *   - (C, g) needing more than 1 MiB of scratch is refused with RPTQ_ERR_UNSUPPORTED (every
- *     C <= RPTQ_MAX_CHANNELS fits for g <= 256);
+ *   - (C, g) needing more than 2 MiB of scratch is refused with RPTQ_ERR_UNSUPPORTED (every
+ *     C <= RPTQ_MAX_CHANNELS with g <= RPTQ_MAX_CLUSTERS fits, so this does not happen within
+ *     the library's limits);
  *   - all calls on a device share the scratch: calls whose kernels may overlap on the GPU
  *     race and can give wrong results, so order them (one stream, or events);
  *   - the scratch keeps the last call's contents; each call re-initialises what it reads;
  *   - the first call on a device looks up the scratch's device address (and the device's
  *     properties) with that device current; make that first call before any stream capture.
  */
-#define RPTQ_KMEANS_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define RPTQ_KMEANS_NOALLOC_SCRATCH_BYTES (2u << 20)
 int rptq_kmeans_noalloc(const float *ch_max, const float *ch_min, int C, int g, int iters,
                         int bits, int32_t *labels, double *centroids, int32_t *R,
                         int32_t *col_cluster, int32_t *offsets, float *scale, int32_t *zero,

@@ -162,7 +162,7 @@ int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iter
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
-    if (km_final_batch(C, g, d.max_smem) < 1) return RPTQ_ERR_UNSUPPORTED;
+    if (!kmeans_supported(C, g, d.max_smem)) return RPTQ_ERR_UNSUPPORTED;
     KmArgs a{ch_max, ch_min, C, g, iters, bits, labels, centroids, R, col_cluster, offsets,
              scale, zero, workspace, (cudaStream_t)stream, d.num_sms, d.max_smem, d.err};
     return cuda_status(launch_kmeans(a));

@@ -111,7 +111,8 @@ cudaError_t launch_kv_quant(const KvArgs &a);
 cudaError_t launch_dequant(const DequantArgs &a);
 cudaError_t launch_kmeans(const KmArgs &a);
 size_t kmeans_ws_bytes(int C, int g);
-int km_final_batch(int C, int g, int max_smem);
+// (C, g) within the limits and the fused KMeans kernel's shared memory within max_smem
+bool kmeans_supported(int C, int g, int max_smem);
 // the sticky device error word of the current device (nullptr if it cannot be looked up)
 int *device_error_word();
 

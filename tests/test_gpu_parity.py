@@ -101,18 +101,21 @@ def _check_kmeans(mx, mn, g, iters, bits):
 
 @pytest.mark.parametrize("C,g,iters,bits,seed", [
     (768, 8, 10, 4, 0), (4096, 32, 20, 4, 1), (4096, 32, 20, 3, 2), (9216, 64, 30, 3, 3),
-    (12288, 64, 50, 3, 4), (1000, 7, 0, 3, 5), (40, 40, 5, 4, 6), (64, 1, 3, 4, 7), (8, 3, 4, 3, 8)])
+    (12288, 64, 50, 3, 4), (1000, 7, 0, 3, 5), (40, 40, 5, 4, 6), (64, 1, 3, 4, 7), (8, 3, 4, 3, 8),
+    (513, 16, 10, 4, 11), (16384, 512, 8, 3, 10), (16384, 64, 50, 3, 12)])
 def test_kmeans_reorder_params(C, g, iters, bits, seed):
     mx, mn = _kmeans_case(C, g, iters, bits, seed, T=256 if C > 4096 else 512)
     _check_kmeans(mx, mn, g, iters, bits)
 
 
-def test_kmeans_duplicate_points_and_empty_clusters():
-    rng = np.random.default_rng(9)
-    C, g = 512, 16
-    mx = np.repeat(rng.normal(0, 1, 8), C // 8).astype(np.float32)  # 8 distinct points only
+@pytest.mark.parametrize("C,distinct", [(512, 8), (2048, 8), (1500, 5)])
+def test_kmeans_duplicate_points_and_empty_clusters(C, distinct):
+    # few distinct points, each repeated across many channels (equal keys inside and across the
+    # 512-channel segments the ranking is split into): ranks of equal keys follow the index
+    rng = np.random.default_rng(9 + C)
+    mx = rng.normal(0, 1, distinct)[rng.integers(0, distinct, C)].astype(np.float32)
     mn = (mx - 1.0).astype(np.float32)
-    _check_kmeans(mx, mn, g, 10, 3)
+    _check_kmeans(mx, mn, 16, 10, 3)
 
 
 # ---------------------------------------------------------------- fused LN + reorder + quant

@@ -78,9 +78,21 @@ def test_noalloc_matches_workspace_version_twice_in_a_row():
     assert rptq.rptq_device_error() == 0
 
 
-def test_noalloc_refuses_sizes_beyond_its_scratch():
-    C, g = 16384, 512  # valid for rptq_kmeans, but needs more than the 1 MiB scratch
-    assert rptq.lib().rptq_kmeans_workspace_size(C, g) > (1 << 20)
-    mx = torch.zeros(C, device="cuda")
+def test_noalloc_largest_problem_fits_its_scratch():
+    C, g = 16384, 512  # the library's largest (C, g): its workspace fits the 2 MiB scratch
+    assert rptq.lib().rptq_kmeans_workspace_size(C, g) <= (2 << 20)
+    mx, mn = _stats(C, 7)
+    ref = rptq.rptq_kmeans(mx, mn, g, 5, 3)
     out = _outputs(C, g)
-    assert _call_c_abi(mx, mx, g, 1, 3, out) == rptq.RPTQ_ERR_UNSUPPORTED
+    assert _call_c_abi(mx, mn, g, 5, 3, out) == rptq.RPTQ_OK
+    torch.cuda.synchronize()
+    _same(out, ref)
+    assert rptq.rptq_device_error() == 0
+
+
+def test_noalloc_refuses_invalid_sizes():
+    C = 1024
+    mx = torch.zeros(C, device="cuda")
+    out = _outputs(C, 8)
+    assert _call_c_abi(mx, mx, C + 1, 1, 3, out) == rptq.RPTQ_ERR_INVALID_ARG   # g > C
+    assert _call_c_abi(mx, mx, 8, 1, 5, out) == rptq.RPTQ_ERR_UNSUPPORTED      # bits
