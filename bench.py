@@ -22,6 +22,7 @@ from __future__ import annotations
 import argparse
 import csv
 import dataclasses
+import datetime
 import hashlib
 import io
 import json
@@ -89,12 +90,15 @@ class Step:
             self.kmv = self._km_out(k.channels, k.g)
             self.wsk = torch.empty(rptq.rptq_kmeans_workspace_size(k.channels, k.g), dtype=torch.uint8,
                                    device=device)
+            self.wsv = torch.empty_like(self.wsk)
             shape = (k.B, k.H, k.S, k.D * k.bits // 8)
             self.kq = torch.empty(shape, dtype=torch.uint8, device=device)
             self.vq = torch.empty(shape, dtype=torch.uint8, device=device)
             kvdt = synthetic.torch_dtype(k.dtype)
             self.khat = torch.empty((k.B, k.H, k.S, k.D), dtype=kvdt, device=device)
             self.vhat = torch.empty_like(self.khat)
+        # the three KMeans problems are independent: they run concurrently on their own streams
+        self.side = [torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)]
 
     def _km_out(self, C, g):
         d = self.dev
@@ -107,42 +111,39 @@ class Step:
                     zero=torch.empty(g, dtype=torch.int32, device=d))
 
     # (name, algorithmic bytes per call, launches of our kernels per call).  A calibration call
-    # without `accumulate` is an init launch + the reduction; a KMeans call is four launches
-    # (prep, rank, the cooperative Lloyd kernel, the final sort / scale kernel).
+    # without `accumulate` is an init launch + the reduction; a KMeans call is two launches (the
+    # workspace clear and the cooperative KMeans kernel).
     def stages(self):
         w, k = self.w, self.kvw
         n = w.T * w.C
-        st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2),
-              ("kmeans_act", 0, 4),
-              ("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+        st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2)]
         if k:
-            st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4),
-                   ("kmeans_kv", 0, 2 * 4),
-                   ("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
+            st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4)]
+        st += [("kmeans", 0, 2 * (3 if k else 1)),
+               ("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+        if k:
+            st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
         st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
         if k:
             st += [("dequant_kv", 2 * W.bytes_dequant(k.elems, k.dtype, k.bits), 2)]
         return st
 
     def run(self, ev=None):
-        """Enqueue one step on the current stream; ev: optional dict name -> (start, end)."""
+        """Enqueue one step on the current stream; ev: optional dict name -> (start, end).
+
+        Order: the streaming calibrations, then the activation, K and V KMeans concurrently
+        (three small cooperative grids on three streams), then quantization and dequantization."""
         r, w, k = self.r, self.w, self.kvw
+        main = torch.cuda.current_stream(self.dev)
 
         def mark(name, i):
             if ev is not None:
-                ev[name][i].record()
+                ev[name][i].record(main)
 
         mark("calib_ln", 0)
         r.rptq_calib_minmax(self.xcal, self.gamma, self.beta, w.eps, ch_max=self.mx, ch_min=self.mn)
         mark("calib_ln", 1)
         pdist.allreduce_minmax(self.mx, self.mn)
-        mark("kmeans_act", 0)
-        r.rptq_kmeans(self.mx, self.mn, w.g, w.iters, w.bits, workspace=self.ws, out=self.km)
-        mark("kmeans_act", 1)
-        mark("ln_reorder_quant", 0)
-        r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
-                                self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
-        mark("ln_reorder_quant", 1)
         if k:
             mark("kv_calib", 0)
             r.rptq_kv_calib_minmax(self.k, ch_max=self.kst[0], ch_min=self.kst[1])
@@ -150,10 +151,26 @@ class Step:
             mark("kv_calib", 1)
             pdist.allreduce_minmax(self.kst[0], self.kst[1])
             pdist.allreduce_minmax(self.kst[2], self.kst[3])
-            mark("kmeans_kv", 0)
-            r.rptq_kmeans(self.kst[0], self.kst[1], k.g, k.iters, k.bits, workspace=self.wsk, out=self.kmk)
-            r.rptq_kmeans(self.kst[2], self.kst[3], k.g, k.iters, k.bits, workspace=self.wsk, out=self.kmv)
-            mark("kmeans_kv", 1)
+        mark("kmeans", 0)
+        if k:
+            for s in self.side:
+                s.wait_stream(main)
+            with torch.cuda.stream(self.side[0]):
+                r.rptq_kmeans(self.kst[0], self.kst[1], k.g, k.iters, k.bits, workspace=self.wsk, out=self.kmk,
+                              stream=self.side[0])
+            with torch.cuda.stream(self.side[1]):
+                r.rptq_kmeans(self.kst[2], self.kst[3], k.g, k.iters, k.bits, workspace=self.wsv, out=self.kmv,
+                              stream=self.side[1])
+        r.rptq_kmeans(self.mx, self.mn, w.g, w.iters, w.bits, workspace=self.ws, out=self.km)
+        if k:
+            for s in self.side:
+                main.wait_stream(s)
+        mark("kmeans", 1)
+        mark("ln_reorder_quant", 0)
+        r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
+                                self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
+        mark("ln_reorder_quant", 1)
+        if k:
             mark("kv_quant", 0)
             r.rptq_kv_quant(self.k, self.v, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],
                             self.kmv["labels"], self.kmv["scale"], self.kmv["zero"], k.bits,
@@ -174,19 +191,26 @@ class Step:
 
 # ------------------------------------------------------------------------------------------
 class Clocks:
-    """nvidia-smi samples every 200 ms while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 100 ms; only those taken inside the timed region are kept."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.t0 = self.t1 = None
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.Q}",
                                        "--format=csv,noheader,nounits", "-lms", "100"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+
+    def start(self):
+        self.t0 = time.time()
+
+    def end(self):
+        self.t1 = time.time()
 
     def stop(self) -> dict:
         if self.p is None:
@@ -198,10 +222,20 @@ class Clocks:
             self.p.kill()
         self.f.flush()
         self.f.seek(0)
-        rows = [r for r in csv.reader(io.StringIO(self.f.read())) if len(r) >= 9]
+        rows = []
+        for r in csv.reader(io.StringIO(self.f.read())):
+            if len(r) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            if self.t0 is not None and self.t0 <= ts <= self.t1:
+                rows.append([x.strip() for x in r[1:]])
         os.unlink(self.f.name)
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        num = lambda v: v.replace(".", "", 1).isdigit()  # noqa: E731
+        sm = [float(r[1]) for r in rows if num(r[1])]
+        mx = [float(r[2]) for r in rows if num(r[2])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
@@ -243,23 +277,34 @@ def run_rptq(args):
     w = scaled_workload(args)
     step = Step(w, rank, dev)
     stages = step.stages()
+    tw = time.perf_counter()
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
+    tw = (time.perf_counter() - tw) / max(1, args.warmup)
     assert rptq.rptq_device_error() == 0, "device error word set during warm-up"
+    # untimed steps while the clock sampler starts (every rank runs the same number)
+    n_pre = int(pdist.max_over_ranks(min(2000, int(0.5 / max(tw, 1e-4)) + 1), dev))
 
     ev = {n: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
           for n, _, _ in stages}
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = Clocks(dev.index) if rank == 0 else None
+    for _ in range(n_pre):  # the sampler starts while the GPU runs these, so it is up when timing starts
+        step.run()
+    torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    if clk:
+        clk.start()
     t0.record()
     for i in range(args.steps):
         step.run({n: ev[n][i] for n in ev})
     t1.record()
     torch.cuda.synchronize()
+    if clk:
+        clk.end()
     if ws > 1:
         torch.distributed.barrier()
     clocks = clk.stop() if clk else None
@@ -487,7 +532,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["rptq", "reference"], default="rptq")
     ap.add_argument("--workload", choices=W.ORDER, default=DEFAULT_WORKLOAD)
