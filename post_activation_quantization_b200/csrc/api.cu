@@ -214,7 +214,7 @@ int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t
     int st = dev_info(&d);
     if (st) return st;
     KvArgs a{k, v, dtype, B, H, S, D, cluster_k, scale_k, zero_k, cluster_v, scale_v, zero_v, g,
-             bits, k_codes, v_codes, d.err, (cudaStream_t)stream};
+             bits, k_codes, v_codes, d.err, (cudaStream_t)stream, d.num_sms};
     return cuda_status(launch_kv_quant(a));
 }
 

@@ -93,6 +93,13 @@ template <> __device__ __forceinline__ void chunk_moments<__half>(const uint4 &v
 }
 
 // Streaming 16-byte global load that does not allocate in L1.
+// 32-bit read-once load (no L1 allocation)
+__device__ __forceinline__ uint32_t ldg_stream32(const void *p)
+{
+    uint32_t v;
+    asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
 __device__ __forceinline__ uint4 ldg_stream(const void *p)
 {
     uint4 v;

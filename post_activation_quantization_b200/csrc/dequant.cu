@@ -4,9 +4,18 @@
 // The code q becomes an exact float without a conversion instruction: the bit pattern
 // 0x4B000000 | q is the float 2^23 + q, and 2^23 + z is exact for |z| < 2^23 - 16, so
 // (2^23 + q) - (2^23 + z) = q - z exactly and one multiply by s gives the same fp32 value as
-// s * (float)(q - z).  A thread whose columns include a larger |z| converts with an integer ->
-// float conversion instead (same result).  Each thread owns DPT consecutive channels (32 when
-// the row length allows, else 8) and keeps their (s, 2^23 + z) in registers across rows.
+// s * (float)(q - z).  A thread whose channels include a larger |z| converts with an integer ->
+// float conversion instead (same result).
+//
+// Span kernels (the common shapes): a lane owns groups of 8 consecutive channels, and the 32
+// lanes of a warp own 32 consecutive groups, so every warp-wide 16-byte store covers 512
+// contiguous bytes of the output (whole 128-byte lines).  The 8 packed codes of a lane are 4
+// bytes (A4: one word per lane) or 3 bytes (A3: 24 lanes load the warp's 96 bytes as words and
+// each lane assembles its 3 bytes with two shuffles and a funnel shift).  Rows layout: warp w
+// of a CTA owns the 256-channel spans w, w + WR, w + 2 WR, ... of every row it walks, with
+// their (s, 2^23 + z) in registers.  BHSD layout: one CTA per (b, h) block of S rows x D
+// channels (contiguous), a warp covers 256 / D consecutive rows per store, so a lane's channel
+// position is fixed.  Other shapes use the general kernel (DPT consecutive channels per thread).
 #include <algorithm>
 
 #include "common.cuh"
@@ -184,6 +193,229 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// span kernels
+template <int BITS>
+__device__ __forceinline__ uint32_t span_load(const uint8_t *span, int lane)
+{
+    // A4: 128 bytes, word `lane`; A3: 96 bytes, words 0..23 (lanes 24..31 load nothing)
+    if constexpr (BITS == 4) return ldg_stream32(span + 4 * lane);
+    return lane < 24 ? ldg_stream32(span + 4 * lane) : 0u;
+}
+// the same when only the first `valid` bytes of the span exist (a partial last span)
+template <int BITS>
+__device__ __forceinline__ uint32_t span_load_partial(const uint8_t *span, int lane, int valid)
+{
+    uint32_t v = 0;
+    for (int b = 0; b < 4; ++b)
+        if (4 * lane + b < valid) v |= (uint32_t)span[4 * lane + b] << (8 * b);
+    return v;
+}
+template <int BITS>
+__device__ __forceinline__ uint32_t span_codes(uint32_t w, int lane)
+{
+    if constexpr (BITS == 4) return w;
+    const int b = 3 * lane, i0 = b >> 2;
+    const uint32_t lo = __shfl_sync(FULL, w, i0), hi = __shfl_sync(FULL, w, (i0 + 1) & 31);
+    return __funnelshift_r(lo, hi, 8 * (b & 3)) & 0xffffffu;
+}
+
+// 8 values s * (q - z) of one group; nzf = -(2^23 + z) (exact path) and the scales
+template <typename T, int BITS>
+__device__ __forceinline__ void decode_store(uint32_t grp, const float (&sc)[8], const float (&nzf)[8], T *dst)
+{
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        const uint32_t q0 = (grp >> (BITS * i)) & ((1u << BITS) - 1), q1 = (grp >> (BITS * (i + 1))) & ((1u << BITS) - 1);
+        const f32x2 x = add2(mk2(__uint_as_float(0x4B000000u | q0), __uint_as_float(0x4B000000u | q1)),
+                             mk2(nzf[i], nzf[i + 1]));
+        const f32x2 y = mul2(x, mk2(sc[i], sc[i + 1]));
+        v[i] = lo2(y);
+        v[i + 1] = hi2(y);
+    }
+    Store<T>::template put<8>(dst, v);
+}
+// the same through an integer subtraction (any z); channels c0 .. c0+7
+template <typename T, int BITS>
+__device__ __forceinline__ void decode_store_slow(uint32_t grp, const float (&sc)[8], const int32_t *cluster, int c0,
+                                               const int32_t *zero, int g, T *dst)
+{
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        int k = cluster[c0 + i];
+        k = (k < 0 || k >= g) ? 0 : k;
+        v[i] = sc[i] * (float)((int)((grp >> (BITS * i)) & ((1u << BITS) - 1)) - zero[k]);
+    }
+    Store<T>::template put<8>(dst, v);
+}
+
+__device__ __forceinline__ int checked_cluster(const int32_t *cluster, int c, int g, int *err)
+{
+    int k = cluster[c];
+    if (k < 0 || k >= g) {
+        raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+        k = 0;
+    }
+    return k;
+}
+
+// Rows layout, C % 256 == 0: CTA = WR warps, warp w owns spans w + WR*i (i < NSPAN) of every row.
+template <typename T, int BITS, int NSPAN>
+__global__ void __launch_bounds__(NSPAN <= 2 ? 1024 : 512)
+    dequant_rows_span(const uint8_t *__restrict__ codes, int64_t rows, int C, const int32_t *__restrict__ cluster,
+                      const float *__restrict__ scale, const int32_t *__restrict__ zero, int g, T *__restrict__ out,
+                      int *err)
+{
+    constexpr int U = 4;  // rows in flight
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, WR = blockDim.x >> 5;
+    const int64_t pitch = (int64_t)C * BITS / 8;
+    float sc[NSPAN][8], nzf[NSPAN][8];
+    bool exact = true;
+#pragma unroll
+    for (int i = 0; i < NSPAN; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = (w + WR * i) * 256 + 8 * lane + e;
+            const int k = checked_cluster(cluster, c, g, err);
+            sc[i][e] = scale[k];
+            const int z = zero[k];
+            const bool ok = z > -(1 << 23) + 16 && z < (1 << 23) - 16;
+            exact &= ok;
+            nzf[i][e] = -(float)((1 << 23) + (ok ? z : 0));
+        }
+    exact = __all_sync(FULL, exact);  // the shuffles below need the whole warp on one path
+    const int64_t step = gridDim.x;
+    for (int64_t r0 = blockIdx.x; r0 < rows; r0 += U * step) {
+        uint32_t wv[U][NSPAN];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + u * step;
+#pragma unroll
+            for (int i = 0; i < NSPAN; ++i)
+                wv[u][i] = r < rows ? span_load<BITS>(codes + r * pitch + (int64_t)(w + WR * i) * (32 * BITS), lane) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = r0 + u * step;
+#pragma unroll
+            for (int i = 0; i < NSPAN; ++i) {
+                const uint32_t grp = span_codes<BITS>(wv[u][i], lane);
+                T *dst = out + r * C + (w + WR * i) * 256 + 8 * lane;
+                if (r < rows) {
+                    if (exact)
+                        decode_store<T, BITS>(grp, sc[i], nzf[i], dst);
+                    else
+                        decode_store_slow<T, BITS>(grp, sc[i], cluster, (w + WR * i) * 256 + 8 * lane, zero, g, dst);
+                }
+            }
+        }
+    }
+}
+
+// BHSD layout, D % 8 == 0 and (D/8) divides 32.  A span is the RPW = 256/D consecutive rows one
+// warp-wide store covers; a work unit is up to 32 spans of one (b, h) block; units are ordered
+// (h, b, chunk) and every warp of a one-wave grid takes a contiguous range of them.  A lane's
+// channel position p is fixed; its 8 (s, 2^23 + z) are reloaded when the head changes.
+constexpr int DQ_SPANS_PER_UNIT = 32;
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+    dequant_bhsd_span(const uint8_t *__restrict__ codes, int B, int H, int S, int D, const int32_t *__restrict__ cluster,
+                      const float *__restrict__ scale, const int32_t *__restrict__ zero, int g, T *__restrict__ out,
+                      int *err)
+{
+    constexpr int U = 4;
+    const int lane = threadIdx.x & 31;
+    const int G8 = D >> 3, RPW = 32 / G8;
+    const int p = 8 * (lane % G8), lrow = lane / G8;
+    const int nspan = (S + RPW - 1) / RPW;  // spans per (b, h)
+    const int nchunk = (nspan + DQ_SPANS_PER_UNIT - 1) / DQ_SPANS_PER_UNIT;
+    // units in (h, b, chunk) order; warp gw takes the contiguous range [u0, u1), so it crosses
+    // at most a few heads and reloads its coefficients only then
+    const int64_t units = (int64_t)H * B * nchunk, TW = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t u0 = units * gw / TW, u1 = units * (gw + 1) / TW;
+    int64_t hb = u0 / nchunk;
+    int chunk = (int)(u0 - hb * nchunk);
+    int h = (int)(hb / B), b = (int)(hb - (int64_t)h * B);
+    float sc[8], nzf[8];
+    bool exact = true;
+    int cur_h = -1;
+    for (int64_t un = u0; un < u1; ++un) {
+        if (h != cur_h) {
+            exact = true;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int k = checked_cluster(cluster, h * D + p + e, g, err);
+                sc[e] = scale[k];
+                const int z = zero[k];
+                const bool ok = z > -(1 << 23) + 16 && z < (1 << 23) - 16;
+                exact &= ok;
+                nzf[e] = -(float)((1 << 23) + (ok ? z : 0));
+            }
+            exact = __all_sync(FULL, exact);
+            cur_h = h;
+        }
+        const int64_t bh = (int64_t)b * H + h;
+        const int sp0 = chunk * DQ_SPANS_PER_UNIT, sp1 = min(nspan, sp0 + DQ_SPANS_PER_UNIT);
+        const int64_t blk = bh * S;  // first row of this (b, h)
+        if (sp1 - sp0 == DQ_SPANS_PER_UNIT && (int64_t)sp1 * RPW <= S) {
+            // a whole unit: 32 full spans, contiguous codes and output from the unit's base
+            const uint8_t *cu = codes + (blk + (int64_t)sp0 * RPW) * D * BITS / 8;
+            T *ou = out + (blk + (int64_t)sp0 * RPW + lrow) * D + p;
+#pragma unroll 1
+            for (int sp = 0; sp < DQ_SPANS_PER_UNIT; sp += 2 * U) {
+                uint32_t wv[2 * U];
+#pragma unroll
+                for (int u = 0; u < 2 * U; ++u) wv[u] = span_load<BITS>(cu + (sp + u) * (32 * BITS), lane);
+#pragma unroll
+                for (int u = 0; u < 2 * U; ++u) {
+                    const uint32_t grp = span_codes<BITS>(wv[u], lane);
+                    T *dst = ou + (int64_t)(sp + u) * 256;
+                    if (exact)
+                        decode_store<T, BITS>(grp, sc, nzf, dst);
+                    else
+                        decode_store_slow<T, BITS>(grp, sc, cluster, h * D + p, zero, g, dst);
+                }
+            }
+        } else
+        for (int sp = sp0; sp < sp1; sp += U) {
+            uint32_t wv[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int spu = sp + u;
+                const int nrow = min(RPW, S - spu * RPW);
+                const uint8_t *src = codes + (blk + (int64_t)spu * RPW) * D * BITS / 8;
+                wv[u] = spu >= sp1 ? 0u
+                        : nrow == RPW ? span_load<BITS>(src, lane)
+                                      : span_load_partial<BITS>(src, lane, nrow * D * BITS / 8);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int spu = sp + u;
+                const uint32_t grp = span_codes<BITS>(wv[u], lane);
+                const int row = spu * RPW + lrow;
+                if (spu < sp1 && row < S) {
+                    T *dst = out + (blk + row) * D + p;
+                    if (exact)
+                        decode_store<T, BITS>(grp, sc, nzf, dst);
+                    else
+                        decode_store_slow<T, BITS>(grp, sc, cluster, h * D + p, zero, g, dst);
+                }
+            }
+        }
+        if (++chunk == nchunk) {  // next unit
+            chunk = 0;
+            if (++b == B) {
+                b = 0;
+                ++h;
+            }
+        }
+    }
+}
+
 template <typename T, int BITS, int DPT>
 static cudaError_t launch_dq_t(const DequantArgs &a)
 {
@@ -204,9 +436,50 @@ static cudaError_t launch_dq_t(const DequantArgs &a)
     return cudaGetLastError();
 }
 
+template <typename T, int BITS, int NSPAN>
+static cudaError_t launch_rows_span(const DequantArgs &a, int WR)
+{
+    const int threads = WR * 32;
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_rows_span<T, BITS, NSPAN>, threads, 0) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(a.n0, (int64_t)a.num_sms * per_sm));
+    dequant_rows_span<T, BITS, NSPAN><<<(unsigned)grid, threads, 0, a.stream>>>(
+        a.codes, a.n0, a.n1, a.cluster, a.scale, a.zero, a.g, (T *)a.out, a.err);
+    return cudaGetLastError();
+}
+
 template <typename T, int BITS>
 static cudaError_t launch_dq_b(const DequantArgs &a)
 {
+    const bool aligned = ((uintptr_t)a.codes % 4 == 0) && ((uintptr_t)a.out % 16 == 0);
+    if (a.layout == RPTQ_LAYOUT_BHSD) {
+        // word loads need every (b, h) block of codes to start on a 4-byte boundary
+        const bool blocks4 = ((int64_t)a.S * a.D * BITS / 8) % 4 == 0;
+        if (aligned && blocks4 && a.D % 8 == 0 && 32 % (a.D / 8) == 0 && a.D <= 256) {
+            int per_sm = 1;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_bhsd_span<T, BITS>, 256, 0) !=
+                    cudaSuccess ||
+                per_sm < 1)
+                per_sm = 1;
+            const int64_t rpw = 32 / (a.D / 8), nspan = (a.S + rpw - 1) / rpw;
+            const int64_t units = a.n0 * a.n1 * ((nspan + DQ_SPANS_PER_UNIT - 1) / DQ_SPANS_PER_UNIT);
+            const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((int64_t)a.num_sms * per_sm, (units + 7) / 8));
+            dequant_bhsd_span<T, BITS><<<(unsigned)grid, 256, 0, a.stream>>>(
+                a.codes, (int)a.n0, a.n1, (int)a.S, a.D, a.cluster, a.scale, a.zero, a.g, (T *)a.out, a.err);
+            return cudaGetLastError();
+        }
+    } else if (aligned && a.n1 % 256 == 0) {
+        const int spans = a.n1 / 256;  // 256-channel spans per row, at most 64
+        // fewest spans per thread (most warps) that keep the CTA within 1024 (NSPAN <= 2) or
+        // 512 threads
+        if (spans <= 32) return launch_rows_span<T, BITS, 1>(a, spans);
+        if (spans % 2 == 0) return launch_rows_span<T, BITS, 2>(a, spans / 2);
+        if (spans % 3 == 0 && spans / 3 <= 16) return launch_rows_span<T, BITS, 3>(a, spans / 3);
+        if (spans % 4 == 0 && spans / 4 <= 16) return launch_rows_span<T, BITS, 4>(a, spans / 4);
+    }
     const int width = a.layout == RPTQ_LAYOUT_BHSD ? a.D : a.n1;
     if (width % 32 == 0) return launch_dq_t<T, BITS, 32>(a);
     return launch_dq_t<T, BITS, 8>(a);

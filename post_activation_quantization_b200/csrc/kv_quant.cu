@@ -5,12 +5,15 @@
 // quantizer as the activations (text after Fig. 2; quantization-basics article, section 1.3).
 //
 // The cache keeps its [B, H, S, D] layout; channel c = h*D + d carries the cluster id of
-// channel c.  A CTA handles one (b, h) pair of one tensor: all its S rows share the same D
-// channels, so every thread loads the coefficients of its DPT consecutive channels once
-//     A_d = 1 / (s_k * qmax),  B_d = z_k / qmax        (u = sat(x*A_d + B_d), code = rint(u*qmax))
-// and then streams rows: 16-byte loads, codes accumulated in registers (the rounding constant
-// 1.5*2^23 leaves each code in the low bits of a float; a shifted sum of those bit patterns
-// minus a known constant is the packed word), and whole-word stores of the packed codes.
+// channel c.  A thread owns DPT consecutive channels of a row; all rows of one (b, h) block share
+// the same D channels, so the thread's coefficients (s, 1/s and the code-domain clamp) serve a
+// whole run of rows.  Per element: a correctly rounded x / s, the clamp, the rounding constant
+// 1.5*2^23 (which leaves the code in the low bits of the float), and a shifted sum of those bit
+// patterns minus a known constant is the packed word; rows are stored as whole words.
+// Warp kernel (D/DPT divides 32): a work unit is 64 rows of one (b, h) block; units are ordered
+// (h, b, chunk) and every warp of a one-wave grid takes a contiguous range of them, reloading its
+// coefficients only when the head changes.  CTA kernel
+// (other D): one CTA per (b, h) block.
 #include <algorithm>
 
 #include "common.cuh"
@@ -29,69 +32,214 @@ __device__ __forceinline__ float div_rn(float x, float s, float r)
     return fmaf(res, r, q0);
 }
 
+constexpr int KV_ROWS_PER_UNIT = 64;
+
+// Coefficients of a thread's DPT channels (h*D + d0 + i) for one head.
+template <int BITS, int DPT>
+struct KvCoef {
+    static constexpr int NG = DPT / 8;
+    static constexpr int QMAX = (1 << BITS) - 1;
+    static constexpr uint32_t MAGIC_BITS = 0x4B400000u;
+    f32x2 ns2[DPT / 2], r2[DPT / 2];  // -s and RN(1/s), two channels per pair
+    float lo_[DPT], hi_[DPT];         // code-domain clamp [-z, qmax - z]
+    uint32_t bias[NG];                // sum_i (MAGIC_BITS - z_i) << (BITS*i): removes the rounding constant
+    bool small_z;                     // |z| < 2^21 keeps q + 1.5*2^23 inside one binade (exact rounding)
+
+    __device__ __forceinline__ void load(const int32_t *cl, const float *sc, const int32_t *zp, int c0, int g,
+                                         int *err)
+    {
+        small_z = true;
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) bias[gi] = 0;
+#pragma unroll
+        for (int i = 0; i < DPT; i += 2) {
+            float sv2[2], rv2[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                int kc = cl[c0 + i + h2];
+                if (kc < 0 || kc >= g) {
+                    raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+                    kc = 0;
+                }
+                sv2[h2] = sc[kc];
+                rv2[h2] = __frcp_rn(sv2[h2]);
+                const int z = zp[kc];
+                lo_[i + h2] = (float)(-z);
+                hi_[i + h2] = (float)(QMAX - z);
+                bias[(i + h2) / 8] += (MAGIC_BITS - (uint32_t)z) << (BITS * ((i + h2) % 8));
+                small_z &= (z > -(1 << 21)) && (z < (1 << 21));
+            }
+            ns2[i / 2] = mk2(-sv2[0], -sv2[1]);
+            r2[i / 2] = mk2(rv2[0], rv2[1]);
+        }
+    }
+};
+
+// Codes of one row's DPT channels (x in VEC-element 16-byte chunks) -> NG packed 8-code groups.
 template <typename T, int BITS, int DPT>
-__global__ void __launch_bounds__(256)
-    kv_quant_kernel(const T *__restrict__ k, const T *__restrict__ v, int H, int64_t S, int D,
-                    const int32_t *__restrict__ ck, const float *__restrict__ sk,
-                    const int32_t *__restrict__ zk, const int32_t *__restrict__ cv,
-                    const float *__restrict__ sv, const int32_t *__restrict__ zv, int g,
-                    uint8_t *__restrict__ kq, uint8_t *__restrict__ vq, int *err)
+__device__ __forceinline__ void kv_quant_row(const uint4 *xb, const KvCoef<BITS, DPT> &cf, uint32_t *grp)
 {
     constexpr int VEC = Elem<T>::VEC;
-    constexpr int NLD = DPT / VEC;  // 16-byte loads per row and thread
-    constexpr int NG = DPT / 8;     // packed 8-code groups per row and thread
-    constexpr int QMAX = (1 << BITS) - 1;
-    constexpr uint32_t MAGIC_BITS = 0x4B400000u;
-    constexpr int U = 4;            // rows whose loads are in flight together
-    const bool is_v = blockIdx.y == 1;
-    const T *src = is_v ? v : k;
-    uint8_t *dst = is_v ? vq : kq;
-    const int32_t *cl = is_v ? cv : ck;
-    const float *sc = is_v ? sv : sk;
-    const int32_t *zp = is_v ? zv : zk;
-    if (src == nullptr) return;
+    constexpr int NG = DPT / 8;
+    const f32x2 magic2 = mk2(MAGIC_RINT, MAGIC_RINT);
+    if (cf.small_z) {
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+            uint32_t acc = 0;
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const int i = gi * 8 + j;
+                // correctly rounded x/s for two channels (reciprocal + one correction)
+                const f32x2 x2 = pair_of<T>(xb[i / VEC], (i % VEC) / 2);
+                const f32x2 q0 = mul2(x2, cf.r2[i / 2]);
+                const f32x2 q1 = fma2(fma2(q0, cf.ns2[i / 2], x2), cf.r2[i / 2], q0);
+                // clamp(rint(q) + z) == rint(clamp(q, -z, qmax - z)) + z
+                const f32x2 qc = mk2(fminf(fmaxf(lo2(q1), cf.lo_[i]), cf.hi_[i]),
+                                     fminf(fmaxf(hi2(q1), cf.lo_[i + 1]), cf.hi_[i + 1]));
+                const f32x2 b2 = add2(qc, magic2);
+                acc += __float_as_uint(lo2(b2)) << (BITS * j);
+                acc += __float_as_uint(hi2(b2)) << (BITS * (j + 1));
+            }
+            grp[gi] = acc - cf.bias[gi];
+        }
+    } else {  // a huge zero point: integer rounding and clamping
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+            uint32_t acc = 0;
+            for (int j = 0; j < 8; ++j) {
+                const int i = gi * 8 + j;
+                const float xf = Elem<T>::get(xb[i / VEC], i % VEC);
+                const float si = (i & 1) ? -hi2(cf.ns2[i / 2]) : -lo2(cf.ns2[i / 2]);
+                const float ri = (i & 1) ? hi2(cf.r2[i / 2]) : lo2(cf.r2[i / 2]);
+                const float q = rintf(div_rn(xf, si, ri));
+                const float c = fminf(fmaxf(q, cf.lo_[i]), cf.hi_[i]) - cf.lo_[i];
+                acc |= (uint32_t)c << (BITS * j);
+            }
+            grp[gi] = acc;
+        }
+    }
+}
 
-    const int bh = blockIdx.x;  // b*H + h
-    const int h = bh % H;
-    const int TPR = D / DPT;    // threads per row
+template <int BITS, int DPT>
+__device__ __forceinline__ void kv_store_row(uint8_t *o, const uint32_t *grp)
+{
+    constexpr int NG = DPT / 8;
+    if constexpr (BITS == 4) {
+        if constexpr (NG == 2)
+            *reinterpret_cast<uint2 *>(o) = make_uint2(grp[0], grp[1]);
+        else
+            *reinterpret_cast<uint32_t *>(o) = grp[0];
+    } else {
+        if constexpr (NG == 2) {  // 6 bytes at an even offset: three 2-byte stores
+            uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
+            o16[0] = (uint16_t)grp[0];
+            o16[1] = (uint16_t)((grp[0] >> 16) | (grp[1] << 8));
+            o16[2] = (uint16_t)(grp[1] >> 8);
+        } else {
+            o[0] = (uint8_t)grp[0];
+            o[1] = (uint8_t)(grp[0] >> 8);
+            o[2] = (uint8_t)(grp[0] >> 16);
+        }
+    }
+}
+
+struct KvTensors {
+    const void *src[2];
+    uint8_t *dst[2];
+    const int32_t *cl[2];
+    const float *sc[2];
+    const int32_t *zp[2];
+};
+
+// Warp kernel: blockIdx.y = tensor (0 = K, 1 = V); contiguous ranges of (h, b, chunk) units per warp.
+template <typename T, int BITS, int DPT>
+__global__ void __launch_bounds__(256, 2)
+    kv_quant_warp(KvTensors t, int B, int H, int S, int D, int g, int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int NLD = DPT / VEC;
+    constexpr int NG = DPT / 8;
+    constexpr int U = 8;  // warp rows-groups whose loads are in flight together
+    const int ti = blockIdx.y;
+    const T *src = static_cast<const T *>(t.src[ti]);
+    if (src == nullptr) return;
+    uint8_t *dst = t.dst[ti];
+    const int lane = threadIdx.x & 31;
+    const int TPR = D / DPT, RPW = 32 / TPR;  // threads per row, rows per warp step
+    const int tl = lane % TPR, lr = lane / TPR, d0 = tl * DPT;
+    const int64_t pitch = (int64_t)D * BITS / 8;
+    const int nchunk = (S + KV_ROWS_PER_UNIT - 1) / KV_ROWS_PER_UNIT;
+    // units in (h, b, chunk) order; warp gw takes the contiguous range [u0, u1), so it crosses
+    // at most a few heads and reloads its coefficients only then
+    const int64_t units = (int64_t)H * B * nchunk, TW = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t u0 = units * gw / TW, u1 = units * (gw + 1) / TW;
+    int64_t hb = u0 / nchunk;  // h * B + b
+    int chunk = (int)(u0 - hb * nchunk);
+    int h = (int)(hb / B), b = (int)(hb - (int64_t)h * B);
+    KvCoef<BITS, DPT> cf;
+    int cur_h = -1;
+    for (int64_t un = u0; un < u1; ++un) {
+        if (h != cur_h) {
+            cf.load(t.cl[ti], t.sc[ti], t.zp[ti], h * D + d0, g, err);
+            cur_h = h;
+        }
+        const int64_t bh = (int64_t)b * H + h;
+        const int r_lo = chunk * KV_ROWS_PER_UNIT, r_hi = min(S, r_lo + KV_ROWS_PER_UNIT);
+        const T *base = src + bh * S * (int64_t)D + d0;
+        uint8_t *obase = dst + bh * S * pitch + (int64_t)tl * (DPT * BITS / 8);
+        for (int s0 = r_lo + lr; s0 < r_hi; s0 += U * RPW) {
+            uint4 xb[U][NLD];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int row = s0 + u * RPW;
+#pragma unroll
+                for (int l = 0; l < NLD; ++l)
+                    xb[u][l] = row < r_hi ? ldg_stream(base + (int64_t)row * D + l * VEC) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int row = s0 + u * RPW;
+                if (row >= r_hi) break;
+                uint32_t grp[NG];
+                kv_quant_row<T, BITS, DPT>(xb[u], cf, grp);
+                kv_store_row<BITS, DPT>(obase + (int64_t)row * pitch, grp);
+            }
+        }
+        if (++chunk == nchunk) {  // next unit
+            chunk = 0;
+            if (++b == B) {
+                b = 0;
+                ++h;
+            }
+        }
+    }
+}
+
+// CTA kernel: blockIdx.x = b*H + h, blockIdx.y = tensor; the CTA streams all S rows of the block.
+template <typename T, int BITS, int DPT>
+__global__ void __launch_bounds__(256)
+    kv_quant_cta(KvTensors t, int H, int64_t S, int D, int g, int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr int NLD = DPT / VEC;
+    constexpr int NG = DPT / 8;
+    constexpr int U = 4;
+    const int ti = blockIdx.y;
+    const T *src = static_cast<const T *>(t.src[ti]);
+    if (src == nullptr) return;
+    uint8_t *dst = t.dst[ti];
+    const int bh = blockIdx.x, h = bh % H;
+    const int TPR = D / DPT;  // threads per row
     const int RPI = blockDim.x / TPR;
     const int tl = threadIdx.x % TPR, rr = threadIdx.x / TPR;
     if (rr >= RPI) return;
     const int d0 = tl * DPT;
-
-    // per-channel divisor s (negated), its reciprocal r, and the code-domain clamp [-z, qmax - z]
-    f32x2 ns2[DPT / 2], r2[DPT / 2];
-    float lo_[DPT], hi_[DPT];
-    uint32_t bias[NG];  // sum_i (MAGIC_BITS - z_i) << (BITS*i): removes the rounding constant
-    bool small_z = true;  // |z| < 2^21 keeps q + 1.5*2^23 inside one binade (exact rounding)
-#pragma unroll
-    for (int gi = 0; gi < NG; ++gi) bias[gi] = 0;
-#pragma unroll
-    for (int i = 0; i < DPT; i += 2) {
-        float sv2[2], rv2[2];
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            int kc = cl[h * D + d0 + i + h2];
-            if (kc < 0 || kc >= g) {
-                raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
-                kc = 0;
-            }
-            sv2[h2] = sc[kc];
-            rv2[h2] = __frcp_rn(sv2[h2]);
-            const int z = zp[kc];
-            lo_[i + h2] = (float)(-z);
-            hi_[i + h2] = (float)(QMAX - z);
-            bias[(i + h2) / 8] += (MAGIC_BITS - (uint32_t)z) << (BITS * ((i + h2) % 8));
-            small_z &= (z > -(1 << 21)) && (z < (1 << 21));
-        }
-        ns2[i / 2] = mk2(-sv2[0], -sv2[1]);
-        r2[i / 2] = mk2(rv2[0], rv2[1]);
-    }
-    const f32x2 magic2 = mk2(MAGIC_RINT, MAGIC_RINT);
+    KvCoef<BITS, DPT> cf;
+    cf.load(t.cl[ti], t.sc[ti], t.zp[ti], h * D + d0, g, err);
     const int64_t pitch = (int64_t)D * BITS / 8;
     const T *base = src + (int64_t)bh * S * D + d0;
     uint8_t *obase = dst + (int64_t)bh * S * pitch + (int64_t)tl * (DPT * BITS / 8);
-
     for (int64_t s0 = rr; s0 < S; s0 += (int64_t)U * RPI) {
         uint4 xb[U][NLD];
 #pragma unroll
@@ -106,81 +254,44 @@ __global__ void __launch_bounds__(256)
             const int64_t row = s0 + (int64_t)u * RPI;
             if (row >= S) break;
             uint32_t grp[NG];
-            if (small_z) {
-#pragma unroll
-                for (int gi = 0; gi < NG; ++gi) {
-                    uint32_t acc = 0;
-#pragma unroll
-                    for (int j = 0; j < 8; j += 2) {
-                        const int i = gi * 8 + j;
-                        // correctly rounded x/s for two channels (reciprocal + one correction)
-                        const f32x2 x2 = pair_of<T>(xb[u][i / VEC], (i % VEC) / 2);
-                        const f32x2 q0 = mul2(x2, r2[i / 2]);
-                        const f32x2 q1 = fma2(fma2(q0, ns2[i / 2], x2), r2[i / 2], q0);
-                        // clamp(rint(q) + z) == rint(clamp(q, -z, qmax - z)) + z
-                        const f32x2 qc = mk2(fminf(fmaxf(lo2(q1), lo_[i]), hi_[i]),
-                                             fminf(fmaxf(hi2(q1), lo_[i + 1]), hi_[i + 1]));
-                        const f32x2 b2 = add2(qc, magic2);
-                        acc += __float_as_uint(lo2(b2)) << (BITS * j);
-                        acc += __float_as_uint(hi2(b2)) << (BITS * (j + 1));
-                    }
-                    grp[gi] = acc - bias[gi];
-                }
-            } else {  // a huge zero point: integer rounding and clamping
-#pragma unroll
-                for (int gi = 0; gi < NG; ++gi) {
-                    uint32_t acc = 0;
-                    for (int j = 0; j < 8; ++j) {
-                        const int i = gi * 8 + j;
-                        const float xf = Elem<T>::get(xb[u][i / VEC], i % VEC);
-                        const float si = (i & 1) ? -hi2(ns2[i / 2]) : -lo2(ns2[i / 2]);
-                        const float ri = (i & 1) ? hi2(r2[i / 2]) : lo2(r2[i / 2]);
-                        const float q = rintf(div_rn(xf, si, ri));
-                        const float c = fminf(fmaxf(q, lo_[i]), hi_[i]) - lo_[i];
-                        acc |= (uint32_t)c << (BITS * j);
-                    }
-                    grp[gi] = acc;
-                }
-            }
-            uint8_t *o = obase + row * pitch;
-            if constexpr (BITS == 4) {
-                if constexpr (NG == 2)
-                    *reinterpret_cast<uint2 *>(o) = make_uint2(grp[0], grp[1]);
-                else
-                    *reinterpret_cast<uint32_t *>(o) = grp[0];
-            } else {
-                if constexpr (NG == 2) {  // 6 bytes at an even offset: three 2-byte stores
-                    uint16_t *o16 = reinterpret_cast<uint16_t *>(o);
-                    o16[0] = (uint16_t)grp[0];
-                    o16[1] = (uint16_t)((grp[0] >> 16) | (grp[1] << 8));
-                    o16[2] = (uint16_t)(grp[1] >> 8);
-                } else {
-                    o[0] = (uint8_t)grp[0];
-                    o[1] = (uint8_t)(grp[0] >> 8);
-                    o[2] = (uint8_t)(grp[0] >> 16);
-                }
-            }
+            kv_quant_row<T, BITS, DPT>(xb[u], cf, grp);
+            kv_store_row<BITS, DPT>(obase + row * pitch, grp);
         }
     }
 }
 
+template <typename T, int BITS>
+static cudaError_t launch_kv_warp(const KvArgs &a)
+{
+    constexpr int DPT = 8;
+    const KvTensors t{{a.k, a.v}, {a.kq, a.vq}, {a.ck, a.cv}, {a.sk, a.sv}, {a.zk, a.zv}};
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kv_quant_warp<T, BITS, DPT>, 256, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t units = (int64_t)a.B * a.H * ((a.S + KV_ROWS_PER_UNIT - 1) / KV_ROWS_PER_UNIT);
+    const int64_t gx = std::max<int64_t>(1, std::min<int64_t>((int64_t)a.num_sms * per_sm / 2, (units + 7) / 8));
+    kv_quant_warp<T, BITS, DPT><<<dim3((unsigned)gx, 2), 256, 0, a.stream>>>(t, a.B, a.H, (int)a.S, a.D, a.g, a.err);
+    return cudaGetLastError();
+}
+
 template <typename T, int BITS, int DPT>
-static cudaError_t launch_kv_t(const KvArgs &a)
+static cudaError_t launch_kv_cta(const KvArgs &a)
 {
     // D <= 2048 (checked by the caller) keeps threads-per-row D / DPT <= 256
-    const int threads = 256;
-    const dim3 grid((unsigned)(a.B * a.H), 2);
-    kv_quant_kernel<T, BITS, DPT><<<grid, threads, 0, a.stream>>>(
-        (const T *)a.k, (const T *)a.v, a.H, a.S, a.D, a.ck, a.sk, a.zk, a.cv, a.sv, a.zv, a.g, a.kq,
-        a.vq, a.err);
+    const KvTensors t{{a.k, a.v}, {a.kq, a.vq}, {a.ck, a.cv}, {a.sk, a.sv}, {a.zk, a.zv}};
+    kv_quant_cta<T, BITS, DPT><<<dim3((unsigned)(a.B * a.H), 2), 256, 0, a.stream>>>(t, a.H, a.S, a.D, a.g, a.err);
     return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_kv_d(const KvArgs &a)
 {
-    if (a.D % 16 == 0) return a.bits == 4 ? launch_kv_t<T, 4, 16>(a) : launch_kv_t<T, 3, 16>(a);
-    return a.bits == 4 ? launch_kv_t<T, 4, 8>(a) : launch_kv_t<T, 3, 8>(a);
+    // warp kernel when the 8-channel groups of a row tile a warp evenly (D in 8, 16, ..., 256)
+    if (a.D % 8 == 0 && a.D <= 256 && 32 % (a.D / 8) == 0 && a.S <= 0x7fffffffLL)
+        return a.bits == 4 ? launch_kv_warp<T, 4>(a) : launch_kv_warp<T, 3>(a);
+    if (a.D % 16 == 0) return a.bits == 4 ? launch_kv_cta<T, 4, 16>(a) : launch_kv_cta<T, 3, 16>(a);
+    return a.bits == 4 ? launch_kv_cta<T, 4, 8>(a) : launch_kv_cta<T, 3, 8>(a);
 }
 
 cudaError_t launch_kv_quant(const KvArgs &a)

@@ -67,6 +67,7 @@ struct KvArgs {
     uint8_t *kq, *vq;
     int *err;
     cudaStream_t stream;
+    int num_sms;
 };
 
 struct DequantArgs {

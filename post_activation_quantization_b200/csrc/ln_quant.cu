@@ -32,7 +32,7 @@
 namespace rptq {
 
 // ------------------------------------------------------------------------------------------
-template <typename T, int BITS, int CPT, bool EXACT>
+template <typename T, int BITS, int CPT>
 __global__ void __launch_bounds__(512, 1)
     ln_quant_fast_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
                          const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
@@ -96,10 +96,7 @@ __global__ void __launch_bounds__(512, 1)
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += gridDim.x, ++lq) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
-        if (EXACT && nrows == 4)  // every chunk of every row is inside the tensor
-            pipe.load_full(xr);
-        else
-            pipe.load(nrows, xr);
+        pipe.load(nrows, xr);
         float rstd[4], nmr[4];
         quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, !alias);
         if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
@@ -111,7 +108,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int k = 0; k < CPT; ++k) {
             const int ch = tid + k * NT;
-            if (!EXACT && ch >= NCH) continue;
+            if (ch >= NCH) continue;
             uint32_t pw[VEC / 2];  // stored positions of the chunk's channels, two u16 per word
             if constexpr (VEC == 8) {
                 const uint4 p = *reinterpret_cast<const uint4 *>(postab + ch * 8);
@@ -282,8 +279,7 @@ static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias
 {
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
     const QuadSmem L = quad_smem_layout(NS, rowbytes, (alias ? 0 : (size_t)a.C * 4) + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
-    const bool exact = (a.C / (int)Elem<T>::VEC) == CPT * NT;  // chunks split evenly over threads
-    auto kern = exact ? ln_quant_fast_kernel<T, BITS, CPT, true> : ln_quant_fast_kernel<T, BITS, CPT, false>;
+    auto kern = ln_quant_fast_kernel<T, BITS, CPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

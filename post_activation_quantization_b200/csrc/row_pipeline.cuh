@@ -84,20 +84,6 @@ struct QuadRows {
             }
         }
     }
-    // The same for a full quad whose chunks are all inside the row (no predicates).
-    __device__ __forceinline__ void load_full(uint4 (&xr)[4][CPT]) const
-    {
-        const int tid = threadIdx.x, NT = blockDim.x;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            uint32_t s, ph;
-            where(r, s, ph);
-            mbar_wait_bounded(bar0 + 8u * s, ph, err);
-            const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)s * rowbytes) + tid;
-#pragma unroll
-            for (int k = 0; k < CPT; ++k) xr[r][k] = src[k * NT];
-        }
-    }
     // thread 0 after the quad's last read of its slots: refill them with the rows NS ahead
     __device__ __forceinline__ void refill(int64_t lq) const
     {

@@ -200,7 +200,8 @@ def test_kv_calib_bit_exact(dtype, B, H, S, D):
 
 
 KV_CASES = [("f16", 2, 4, 33, 128, 6, 3), ("bf16", 1, 3, 17, 64, 5, 4), ("f32", 2, 2, 9, 128, 8, 4),
-            ("f16", 1, 2, 11, 40, 4, 3), ("bf16", 3, 5, 7, 256, 7, 3)]
+            ("f16", 1, 2, 11, 40, 4, 3), ("bf16", 3, 5, 7, 256, 7, 3), ("bf16", 2, 3, 300, 128, 6, 3),
+            ("f16", 1, 2, 5, 512, 4, 4), ("bf16", 2, 2, 130, 32, 5, 3), ("f32", 1, 3, 19, 8, 3, 4)]
 
 
 @pytest.mark.parametrize("dtype,B,H,S,D,g,bits", KV_CASES)
@@ -230,7 +231,8 @@ def test_kv_quant(dtype, B, H, S, D, g, bits):
 
 # ---------------------------------------------------------------- dequantization
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.float16, torch.bfloat16])
-@pytest.mark.parametrize("rows,C,bits", [(37, 768, 4), (5, 4096, 3), (3, 72, 3), (2, 40, 4)])
+@pytest.mark.parametrize("rows,C,bits", [(37, 768, 4), (5, 4096, 3), (3, 72, 3), (2, 40, 4), (9, 12288, 3),
+                                         (6, 12288, 4), (11, 9216, 3), (4, 256, 3), (3, 16384, 4)])
 def test_dequant_rows_bit_exact(out_dtype, rows, C, bits):
     rng = np.random.default_rng(rows * C)
     g = 9
@@ -247,13 +249,18 @@ def test_dequant_rows_bit_exact(out_dtype, rows, C, bits):
     assert torch.equal(out.cpu(), ref)
 
 
-@pytest.mark.parametrize("B,H,S,D,bits", [(2, 3, 5, 128, 3), (1, 2, 4, 40, 4), (1, 4, 3, 64, 4)])
-def test_dequant_bhsd_bit_exact(B, H, S, D, bits):
+@pytest.mark.parametrize("B,H,S,D,bits", [(2, 3, 5, 128, 3), (1, 2, 4, 40, 4), (1, 4, 3, 64, 4), (2, 2, 67, 128, 3),
+                                          (1, 3, 9, 256, 4), (2, 1, 35, 8, 3), (2, 1, 36, 8, 3), (1, 2, 13, 32, 3),
+                                          (1, 1, 16, 16, 4)])
+@pytest.mark.parametrize("huge_z", [False, True])
+def test_dequant_bhsd_bit_exact(B, H, S, D, bits, huge_z):
     rng = np.random.default_rng(B * H * S * D)
     g = 6
     labels = rng.integers(0, g, H * D).astype(np.int32)
     s = rng.lognormal(-2, 1, g).astype(np.float32)
     z = rng.integers(-30, 30, g).astype(np.int32)
+    if huge_z:
+        z[labels[0]] = -9_000_000  # beyond the exact float path
     q = rng.integers(0, 2 ** bits, (B * H * S, D)).astype(np.uint8)
     packed = oracle.pack(q, bits).reshape(B, H, S, D * bits // 8)
     out = rptq.rptq_dequant(torch.from_numpy(packed).to(DEV), torch.from_numpy(labels).to(DEV),
