@@ -257,18 +257,32 @@ __global__ void __launch_bounds__(512, 1)
         pipe.load(nrows, xr);
         float rstd[4], nmr[4];
         quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
+        if (nrows == 4) {  // normalised values of tokens (0, 1) and (2, 3) two lanes at a time
+            const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
+            const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
 #pragma unroll
-        for (int k = 0; k < CPT; ++k)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                if (r >= nrows) break;
+            for (int k = 0; k < CPT; ++k)
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
-                    const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
-                    tmax[k][e] = fmaxf(tmax[k][e], t);
-                    tmin[k][e] = fminf(tmin[k][e], t);
+                    const f32x2 t01 = fma2(mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e)), rs01, nm01);
+                    const f32x2 t23 = fma2(mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e)), rs23, nm23);
+                    tmax[k][e] = max3f(max3f(tmax[k][e], lo2(t01), hi2(t01)), lo2(t23), hi2(t23));
+                    tmin[k][e] = min3f(min3f(tmin[k][e], lo2(t01), hi2(t01)), lo2(t23), hi2(t23));
                 }
-            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < CPT; ++k)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    if (r >= nrows) break;
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
+                        tmax[k][e] = fmaxf(tmax[k][e], t);
+                        tmin[k][e] = fminf(tmin[k][e], t);
+                    }
+                }
+        }
         pipe.advance();
     }
     if (lq == 0) return;  // this CTA saw no rows

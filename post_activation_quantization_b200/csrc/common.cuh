@@ -93,6 +93,20 @@ template <> __device__ __forceinline__ void chunk_moments<__half>(const uint4 &v
 }
 
 // Streaming 16-byte global load that does not allocate in L1.
+// three-input max / min (one instruction on sm_100; NaN operands are ignored like fmaxf/fminf)
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float min3f(float a, float b, float c)
+{
+    float r;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 32-bit read-once load (no L1 allocation)
 __device__ __forceinline__ uint32_t ldg_stream32(const void *p)
 {
