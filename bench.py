@@ -290,7 +290,7 @@ def run_rptq(args):
           for n, _, _ in stages}
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clk = Clocks(dev.index) if rank == 0 else None
-    for _ in range(n_pre):  # the sampler starts while the GPU runs these, so it is up when timing starts
+    for _ in range(n_pre if args.clock_warmup else 0):  # the sampler starts while these run
         step.run()
     torch.cuda.synchronize()
     if ws > 1:
@@ -542,6 +542,8 @@ def main():
     ap.add_argument("--ref-frac", type=float, default=1 / 32,
                     help="fraction of the tokens per step of the --impl reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clock-warmup", dest="clock_warmup", action="store_false",
+                    help="skip the untimed steps that let the clock sampler start (profiling runs)")
     ap.add_argument("--token-scale", type=float, default=1.0,
                     help="shrink the token counts (a small case for ncu captures; not a bench config)")
     args = ap.parse_args()
