@@ -32,42 +32,31 @@
 namespace rptq {
 
 // ------------------------------------------------------------------------------------------
-template <typename T, int BITS, int CPT>
-__global__ void __launch_bounds__(512, 1)
-    ln_quant_fast_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
-                         const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
-                         const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
-                         const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int NS,
-                         int alias, int *err)
+// Pieces shared by the two fast kernels.
+
+// Per-channel tables: postab[c] = code-buffer offset of channel c's stored column, and the
+// thread's affine coefficients pA, pB for its chunks (tid + k*NT).
+template <typename T, int BITS, int CPT, typename P>
+__device__ __forceinline__ void quant_tables(const int32_t *R, const int32_t *col_cluster, const float *scale,
+                                             const int32_t *zero, const float *gamma, const float *beta, int g, int C,
+                                             P *postab, uint32_t pbase, float (&pA)[CPT][Elem<T>::VEC],
+                                             float (&pB)[CPT][Elem<T>::VEC], int *err)
 {
+    // postab[c] = pbase + code-buffer offset of channel c's stored column (P = uint16_t: the
+    // offset alone; P = uint32_t: the shared-memory address of the word)
     constexpr int VEC = Elem<T>::VEC;
     constexpr float QMAX = (float)((1 << BITS) - 1);
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int tid = threadIdx.x, NT = blockDim.x;
-    const int NCH = C / VEC;
-    const uint32_t rowbytes = (uint32_t)C * sizeof(T);
-    const size_t cb_bytes = alias ? 0 : (size_t)C * 4;
-    const QuadSmem L = quad_smem_layout(NS, rowbytes, cb_bytes + (size_t)C * 2 + 2 * 8 * 32 * 4);
-    uint8_t *codebuf = smem + L.extra_off;                                    // 4*C bytes (own)
-    uint16_t *postab = reinterpret_cast<uint16_t *>(smem + L.extra_off + cb_bytes);  // 2*C bytes
-    float *red = reinterpret_cast<float *>(postab + C);                      // 8*32 floats
-    float *red2 = red + 8 * 32;
-
-    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
-    pipe.start();
-
-    // ---- per-channel tables: stored position (code-buffer offset) and affine coefficients
-    for (int c = tid; c < C; c += NT) postab[c] = 0;
+    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC;
+    for (int c = tid; c < C; c += NT) postab[c] = (P)pbase;
     __syncthreads();
     for (int j = tid; j < C; j += NT) {
         const int c = R[j];
         if (c >= 0 && c < C)
-            postab[c] = (uint16_t)codebuf_offset((uint32_t)j);
+            postab[c] = (P)(pbase + codebuf_offset((uint32_t)j));
         else
             raise_error(err, RPTQ_DEVERR_REORDER);
     }
     __syncthreads();
-    float pA[CPT][VEC], pB[CPT][VEC];
 #pragma unroll
     for (int k = 0; k < CPT; ++k) {
         const int ch = tid + k * NT;
@@ -77,7 +66,7 @@ __global__ void __launch_bounds__(512, 1)
             pB[k][e] = 0.f;
             if (ch < NCH) {
                 const int c = ch * VEC + e;
-                const int j = (int)codebuf_index(postab[c]);
+                const int j = (int)codebuf_index((uint32_t)postab[c] - pbase);
                 int kc = col_cluster[j];
                 if (kc < 0 || kc >= g) {
                     raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
@@ -89,6 +78,131 @@ __global__ void __launch_bounds__(512, 1)
             }
         }
     }
+}
+
+// Codes of the quad's four tokens for every channel of the thread -> one word per channel at
+// its stored position in the code buffer.
+template <typename T, int BITS, int CPT, bool ABS>
+__device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const float (&rstd)[4], const float (&nmr)[4],
+                                              const float (&pA)[CPT][Elem<T>::VEC],
+                                              const float (&pB)[CPT][Elem<T>::VEC], const void *postab,
+                                              uint8_t *codebuf, int NCH)
+{
+    // ABS: postab holds 32-bit shared-memory addresses (stored directly, no extraction);
+    // otherwise 16-bit offsets into codebuf, two per word
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr float QMAX = (float)((1 << BITS) - 1);
+    const int tid = threadIdx.x, NT = blockDim.x;
+    const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
+    const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
+    const f32x2 qm2 = mk2(QMAX, QMAX), mg2 = mk2(MAGIC_RINT, MAGIC_RINT);
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+        const int ch = tid + k * NT;
+        if (ch >= NCH) continue;
+        uint32_t pw[ABS ? VEC : VEC / 2];
+        if constexpr (ABS) {
+            const uint4 *p4 = reinterpret_cast<const uint4 *>(static_cast<const uint32_t *>(postab) + ch * VEC);
+#pragma unroll
+            for (int i = 0; i < VEC / 4; ++i) {
+                const uint4 p = p4[i];
+                pw[4 * i] = p.x, pw[4 * i + 1] = p.y, pw[4 * i + 2] = p.z, pw[4 * i + 3] = p.w;
+            }
+        } else if constexpr (VEC == 8) {
+            const uint4 p = *reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(postab) + ch * 8);
+            pw[0] = p.x, pw[1] = p.y, pw[2] = p.z, pw[3] = p.w;
+        } else {
+            const uint2 p = *reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(postab) + ch * 4);
+            pw[0] = p.x, pw[1] = p.y;
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            // normalised values of channel e for tokens (0,1) and (2,3), two lanes at a time
+            const f32x2 t01 = fma2(mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e)), rs01, nm01);
+            const f32x2 t23 = fma2(mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e)), rs23, nm23);
+            const float A = pA[k][e], Bc = pB[k][e];
+            // u = sat(y / (s qmax) + z / qmax); code = rint(u qmax) (the 1.5*2^23 rounding add)
+            const f32x2 u01 = mk2(fma_sat(lo2(t01), A, Bc), fma_sat(hi2(t01), A, Bc));
+            const f32x2 u23 = mk2(fma_sat(lo2(t23), A, Bc), fma_sat(hi2(t23), A, Bc));
+            const f32x2 b01 = fma2(u01, qm2, mg2), b23 = fma2(u23, qm2, mg2);
+            const uint32_t word = prmt(prmt(__float_as_uint(lo2(b01)), __float_as_uint(hi2(b01)), 0x0040),
+                                       prmt(__float_as_uint(lo2(b23)), __float_as_uint(hi2(b23)), 0x0040), 0x5410);
+            if constexpr (ABS) {
+                asm volatile("st.shared.b32 [%0], %1;" ::"r"(pw[e]), "r"(word) : "memory");
+            } else {
+                const uint32_t pos = (e & 1) ? (pw[e >> 1] >> 16) : (pw[e >> 1] & 0xffffu);
+                *reinterpret_cast<uint32_t *>(codebuf + pos) = word;
+            }
+        }
+    }
+}
+
+// Pack 32 stored positions x 4 tokens per thread from the code buffer and write whole words of
+// rows 4*gq .. 4*gq + nrows - 1.
+template <int BITS>
+__device__ __forceinline__ void pack_store(const uint8_t *codebuf, uint8_t *codes, int64_t gq, int64_t pitch, int nrows,
+                                           int NU)
+{
+    for (int u = threadIdx.x; u < NU; u += blockDim.x) {
+        uint32_t o[4][4];  // [group m of 8 positions][token r]
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            uint32_t w[8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t slot = 8u * u + ((2 * m + h) ^ (u & 7));
+                const uint4 q = *reinterpret_cast<const uint4 *>(codebuf + (slot << 4));
+                w[4 * h + 0] = q.x;
+                w[4 * h + 1] = q.y;
+                w[4 * h + 2] = q.z;
+                w[4 * h + 3] = q.w;
+            }
+            if constexpr (BITS == 4)
+                pack8x4_a4(w, o[m]);
+            else
+                pack8x4_a3(w, o[m]);
+        }
+        uint8_t *dst = codes + 4 * gq * pitch + (BITS == 4 ? 16 : 12) * (int64_t)u;
+#pragma unroll
+        for (int r = 0; r < 4; ++r, dst += pitch) {
+            if (r >= nrows) break;
+            if constexpr (BITS == 4) {
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0][r], o[1][r], o[2][r], o[3][r]);
+            } else {
+                uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
+                d32[0] = o[0][r] | (o[1][r] << 24);
+                d32[1] = (o[1][r] >> 8) | (o[2][r] << 16);
+                d32[2] = (o[2][r] >> 16) | (o[3][r] << 8);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Fast kernel, rows staged through the shared-memory ring (row_pipeline.cuh).
+template <typename T, int BITS, int CPT>
+__global__ void __launch_bounds__(512, 1)
+    ln_quant_fast_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                         const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
+                         const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                         const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int NS,
+                         int alias, int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int NCH = C / VEC;
+    const uint32_t rowbytes = (uint32_t)C * sizeof(T);
+    const size_t cb_bytes = alias ? 0 : (size_t)C * 4;
+    const QuadSmem L = quad_smem_layout(NS, rowbytes, cb_bytes + (size_t)C * 2 + 2 * 8 * 32 * 4);
+    uint8_t *codebuf = smem + L.extra_off;                                    // 4*C bytes (own)
+    uint16_t *postab = reinterpret_cast<uint16_t *>(smem + L.extra_off + cb_bytes);  // 2*C bytes
+    float *red = reinterpret_cast<float *>(postab + C);                      // 8*32 floats
+    float *red2 = red + 8 * 32;
+
+    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
+    pipe.start();
+    float pA[CPT][VEC], pB[CPT][VEC];
+    quant_tables<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, 0u, pA, pB, err);
 
     const int64_t pitch = (int64_t)C * BITS / 8;
     const int NU = C >> 5;  // 32-position pack units
@@ -100,81 +214,103 @@ __global__ void __launch_bounds__(512, 1)
         float rstd[4], nmr[4];
         quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, !alias);
         if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
-
-        // ---- codes of four tokens per channel -> one word at the channel's stored position
-        const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
-        const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
-        const f32x2 qm2 = mk2(QMAX, QMAX), mg2 = mk2(MAGIC_RINT, MAGIC_RINT);
-#pragma unroll
-        for (int k = 0; k < CPT; ++k) {
-            const int ch = tid + k * NT;
-            if (ch >= NCH) continue;
-            uint32_t pw[VEC / 2];  // stored positions of the chunk's channels, two u16 per word
-            if constexpr (VEC == 8) {
-                const uint4 p = *reinterpret_cast<const uint4 *>(postab + ch * 8);
-                pw[0] = p.x, pw[1] = p.y, pw[2] = p.z, pw[3] = p.w;
-            } else {
-                const uint2 p = *reinterpret_cast<const uint2 *>(postab + ch * 4);
-                pw[0] = p.x, pw[1] = p.y;
-            }
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                // normalised values of channel e for tokens (0,1) and (2,3), two lanes at a time
-                const f32x2 t01 = fma2(mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e)), rs01, nm01);
-                const f32x2 t23 = fma2(mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e)), rs23, nm23);
-                const float A = pA[k][e], Bc = pB[k][e];
-                // u = sat(y / (s qmax) + z / qmax); code = rint(u qmax) (the 1.5*2^23 rounding add)
-                const f32x2 u01 = mk2(fma_sat(lo2(t01), A, Bc), fma_sat(hi2(t01), A, Bc));
-                const f32x2 u23 = mk2(fma_sat(lo2(t23), A, Bc), fma_sat(hi2(t23), A, Bc));
-                const f32x2 b01 = fma2(u01, qm2, mg2), b23 = fma2(u23, qm2, mg2);
-                const uint32_t word = prmt(prmt(__float_as_uint(lo2(b01)), __float_as_uint(hi2(b01)), 0x0040),
-                                           prmt(__float_as_uint(lo2(b23)), __float_as_uint(hi2(b23)), 0x0040),
-                                           0x5410);
-                const uint32_t pos = (e & 1) ? (pw[e >> 1] >> 16) : (pw[e >> 1] & 0xffffu);
-                *reinterpret_cast<uint32_t *>(codebuf + pos) = word;
-            }
-        }
+        quant_scatter<T, BITS, CPT, false>(xr, rstd, nmr, pA, pB, postab, codebuf, NCH);
         __syncthreads();
-
-        // ---- pack 32 stored positions x 4 tokens per thread, write whole words
-        for (int u = tid; u < NU; u += NT) {
-            uint32_t o[4][4];  // [group m of 8 positions][token r]
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint32_t w[8];
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const uint32_t slot = 8u * u + ((2 * m + h) ^ (u & 7));
-                    const uint4 q = *reinterpret_cast<const uint4 *>(codebuf + (slot << 4));
-                    w[4 * h + 0] = q.x;
-                    w[4 * h + 1] = q.y;
-                    w[4 * h + 2] = q.z;
-                    w[4 * h + 3] = q.w;
-                }
-                if constexpr (BITS == 4)
-                    pack8x4_a4(w, o[m]);
-                else
-                    pack8x4_a3(w, o[m]);
-            }
-            uint8_t *dst = codes + 4 * gq * pitch + (BITS == 4 ? 16 : 12) * (int64_t)u;
-#pragma unroll
-            for (int r = 0; r < 4; ++r, dst += pitch) {
-                if (r >= nrows) break;
-                if constexpr (BITS == 4) {
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0][r], o[1][r], o[2][r], o[3][r]);
-                } else {
-                    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
-                    d32[0] = o[0][r] | (o[1][r] << 24);
-                    d32[1] = (o[1][r] >> 8) | (o[2][r] << 16);
-                    d32[2] = (o[2][r] >> 16) | (o[3][r] << 8);
-                }
-            }
-        }
+        pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU);
         if (alias) {  // the quad's slots held its codes until now
             __syncthreads();
             pipe.refill(lq);
         }
         pipe.advance();
+    }
+}
+
+// Direct kernel: rows go from global memory straight to registers (coalesced 16-byte loads),
+// with the DRAM stream kept ahead by bulk L2 prefetches of whole quads (four contiguous rows,
+// one instruction, two quads ahead); the next quad's loads are issued as soon as the current
+// quad's rows are dead (after the scatter), so they fly during the pack.  Shared memory holds
+// only the code buffer and the tables (the stored positions as 32-bit shared addresses).
+struct NoRefill {
+    __device__ __forceinline__ void refill(int64_t) const {}
+};
+
+template <typename T, int CPT>
+__device__ __forceinline__ void load_quad_direct(const T *x, int64_t T_, int C, int64_t gq, bool exact,
+                                                 uint4 (&xr)[4][CPT])
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC;
+    const T *src = x + 4 * gq * (int64_t)C + tid * VEC;
+    if (exact && 4 * gq + 4 <= T_) {  // a full quad and every chunk inside the row: no predicates
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int k = 0; k < CPT; ++k) xr[r][k] = ldg_stream(src + (int64_t)r * C + k * NT * VEC);
+        return;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int64_t row = 4 * gq + r;
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+            const int ch = tid + k * NT;
+            xr[r][k] = (row < T_ && ch < NCH) ? ldg_stream(src + (int64_t)r * C + k * NT * VEC) : make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ void prefetch_quad_l2(const void *x, int64_t T_, uint32_t rowbytes, int64_t gq)
+{
+    if (threadIdx.x == 0 && 4 * gq < T_) {
+        const int64_t n = (T_ - 4 * gq < 4 ? T_ - 4 * gq : 4) * (int64_t)rowbytes;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const uint8_t *>(x) +
+                                                                          4 * gq * (int64_t)rowbytes),
+                     "r"((uint32_t)n)
+                     : "memory");
+    }
+}
+
+// 512 threads for up to 3 chunks per thread, 384 threads (more registers) for 4
+template <typename T, int BITS, int CPT>
+__global__ void __launch_bounds__(CPT <= 3 ? 512 : 384, 1)
+    ln_quant_direct_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+                           const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
+                           const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                           const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int NCH = C / VEC;
+    const uint32_t rowbytes = (uint32_t)C * sizeof(T);
+    uint8_t *codebuf = smem;                                                    // 4*C bytes
+    uint32_t *postab = reinterpret_cast<uint32_t *>(smem + (size_t)C * 4);     // 4*C bytes
+    float *red = reinterpret_cast<float *>(postab + C);                        // 8*32 floats
+    float *red2 = red + 8 * 32;
+    const int64_t G = gridDim.x;
+    const bool exact = NCH == CPT * (int)blockDim.x;  // the chunks split evenly over the threads
+    prefetch_quad_l2(x, T_, rowbytes, blockIdx.x);
+    prefetch_quad_l2(x, T_, rowbytes, blockIdx.x + G);
+    float pA[CPT][VEC], pB[CPT][VEC];
+    quant_tables<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, smem_u32(codebuf), pA, pB,
+                               err);
+
+    const int64_t pitch = (int64_t)C * BITS / 8;
+    const int NU = C >> 5;
+    const NoRefill none;
+    uint4 xr[4][CPT];
+    load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr);
+    for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += G) {
+        const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
+        float rstd[4], nmr[4];
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, none, 0, rstd, nmr, false);
+        quant_scatter<T, BITS, CPT, true>(xr, rstd, nmr, pA, pB, postab, codebuf, NCH);
+        // the rows are dead: next quad's loads fly during the pack, and one more quad to L2
+        load_quad_direct<T, CPT>(x, T_, C, gq + G, exact, xr);
+        prefetch_quad_l2(x, T_, rowbytes, gq + 2 * G);
+        __syncthreads();
+        pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU);
+        // the next quad's scatter overwrites the code buffer only after the barrier inside its
+        // LayerNorm statistics, which every thread reaches after this pack
     }
 }
 
@@ -275,6 +411,24 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------------------------------
 
 template <typename T, int BITS, int CPT>
+static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
+{
+    const size_t smem = (size_t)a.C * 8 + 2 * 8 * 32 * 4;
+    auto kern = ln_quant_direct_kernel<T, BITS, CPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t quads = (a.T + 3) / 4;
+    const int64_t grid = std::min<int64_t>(quads, (int64_t)per_sm * a.num_sms);
+    kern<<<(unsigned)grid, NT, smem, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps, a.R,
+                                                 a.col_cluster, a.scale, a.zero, a.g, a.codes, a.err);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS, int CPT>
 static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias)
 {
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
@@ -297,6 +451,15 @@ static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias
 template <typename T, int BITS>
 static cudaError_t launch_fast_b(const LnQuantArgs &a, int CPT, int NT, int NS, int alias)
 {
+    if (alias == 2) {
+        switch (CPT) {
+        case 1: return launch_direct_t<T, BITS, 1>(a, NT);
+        case 2: return launch_direct_t<T, BITS, 2>(a, NT);
+        case 3: return launch_direct_t<T, BITS, 3>(a, NT);
+        case 4: return launch_direct_t<T, BITS, 4>(a, NT);
+        default: return cudaErrorInvalidValue;
+        }
+    }
     switch (CPT) {
     case 1: return launch_fast_t<T, BITS, 1>(a, NT, NS, alias);
     case 2: return launch_fast_t<T, BITS, 2>(a, NT, NS, alias);
@@ -311,8 +474,10 @@ static cudaError_t launch_fast_d(const LnQuantArgs &a, int CPT, int NT, int NS, 
     return a.bits == 4 ? launch_fast_b<T, 4>(a, CPT, NT, NS, alias) : launch_fast_b<T, 3>(a, CPT, NT, NS, alias);
 }
 
-// Plan of the fast kernel for (C, dtype): threads, chunks per thread and ring depth;
-// returns false when the shape needs the simple kernel.
+// Plan of the fast kernels for (C, dtype): threads, chunks per thread and, for the ring kernel,
+// ring depth and code-buffer placement (*alias = 0: own buffer, 1: in the quad's slots);
+// *alias = 2 selects the direct kernel (no ring).  Returns false when the shape needs the
+// simple kernel.
 bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS, int *alias)
 {
     if (C % 32 != 0) return false;
@@ -326,6 +491,23 @@ bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *
             nt = n;
             break;
         }
+    }
+    if ((size_t)C * 8 + 2 * 8 * 32 * 4 <= (size_t)max_smem) {  // direct kernel
+        // 384 threads x 4 chunks when that splits the row exactly (every thread also packs one
+        // 32-position unit), else the ring kernel's choice of up to 512 threads
+        int dc = cpt, dn = nt;
+#ifndef RPTQ_DIRECT_512
+        if (NCH % (4 * 32) == 0 && NCH / 4 <= 384 && NCH / 4 >= 256) {
+            dc = 4;
+            dn = NCH / 4;
+        }
+#endif
+        if (!dc) return false;
+        *CPT = dc;
+        *NT = dn;
+        *NS = 0;
+        *alias = 2;
+        return true;
     }
     if (!cpt) return false;
     const uint32_t rowbytes = (uint32_t)C * esize;

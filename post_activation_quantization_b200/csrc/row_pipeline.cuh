@@ -84,13 +84,13 @@ struct QuadRows {
             }
         }
     }
-    // thread 0 after the quad's last read of its slots: refill them with the rows NS ahead
-    __device__ __forceinline__ void refill(int64_t lq) const
+    // thread 0 after the quad's last read of its slots r0 .. r1-1: refill them with the rows NS
+    // ahead
+    __device__ __forceinline__ void refill(int64_t lq, int r0 = 0, int r1 = 4) const
     {
         if (threadIdx.x == 0) {
             fence_proxy_async_smem();
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
+            for (int r = r0; r < r1; ++r) {
                 uint32_t s, ph;
                 where(r, s, ph);
                 issue(4 * lq + NS + r, s);  // the same slot, NS rows later
