@@ -105,7 +105,7 @@ struct KmArgs {
 
 // force_simple = 1 routes codes-only calls to the general kernel (used by tests of that path)
 cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple);
-bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS, int *alias);
+bool ln_quant_fast_plan(int C, int esize, int max_smem, bool allow_direct, int *CPT, int *NT, int *NS, int *alias);
 cudaError_t launch_calib(const CalibArgs &a);
 cudaError_t launch_kv_calib(const KvCalibArgs &a);
 cudaError_t launch_kv_quant(const KvArgs &a);

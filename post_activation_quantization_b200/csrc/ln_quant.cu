@@ -80,6 +80,93 @@ __device__ __forceinline__ void quant_tables(const int32_t *R, const int32_t *co
     }
 }
 
+// The same tables for the direct kernel, built with coalesced loads: one pass over the stored
+// columns j (R and col_cluster read as int4) records each channel's code-buffer address and
+// cluster; a per-cluster table holds 1 / (s qmax) and z / qmax in fp64, so a channel's
+// coefficients are one multiply and one fused multiply-add (A = gamma / (s qmax),
+// B = beta / (s qmax) + z / qmax).  Needs C % 4 == 0 and 16-byte aligned R, col_cluster,
+// gamma and beta.
+template <typename T, int BITS, int CPT>
+__device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int32_t *col_cluster, const float *scale,
+                                                    const int32_t *zero, const float *gamma, const float *beta,
+                                                    int g, int C, uint32_t *postab, uint16_t *ctab, double *ctl,
+                                                    uint32_t pbase, float (&pA)[CPT][Elem<T>::VEC],
+                                                    float (&pB)[CPT][Elem<T>::VEC], int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    constexpr double QMAX = (double)((1 << BITS) - 1);
+    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC;
+    for (int c = tid; c < C; c += NT) {
+        postab[c] = pbase;
+        ctab[c] = 0;
+    }
+    for (int k = tid; k < g; k += NT) {
+        const double s = (double)scale[k] * QMAX;
+        ctl[2 * k] = 1.0 / s;
+        ctl[2 * k + 1] = (double)zero[k] / QMAX;
+    }
+    __syncthreads();
+    const int4 *R4 = reinterpret_cast<const int4 *>(R);
+    const int4 *K4 = reinterpret_cast<const int4 *>(col_cluster);
+    const int C4 = C / 4;
+    for (int b0 = tid; b0 < C4; b0 += 4 * NT) {  // four int4 of R and of col_cluster in flight
+        int4 r[4], kk[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j4 = b0 + u * NT;
+            r[u] = j4 < C4 ? R4[j4] : make_int4(-1, -1, -1, -1);
+            kk[u] = j4 < C4 ? K4[j4] : make_int4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j4 = b0 + u * NT;
+            if (j4 >= C4) continue;
+            const int rv[4] = {r[u].x, r[u].y, r[u].z, r[u].w}, kv[4] = {kk[u].x, kk[u].y, kk[u].z, kk[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = rv[i], k = kv[i];
+                if (c >= 0 && c < C) {
+                    postab[c] = pbase + codebuf_offset((uint32_t)(4 * j4 + i));
+                    ctab[c] = (uint16_t)((k >= 0 && k < g) ? k : 0);
+                } else {
+                    raise_error(err, RPTQ_DEVERR_REORDER);
+                }
+                if (k < 0 || k >= g) raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+            }
+        }
+    }
+    __syncthreads();
+    // gamma, beta of the thread's chunks as 16-byte loads, all in flight before the arithmetic
+    float4 gm[CPT][VEC / 4], bt[CPT][VEC / 4];
+#pragma unroll
+    for (int kc = 0; kc < CPT; ++kc) {
+        const int ch = tid + kc * NT;
+#pragma unroll
+        for (int q = 0; q < VEC / 4; ++q) {
+            gm[kc][q] = ch < NCH ? __ldg(reinterpret_cast<const float4 *>(gamma + ch * VEC) + q) : make_float4(0, 0, 0, 0);
+            bt[kc][q] = ch < NCH ? __ldg(reinterpret_cast<const float4 *>(beta + ch * VEC) + q) : make_float4(0, 0, 0, 0);
+        }
+    }
+#pragma unroll
+    for (int kc = 0; kc < CPT; ++kc) {
+        const int ch = tid + kc * NT;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            const float4 g4 = gm[kc][e / 4], b4 = bt[kc][e / 4];
+            const float gv = (e & 3) == 0 ? g4.x : (e & 3) == 1 ? g4.y : (e & 3) == 2 ? g4.z : g4.w;
+            const float bv = (e & 3) == 0 ? b4.x : (e & 3) == 1 ? b4.y : (e & 3) == 2 ? b4.z : b4.w;
+            pA[kc][e] = 0.f;
+            pB[kc][e] = 0.f;
+            if (ch < NCH) {
+                const int k = ctab[ch * VEC + e];
+                const double inv = ctl[2 * k];
+                pA[kc][e] = (float)((double)gv * inv);
+                pB[kc][e] = (float)fma((double)bv, inv, ctl[2 * k + 1]);
+            }
+        }
+    }
+}
+
 // Codes of the quad's four tokens for every channel of the thread -> one word per channel at
 // its stored position in the code buffer.
 template <typename T, int BITS, int CPT, bool ABS>
@@ -270,6 +357,12 @@ __device__ __forceinline__ void prefetch_quad_l2(const void *x, int64_t T_, uint
     }
 }
 
+// code buffer 4C | positions 4C | reductions 2 KB | cluster table 16 g | channel clusters 2C
+static inline size_t direct_smem_bytes(int C, int g)
+{
+    return (size_t)C * 10 + 2 * 8 * 32 * 4 + (size_t)g * 16;
+}
+
 // 512 threads for up to 3 chunks per thread, 384 threads (more registers) for 4
 template <typename T, int BITS, int CPT>
 __global__ void __launch_bounds__(CPT <= 3 ? 512 : 384, 1)
@@ -286,19 +379,21 @@ __global__ void __launch_bounds__(CPT <= 3 ? 512 : 384, 1)
     uint32_t *postab = reinterpret_cast<uint32_t *>(smem + (size_t)C * 4);     // 4*C bytes
     float *red = reinterpret_cast<float *>(postab + C);                        // 8*32 floats
     float *red2 = red + 8 * 32;
+    double *ctl = reinterpret_cast<double *>(red2 + 8 * 32);                   // 2*g doubles
+    uint16_t *ctab = reinterpret_cast<uint16_t *>(ctl + 2 * g);                // C u16
     const int64_t G = gridDim.x;
     const bool exact = NCH == CPT * (int)blockDim.x;  // the chunks split evenly over the threads
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x);
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x + G);
     float pA[CPT][VEC], pB[CPT][VEC];
-    quant_tables<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, smem_u32(codebuf), pA, pB,
-                               err);
+    quant_tables_direct<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, ctab, ctl,
+                                      smem_u32(codebuf), pA, pB, err);
+    uint4 xr[4][CPT];
+    load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr);  // the L2 prefetch above is in flight
 
     const int64_t pitch = (int64_t)C * BITS / 8;
     const int NU = C >> 5;
     const NoRefill none;
-    uint4 xr[4][CPT];
-    load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr);
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += G) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         float rstd[4], nmr[4];
@@ -413,7 +508,7 @@ __global__ void __launch_bounds__(256)
 template <typename T, int BITS, int CPT>
 static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
 {
-    const size_t smem = (size_t)a.C * 8 + 2 * 8 * 32 * 4;
+    const size_t smem = direct_smem_bytes(a.C, a.g);
     auto kern = ln_quant_direct_kernel<T, BITS, CPT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -476,9 +571,9 @@ static cudaError_t launch_fast_d(const LnQuantArgs &a, int CPT, int NT, int NS, 
 
 // Plan of the fast kernels for (C, dtype): threads, chunks per thread and, for the ring kernel,
 // ring depth and code-buffer placement (*alias = 0: own buffer, 1: in the quad's slots);
-// *alias = 2 selects the direct kernel (no ring).  Returns false when the shape needs the
-// simple kernel.
-bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *NS, int *alias)
+// *alias = 2 selects the direct kernel (no ring; allow_direct: R and col_cluster are 16-byte
+// aligned for its vector loads).  Returns false when the shape needs the simple kernel.
+bool ln_quant_fast_plan(int C, int esize, int max_smem, bool allow_direct, int *CPT, int *NT, int *NS, int *alias)
 {
     if (C % 32 != 0) return false;
     const int VEC = 16 / esize;
@@ -492,7 +587,7 @@ bool ln_quant_fast_plan(int C, int esize, int max_smem, int *CPT, int *NT, int *
             break;
         }
     }
-    if ((size_t)C * 8 + 2 * 8 * 32 * 4 <= (size_t)max_smem) {  // direct kernel
+    if (allow_direct && direct_smem_bytes(C, RPTQ_MAX_CLUSTERS) <= (size_t)max_smem) {  // direct kernel
         // 384 threads x 4 chunks when that splits the row exactly (every thread also packs one
         // 32-position unit), else the ring kernel's choice of up to 512 threads
         int dc = cpt, dn = nt;
@@ -558,8 +653,10 @@ cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple)
     if (a.T == 0) return cudaSuccess;
     const int esize = a.dtype == RPTQ_F32 ? 4 : 2;
     int CPT = 0, NT = 0, NS = 0, alias = 0;
+    const bool vec_tables = (uintptr_t)a.R % 16 == 0 && (uintptr_t)a.col_cluster % 16 == 0 &&
+                            (uintptr_t)a.gamma % 16 == 0 && (uintptr_t)a.beta % 16 == 0;
     const bool fast = !force_simple && a.ln_out == nullptr && a.codes != nullptr &&
-                      ln_quant_fast_plan(a.C, esize, a.max_smem, &CPT, &NT, &NS, &alias);
+                      ln_quant_fast_plan(a.C, esize, a.max_smem, vec_tables, &CPT, &NT, &NS, &alias);
     if (fast) {
         switch (a.dtype) {
         case RPTQ_F32: return launch_fast_d<float>(a, CPT, NT, NS, alias);

@@ -122,7 +122,8 @@ def test_kmeans_duplicate_points_and_empty_clusters(C, distinct):
 LN_CASES = [  # (dtype, T, C, g, bits)
     ("f32", 512, 768, 8, 4), ("f32", 7, 768, 8, 3), ("f16", 203, 4096, 32, 4),
     ("bf16", 130, 9216, 64, 3), ("bf16", 65, 12288, 64, 3), ("bf16", 1, 12288, 64, 4),
-    ("f16", 6, 256, 5, 3), ("bf16", 33, 2048, 16, 4), ("f32", 9, 4096, 16, 3)]
+    ("f16", 6, 256, 5, 3), ("bf16", 33, 2048, 16, 4), ("f32", 9, 4096, 16, 3),
+    ("bf16", 1203, 12288, 64, 3), ("f16", 97, 16384, 512, 4), ("bf16", 70, 8192, 300, 3)]
 
 
 @pytest.mark.parametrize("dtype,T,C,g,bits", LN_CASES)
@@ -138,6 +139,29 @@ def test_ln_reorder_quant_codes(dtype, T, C, g, bits):
     ref, _, _ = oracle.ln_reorder_quant(x, gamma, beta, cal["R"], cal["col_cluster"], cal["scale"],
                                         cal["zero"], bits)
     compare_codes(to_np(codes), ref, C, bits, f"{dtype} T={T} C={C}")
+
+
+@pytest.mark.parametrize("dtype,T,C,g,bits", [("bf16", 37, 12288, 64, 3), ("f16", 9, 4096, 32, 4),
+                                               ("bf16", 21, 9216, 64, 3)])
+def test_ln_reorder_quant_unaligned_tables(dtype, T, C, g, bits):
+    """R and col_cluster 4 bytes off a 16-byte boundary: the kernel that stages rows through the
+    shared-memory ring (no vector loads of the tables) gives the same codes."""
+    seed = 5 * T + C
+    m, gamma, beta = model_inputs(C, seed)
+    xc = synthetic.activations(64, m, seed, dtype=dtype, calibration=True)
+    cal = oracle_calibration(xc, gamma, beta, g, 10, bits)
+    x = synthetic.activations(T, m, seed, dtype=dtype)
+    p = dev_params(cal)
+    bufR = torch.empty(C + 4, dtype=torch.int32, device=DEV)
+    bufK = torch.empty(C + 4, dtype=torch.int32, device=DEV)
+    R, K = bufR[1:C + 1], bufK[1:C + 1]
+    R.copy_(p["R"])
+    K.copy_(p["col_cluster"])
+    assert R.data_ptr() % 16 != 0
+    codes, _ = rptq.rptq_ln_reorder_quant(x.to(DEV), gamma.to(DEV), beta.to(DEV), R, K, p["scale"], p["zero"], bits)
+    ref, _, _ = oracle.ln_reorder_quant(x, gamma, beta, cal["R"], cal["col_cluster"], cal["scale"],
+                                        cal["zero"], bits)
+    compare_codes(to_np(codes), ref, C, bits, f"unaligned {dtype} T={T} C={C}")
 
 
 @pytest.mark.parametrize("dtype,T,C,g,bits", [
