@@ -93,6 +93,14 @@ template <> __device__ __forceinline__ void chunk_moments<__half>(const uint4 &v
 }
 
 // Streaming 16-byte global load that does not allocate in L1.
+// Bulk prefetch of a contiguous range into L2 (one instruction; 16-byte aligned start, size a
+// multiple of 16 bytes).  Brings a later work unit close without holding registers or shared
+// memory for it.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // three-input max / min (one instruction on sm_100; NaN operands are ignored like fmaxf/fminf)
 __device__ __forceinline__ float max3f(float a, float b, float c)
 {

@@ -350,10 +350,7 @@ __device__ __forceinline__ void prefetch_quad_l2(const void *x, int64_t T_, uint
 {
     if (threadIdx.x == 0 && 4 * gq < T_) {
         const int64_t n = (T_ - 4 * gq < 4 ? T_ - 4 * gq : 4) * (int64_t)rowbytes;
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const uint8_t *>(x) +
-                                                                          4 * gq * (int64_t)rowbytes),
-                     "r"((uint32_t)n)
-                     : "memory");
+        prefetch_l2(static_cast<const uint8_t *>(x) + 4 * gq * (int64_t)rowbytes, (uint32_t)n);
     }
 }
 
