@@ -422,108 +422,131 @@ def run_e2e(step: Step, args, dev, step_bytes, ws):
 
 
 # ------------------------------------------------------------------------------------------
-def oracle_sample(w: W.Workload, frac: float, seed_rank: int = 0):
+class OracleSample:
     """The CPU oracle on a bounded sample of one step: `frac` of the tokens of every
-    token-parallel stage, the three KMeans runs in full.  Returns (bytes the full step moves,
-    extrapolated seconds for the full step, description)."""
-    import numpy as np
+    token-parallel stage (inputs generated once, outside the timing), the three KMeans problems
+    in full.  `time_tokens()` times the token-parallel stages once; `time_kmeans()` the KMeans
+    problems (deterministic: the same inputs give the same work every time)."""
 
-    import oracle
-    oracle.build()
-    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
-    m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
-    gamma, beta = synthetic.ln_params(w.C, w.seed)
-    t_cal = max(4, int((w.T_cal or w.T) * frac))
-    t_x = max(4, int(w.T * frac))
-    secs = {}
-    # calibration on t_cal tokens, in chunks (host memory stays bounded)
-    mx = mn = None
-    tt = 0.0
-    for r0 in range(0, t_cal, 4096):
-        n = min(4096, t_cal - r0)
-        xc = oracle._f32(synthetic.activations(n, m, w.seed + r0, dtype=w.dtype, calibration=True,
-                                               device=gen_dev).cpu())
+    def __init__(self, w: W.Workload, frac: float):
+        import numpy as np
+
+        import oracle
+        oracle.build()
+        self.o, self.w = oracle, w
+        gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+        m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
+        self.gamma, self.beta = synthetic.ln_params(w.C, w.seed)
+        self.t_cal = max(4, int((w.T_cal or w.T) * frac))
+        self.t_x = max(4, int(w.T * frac))
+        self.xc = [oracle._f32(synthetic.activations(min(4096, self.t_cal - r0), m, w.seed + r0, dtype=w.dtype,
+                                                    calibration=True, device=gen_dev).cpu())
+                   for r0 in range(0, self.t_cal, 4096)]
+        self.x = oracle._f32(synthetic.activations(self.t_x, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
+        mx = mn = None
+        for xc in self.xc:
+            mx, mn = oracle.minmax_ln(xc, self.gamma, self.beta, w.eps, ch_max=mx, ch_min=mn)
+        self.mx, self.mn = mx, mn
+        self.desc = f"oracle (1 core) on {self.t_cal} calibration tokens and {self.t_x} tokens of the batch, full KMeans"
+        self.kv = []
+        if w.kv:
+            k = w.kv
+            self.s_s = max(1, int(k.S * frac))
+            for tag, which in ((1, "k"), (2, "v")):
+                mk = synthetic.channel_model(k.channels, w.seed, k.outlier_frac, k.outlier_factor, tag=tag)
+                kvf = oracle._f32(synthetic.kv_cache(k.B, k.H, self.s_s, k.D, mk, w.seed, which, k.dtype,
+                                                    device=gen_dev).cpu())
+                flat = np.ascontiguousarray(kvf.transpose(0, 2, 1, 3).reshape(-1, k.channels))
+                kmx, kmn = oracle.minmax(flat)
+                self.kv.append((kvf, flat, kmx, kmn))
+            self.desc += f", K and V with {self.s_s} of {k.S} sequence positions"
+        self.desc += "; stage times scaled to the full step"
+        self.cal = oracle.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
+        self.kcal = [oracle.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits) for _, _, kmx, kmn in self.kv]
+
+    def bytes_per_step(self) -> int:
+        w = self.w
+        n = W.bytes_calib(w.T_cal or w.T, w.C, w.dtype) + W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits) \
+            + W.bytes_dequant(w.T * w.C, w.dtype, w.bits)
+        if w.kv:
+            k = w.kv
+            n += 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype) + \
+                W.bytes_kv_quant(k.elems, k.dtype, k.bits) + 2 * W.bytes_dequant(k.elems, k.dtype, k.bits)
+        return n
+
+    def time_kmeans(self) -> float:
+        o, w = self.o, self.w
         t = time.perf_counter()
-        mx, mn = oracle.minmax_ln(xc, gamma, beta, w.eps, ch_max=mx, ch_min=mn)
-        tt += time.perf_counter() - t
-    secs["calib_ln"] = tt / (t_cal / (w.T_cal or w.T))
-    t = time.perf_counter()
-    cal = oracle.calibrate(mx, mn, w.g, w.iters, w.bits)
-    secs["kmeans_act"] = time.perf_counter() - t
-    x = oracle._f32(synthetic.activations(t_x, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
-    t = time.perf_counter()
-    packed, _, _ = oracle.ln_reorder_quant(x, gamma, beta, cal["R"], cal["col_cluster"], cal["scale"],
-                                           cal["zero"], w.bits, eps=w.eps)
-    secs["ln_reorder_quant"] = (time.perf_counter() - t) / (t_x / w.T)
-    q = oracle.unpack(packed, w.C, w.bits)
-    t = time.perf_counter()
-    oracle.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])
-    secs["dequant_act"] = (time.perf_counter() - t) / (t_x / w.T)
-    desc = (f"oracle (1 core) on {t_cal} calibration tokens and {t_x} tokens of the batch, full "
-            f"KMeans")
-    if w.kv:
-        k = w.kv
-        s_s = max(1, int(k.S * frac))
-        f_kv = s_s / k.S
-        calib_t = quant_t = deq_t = km_t = 0.0
-        for tag, which in ((1, "k"), (2, "v")):
-            mk = synthetic.channel_model(k.channels, w.seed, k.outlier_frac, k.outlier_factor, tag=tag)
-            kv = synthetic.kv_cache(k.B, k.H, s_s, k.D, mk, w.seed, which, k.dtype, device=gen_dev)
-            kvf = oracle._f32(kv.cpu())
-            flat = np.ascontiguousarray(kvf.transpose(0, 2, 1, 3).reshape(-1, k.channels))
+        o.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
+        for _, _, kmx, kmn in self.kv:
+            o.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits)
+        return time.perf_counter() - t
+
+    def time_tokens(self) -> float:
+        """Seconds the token-parallel stages of a full step take, scaled from the sample."""
+        o, w, cal = self.o, self.w, self.cal
+        secs = 0.0
+        t = time.perf_counter()
+        for xc in self.xc:
+            o.minmax_ln(xc, self.gamma, self.beta, w.eps)
+        secs += (time.perf_counter() - t) / (self.t_cal / (w.T_cal or w.T))
+        t = time.perf_counter()
+        packed, _, _ = o.ln_reorder_quant(self.x, self.gamma, self.beta, cal["R"], cal["col_cluster"],
+                                          cal["scale"], cal["zero"], w.bits, eps=w.eps)
+        q = o.unpack(packed, w.C, w.bits)
+        o.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])
+        secs += (time.perf_counter() - t) / (self.t_x / w.T)
+        if w.kv:
+            k = w.kv
             t = time.perf_counter()
-            kmx, kmn = oracle.minmax(flat)
-            calib_t += time.perf_counter() - t
-            t = time.perf_counter()
-            kc = oracle.calibrate(kmx, kmn, k.g, k.iters, k.bits)
-            km_t += time.perf_counter() - t
-            t = time.perf_counter()
-            pk = oracle.kv_quant(kvf, kc["labels"], kc["scale"], kc["zero"], k.bits)
-            quant_t += time.perf_counter() - t
-            t = time.perf_counter()
-            oracle.kv_dequant(pk, k.D, kc["labels"], kc["scale"], kc["zero"], k.bits)
-            deq_t += time.perf_counter() - t
-        secs["kv_calib"] = calib_t / f_kv
-        secs["kmeans_kv"] = km_t
-        secs["kv_quant"] = quant_t / f_kv
-        secs["dequant_kv"] = deq_t / f_kv
-        desc += f", K and V with {s_s} of {k.S} sequence positions"
-    total_bytes = W.bytes_calib(w.T_cal or w.T, w.C, w.dtype) + W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits) \
-        + W.bytes_dequant(w.T * w.C, w.dtype, w.bits)
-    if w.kv:
-        k = w.kv
-        total_bytes += 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype) + \
-            W.bytes_kv_quant(k.elems, k.dtype, k.bits) + 2 * W.bytes_dequant(k.elems, k.dtype, k.bits)
-    return total_bytes, sum(secs.values()), desc + "; stage times scaled to the full step"
+            for (kvf, flat, _, _), kc in zip(self.kv, self.kcal):
+                o.minmax(flat)
+                pk = o.kv_quant(kvf, kc["labels"], kc["scale"], kc["zero"], k.bits)
+                o.kv_dequant(pk, k.D, kc["labels"], kc["scale"], kc["zero"], k.bits)
+            secs += (time.perf_counter() - t) / (self.s_s / k.S)
+        return secs
 
 
 def cpu_baseline(w, args):
-    nbytes, secs, desc = oracle_sample(w, args.cpu_frac)
-    return {"value": round(nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": desc, "seconds_per_step_extrapolated": round(secs, 2)}
+    smp = OracleSample(w, args.cpu_frac)
+    secs = smp.time_tokens() + smp.time_kmeans()
+    return {"value": round(smp.bytes_per_step() / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": smp.desc, "seconds_per_step_extrapolated": round(secs, 2)}
 
 
 def run_reference(args):
+    """The reference arm: the oracle on the host, one bounded sample per step.  The sample size
+    keeps the whole --steps K --warmup W run near `--ref-budget-s` seconds; the three KMeans
+    problems (deterministic, the same work each step) are timed once and counted in every step."""
     rank, ws, _ = pdist.world()
     if rank != 0:
         return  # under torchrun only rank 0 runs the CPU reference
     w = W.WORKLOADS[args.workload]
-    vals = []
+    probe = OracleSample(w, 1 / 256)
+    t0 = time.perf_counter()
+    probe.time_tokens()
+    per_frac = (time.perf_counter() - t0) * 256  # seconds of token work per full-step fraction 1
+    per_step = args.ref_budget_s / max(1, args.steps + args.warmup)
+    frac = min(args.ref_frac, max(1 / 4096, per_step / max(per_frac, 1e-9)))
+    smp = OracleSample(w, frac)
+    km_secs = smp.time_kmeans()
     for _ in range(args.warmup):
-        oracle_sample(w, args.ref_frac)
+        smp.time_tokens()
+    vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        nbytes, secs, desc = oracle_sample(w, args.ref_frac)
-        vals.append(nbytes / secs / 1e9)
+        vals.append(smp.bytes_per_step() / (smp.time_tokens() + km_secs) / 1e9)
     wall = time.perf_counter() - t0
     value = statistics.mean(vals)
+    nbytes = smp.bytes_per_step()
     line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(nbytes / (value * 1e9) * 1e3, 1), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w), "impl": "reference",
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": desc, "wall_s": round(wall, 1)},
+                             "sample": smp.desc + f" (token fraction {frac:.5f}; KMeans timed once)",
+                             "wall_s": round(wall, 1)},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -540,7 +563,9 @@ def main():
     ap.add_argument("--cpu-frac", type=float, default=1 / 2,
                     help="fraction of the tokens the CPU oracle processes for its baseline")
     ap.add_argument("--ref-frac", type=float, default=1 / 32,
-                    help="fraction of the tokens per step of the --impl reference arm")
+                    help="largest fraction of the tokens per step of the --impl reference arm")
+    ap.add_argument("--ref-budget-s", type=float, default=120.0,
+                    help="target seconds of host work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clock-warmup", dest="clock_warmup", action="store_false",
                     help="skip the untimed steps that let the clock sampler start (profiling runs)")
