@@ -360,9 +360,10 @@ static inline size_t direct_smem_bytes(int C, int g)
     return (size_t)C * 10 + 2 * 8 * 32 * 4 + (size_t)g * 16;
 }
 
-// 512 threads for up to 3 chunks per thread, 384 threads (more registers) for 4
-template <typename T, int BITS, int CPT>
-__global__ void __launch_bounds__(CPT <= 3 ? 512 : 384, 1)
+// MAXT bounds the threads per CTA and so the registers per thread: 512 (128 registers) or 384
+// (168 registers, for 4 chunks per thread, or 3 chunks when 384 threads cover the row)
+template <typename T, int BITS, int CPT, int MAXT>
+__global__ void __launch_bounds__(MAXT, 1)
     ln_quant_direct_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
                            const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
                            const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
@@ -502,11 +503,11 @@ __global__ void __launch_bounds__(256)
 // Host launchers
 // ------------------------------------------------------------------------------------------
 
-template <typename T, int BITS, int CPT>
+template <typename T, int BITS, int CPT, int MAXT>
 static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
 {
     const size_t smem = direct_smem_bytes(a.C, a.g);
-    auto kern = ln_quant_direct_kernel<T, BITS, CPT>;
+    auto kern = ln_quant_direct_kernel<T, BITS, CPT, MAXT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
@@ -545,10 +546,10 @@ static cudaError_t launch_fast_b(const LnQuantArgs &a, int CPT, int NT, int NS, 
 {
     if (alias == 2) {
         switch (CPT) {
-        case 1: return launch_direct_t<T, BITS, 1>(a, NT);
-        case 2: return launch_direct_t<T, BITS, 2>(a, NT);
-        case 3: return launch_direct_t<T, BITS, 3>(a, NT);
-        case 4: return launch_direct_t<T, BITS, 4>(a, NT);
+        case 1: return launch_direct_t<T, BITS, 1, 512>(a, NT);
+        case 2: return launch_direct_t<T, BITS, 2, 512>(a, NT);
+        case 3: return NT <= 384 ? launch_direct_t<T, BITS, 3, 384>(a, NT) : launch_direct_t<T, BITS, 3, 512>(a, NT);
+        case 4: return launch_direct_t<T, BITS, 4, 384>(a, NT);
         default: return cudaErrorInvalidValue;
         }
     }
@@ -585,15 +586,17 @@ bool ln_quant_fast_plan(int C, int esize, int max_smem, bool allow_direct, int *
         }
     }
     if (allow_direct && direct_smem_bytes(C, RPTQ_MAX_CLUSTERS) <= (size_t)max_smem) {  // direct kernel
-        // 384 threads x 4 chunks when that splits the row exactly (every thread also packs one
-        // 32-position unit), else the ring kernel's choice of up to 512 threads
+        // 320..384 threads x 3 chunks, or 256..384 threads x 4 chunks, when that splits the row
+        // exactly (every thread also packs one 32-position unit), else the ring kernel's choice
+        // of up to 512 threads
         int dc = cpt, dn = nt;
-#ifndef RPTQ_DIRECT_512
-        if (NCH % (4 * 32) == 0 && NCH / 4 <= 384 && NCH / 4 >= 256) {
+        if (NCH % (3 * 32) == 0 && NCH / 3 <= 384 && NCH / 3 >= 320) {
+            dc = 3;
+            dn = NCH / 3;
+        } else if (NCH % (4 * 32) == 0 && NCH / 4 <= 384 && NCH / 4 >= 256) {
             dc = 4;
             dn = NCH / 4;
         }
-#endif
         if (!dc) return false;
         *CPT = dc;
         *NT = dn;
