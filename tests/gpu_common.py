@@ -1,6 +1,6 @@
 """Helpers for the GPU parity tests: seeded inputs, oracle calls and the comparison rules.
 
-Tolerances (derived in DESIGN.md, section "Parity bars"):
+Tolerances (each follows from the arithmetic of the two sides):
   * min/max in raw mode, R, labels, offsets, col_cluster, scale, zero, dequantized values:
     bit-exact;
   * centroids: relative 1e-6 (the GPU sums cluster members in a different fixed order);
