@@ -193,6 +193,7 @@ int rptq_kmeans_noalloc(const float *ch_max, const float *ch_min, int C, int g, 
  *   scale, zero  fp32 [g], int32 [g]; g is the length of these tables.
  *   codes        uint8 [T, C*bits/8] packed codes in stored order, or NULL.
  *   ln_out       [T, C] of `dtype`, stored order, or NULL.  At least one of codes / ln_out.
+ * T == 0 is valid: nothing is launched and x, codes and ln_out may all be NULL.
  * Codes are computed in fp32 and may differ from an exact-arithmetic reference by one step
  * where y / scale lies within fp32 rounding of a half-integer.
  */
@@ -210,7 +211,8 @@ int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const floa
  * so no reorder applies.  scale_*, zero_*: fp32 / int32 [g].
  *   code = clamp(rint(x / s) + z, 0, qmax), packed along D:
  *   k_codes / v_codes uint8 [B, H, S, D*bits/8].
- * D must be a multiple of 8 and H*D <= RPTQ_MAX_CHANNELS.
+ * D must be a multiple of 8 and H*D <= RPTQ_MAX_CHANNELS.  B == 0 or S == 0 is valid: nothing
+ * is launched and no pointer is read (any of them may be NULL).
  */
 int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t S, int D,
                   const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
@@ -225,6 +227,7 @@ int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t
  *   layout RPTQ_LAYOUT_BHSD: codes [n0, n1, S, D*bits/8] with n0 = B, n1 = H; cluster[c] is
  *          the cluster of channel c = h*D + d.
  *   out: same shape with unpacked values of out_dtype.
+ * n0 == 0 (or S == 0 for BHSD) is valid: nothing is launched and codes / out may be NULL.
  */
 int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,
                  const int32_t *cluster, const float *scale, const int32_t *zero, int g,

@@ -177,9 +177,10 @@ int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const floa
     if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
     if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
     if (T < 0 || g <= 0 || g > C || !(eps >= 0.0f)) return RPTQ_ERR_INVALID_ARG;
-    if (!codes && !ln_out) return RPTQ_ERR_INVALID_ARG;
     if (!gamma || !beta || !R || !col_cluster || !scale || !zero) return RPTQ_ERR_INVALID_ARG;
-    if (T > 0 && (!x || !aligned16(x))) return RPTQ_ERR_INVALID_ARG;
+    if (T == 0) return RPTQ_OK;  // no rows: nothing to launch, outputs may be empty (NULL)
+    if (!codes && !ln_out) return RPTQ_ERR_INVALID_ARG;
+    if (!x || !aligned16(x)) return RPTQ_ERR_INVALID_ARG;
     if (codes && !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
     if (ln_out && !aligned16(ln_out)) return RPTQ_ERR_INVALID_ARG;
     DevInfo d;
@@ -201,13 +202,11 @@ int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t
     if (D <= 0 || D % 8 != 0 || D > 2048 || H <= 0 || (int64_t)H * D > RPTQ_MAX_CHANNELS)
         return RPTQ_ERR_UNSUPPORTED;
     if (B < 0 || S < 0 || g <= 0) return RPTQ_ERR_INVALID_ARG;
+    if (B == 0 || S == 0) return RPTQ_OK;  // an empty cache: nothing to launch, no pointer read
     if (!k && !v) return RPTQ_ERR_INVALID_ARG;
-    const bool work = B > 0 && S > 0;
-    if (k && (!cluster_k || !scale_k || !zero_k || !k_codes || !aligned16(k_codes) ||
-              (work && !aligned16(k))))
+    if (k && (!cluster_k || !scale_k || !zero_k || !k_codes || !aligned16(k_codes) || !aligned16(k)))
         return RPTQ_ERR_INVALID_ARG;
-    if (v && (!cluster_v || !scale_v || !zero_v || !v_codes || !aligned16(v_codes) ||
-              (work && !aligned16(v))))
+    if (v && (!cluster_v || !scale_v || !zero_v || !v_codes || !aligned16(v_codes) || !aligned16(v)))
         return RPTQ_ERR_INVALID_ARG;
     if ((int64_t)B * H > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
     DevInfo d;
@@ -226,8 +225,11 @@ int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S
     if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
     if (layout != RPTQ_LAYOUT_ROWS && layout != RPTQ_LAYOUT_BHSD) return RPTQ_ERR_INVALID_ARG;
     if (n0 < 0 || n1 <= 0 || g <= 0) return RPTQ_ERR_INVALID_ARG;
-    if (!codes || !cluster || !scale || !zero || !out) return RPTQ_ERR_INVALID_ARG;
-    if (!aligned16(codes) || !aligned16(out)) return RPTQ_ERR_INVALID_ARG;
+    if (!cluster || !scale || !zero) return RPTQ_ERR_INVALID_ARG;
+    // no rows (or no positions): nothing to launch, codes / out may be empty (NULL)
+    const bool work = n0 > 0 && (layout == RPTQ_LAYOUT_ROWS || S > 0);
+    if (work && (!codes || !out || !aligned16(codes) || !aligned16(out)))
+        return RPTQ_ERR_INVALID_ARG;
     if (layout == RPTQ_LAYOUT_ROWS) {
         if (n1 % 8 != 0 || n1 > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
     } else {
@@ -235,6 +237,7 @@ int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S
             return RPTQ_ERR_UNSUPPORTED;
         if (S < 0 || S > 0x7fffffffLL || n0 * n1 > 0x7fffffffLL) return RPTQ_ERR_INVALID_ARG;
     }
+    if (!work) return RPTQ_OK;
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;

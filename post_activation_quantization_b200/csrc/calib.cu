@@ -255,9 +255,9 @@ __global__ void __launch_bounds__(512, 1)
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
         pipe.load(nrows, xr);
-        float rstd[4], nmr[4];
-        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr);
-        if (nrows == 4) {  // normalised values of tokens (0, 1) and (2, 3) two lanes at a time
+        float rstd[4], nmr[4], sub[4];
+        const bool offs = quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, sub);
+        if (nrows == 4 && !offs) {  // normalised values of tokens (0, 1) and (2, 3) two lanes at a time
             const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
             const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
 #pragma unroll
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(512, 1)
                     tmax[k][e] = max3f(max3f(tmax[k][e], lo2(t01), hi2(t01)), lo2(t23), hi2(t23));
                     tmin[k][e] = min3f(min3f(tmin[k][e], lo2(t01), hi2(t01)), lo2(t23), hi2(t23));
                 }
-        } else {
+        } else {  // a partial quad, or one with an offset row (x - sub is exact; see quad_stats)
 #pragma unroll
             for (int k = 0; k < CPT; ++k)
 #pragma unroll
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(512, 1)
                     if (r >= nrows) break;
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) {
-                        const float t = fmaf(Elem<T>::get(xr[r][k], e), rstd[r], nmr[r]);
+                        const float t = fmaf(Elem<T>::get(xr[r][k], e) - sub[r], rstd[r], nmr[r]);
                         tmax[k][e] = fmaxf(tmax[k][e], t);
                         tmin[k][e] = fminf(tmin[k][e], t);
                     }
@@ -332,19 +332,10 @@ __global__ void __launch_bounds__(256)
         }
         float v8[8] = {s, 0, 0, 0, 0, 0, 0, 0};
         cta_sum8(v8, red);
-        const float mean = v8[0] / (float)C;
-        float ss = 0.f;
+        float hi, rstd, nmr;
+        row_moments(xs, C, v8[0], eps, red, hi, rstd, nmr);
         for (int c = tid; c < C; c += NT) {
-            const float d = xs[c] - mean;
-            ss = fmaf(d, d, ss);
-        }
-        float w8[8] = {ss, 0, 0, 0, 0, 0, 0, 0};
-        __syncthreads();  // red is reused
-        cta_sum8(w8, red);
-        const float rstd = rsqrtf(w8[0] / (float)C + eps);
-        const float nmr = -mean * rstd;
-        for (int c = tid; c < C; c += NT) {
-            const float tv = fmaf(xs[c], rstd, nmr);
+            const float tv = fmaf(xs[c] - hi, rstd, nmr);
             tmx[c] = fmaxf(tmx[c], tv);
             tmn[c] = fminf(tmn[c], tv);
         }

@@ -168,9 +168,11 @@ __device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int3
 }
 
 // Codes of the quad's four tokens for every channel of the thread -> one word per channel at
-// its stored position in the code buffer.
-template <typename T, int BITS, int CPT, bool ABS>
+// its stored position in the code buffer.  SUB: subtract sub[r] before the normalising fma (the
+// quad holds a row with a large offset or no spread; see quad_stats).
+template <typename T, int BITS, int CPT, bool ABS, bool SUB>
 __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const float (&rstd)[4], const float (&nmr)[4],
+                                              const float (&sub)[4],
                                               const float (&pA)[CPT][Elem<T>::VEC],
                                               const float (&pB)[CPT][Elem<T>::VEC], const void *postab,
                                               uint8_t *codebuf, int NCH)
@@ -182,6 +184,7 @@ __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const f
     const int tid = threadIdx.x, NT = blockDim.x;
     const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
     const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
+    const f32x2 ms01 = mk2(-sub[0], -sub[1]), ms23 = mk2(-sub[2], -sub[3]);
     const f32x2 qm2 = mk2(QMAX, QMAX), mg2 = mk2(MAGIC_RINT, MAGIC_RINT);
 #pragma unroll
     for (int k = 0; k < CPT; ++k) {
@@ -205,8 +208,14 @@ __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const f
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             // normalised values of channel e for tokens (0,1) and (2,3), two lanes at a time
-            const f32x2 t01 = fma2(mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e)), rs01, nm01);
-            const f32x2 t23 = fma2(mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e)), rs23, nm23);
+            f32x2 x01 = mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e));
+            f32x2 x23 = mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e));
+            if constexpr (SUB) {
+                x01 = add2(x01, ms01);
+                x23 = add2(x23, ms23);
+            }
+            const f32x2 t01 = fma2(x01, rs01, nm01);
+            const f32x2 t23 = fma2(x23, rs23, nm23);
             const float A = pA[k][e], Bc = pB[k][e];
             // u = sat(y / (s qmax) + z / qmax); code = rint(u qmax) (the 1.5*2^23 rounding add)
             const f32x2 u01 = mk2(fma_sat(lo2(t01), A, Bc), fma_sat(hi2(t01), A, Bc));
@@ -298,10 +307,13 @@ __global__ void __launch_bounds__(512, 1)
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         uint4 xr[4][CPT];
         pipe.load(nrows, xr);
-        float rstd[4], nmr[4];
-        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, !alias);
+        float rstd[4], nmr[4], sub[4];
+        const bool offs = quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, sub, !alias);
         if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
-        quant_scatter<T, BITS, CPT, false>(xr, rstd, nmr, pA, pB, postab, codebuf, NCH);
+        if (offs)
+            quant_scatter<T, BITS, CPT, false, true>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
+        else
+            quant_scatter<T, BITS, CPT, false, false>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
         __syncthreads();
         pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU);
         if (alias) {  // the quad's slots held its codes until now
@@ -394,9 +406,11 @@ __global__ void __launch_bounds__(MAXT, 1)
     const NoRefill none;
     for (int64_t gq = blockIdx.x; 4 * gq < T_; gq += G) {
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
-        float rstd[4], nmr[4];
-        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, none, 0, rstd, nmr, false);
-        quant_scatter<T, BITS, CPT, true>(xr, rstd, nmr, pA, pB, postab, codebuf, NCH);
+        float rstd[4], nmr[4], sub[4];
+        if (quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, none, 0, rstd, nmr, sub, false))
+            quant_scatter<T, BITS, CPT, true, true>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
+        else
+            quant_scatter<T, BITS, CPT, true, false>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
         // the rows are dead: next quad's loads fly during the pack, and one more quad to L2
         load_quad_direct<T, CPT>(x, T_, C, gq + G, exact, xr);
         prefetch_quad_l2(x, T_, rowbytes, gq + 2 * G);
@@ -448,17 +462,8 @@ __global__ void __launch_bounds__(256)
         }
         float v8[8] = {s, 0, 0, 0, 0, 0, 0, 0};
         cta_sum8(v8, red);
-        const float mean = v8[0] / (float)C;
-        float ss = 0.f;
-        for (int c = tid; c < C; c += NT) {
-            const float d = xs[c] - mean;
-            ss = fmaf(d, d, ss);
-        }
-        float w8[8] = {ss, 0, 0, 0, 0, 0, 0, 0};
-        __syncthreads();  // red is reused
-        cta_sum8(w8, red);
-        const float rstd = rsqrtf(w8[0] / (float)C + eps);
-        const float nmr = -mean * rstd;
+        float hi, rstd, nmr;
+        row_moments(xs, C, v8[0], eps, red, hi, rstd, nmr);
         for (int j = tid; j < C; j += NT) {
             int c = R[j];
             if (c < 0 || c >= C) {
@@ -470,7 +475,7 @@ __global__ void __launch_bounds__(256)
                 raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
                 k = 0;
             }
-            const float y = fmaf(fmaf(xs[c], rstd, nmr), gamma[c], beta[c]);
+            const float y = fmaf(fmaf(xs[c] - hi, rstd, nmr), gamma[c], beta[c]);
             if (ln_out) ln_out[t * (int64_t)C + j] = from_f32<T>(y);
             if (codes) {
                 const float q = rintf(__fdiv_rn(y, scale[k])) + (float)zero[k];

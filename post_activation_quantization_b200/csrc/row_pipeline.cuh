@@ -108,14 +108,22 @@ struct QuadRows {
     }
 };
 
-// LayerNorm statistics of the four rows in xr.  Returns rstd[r] and nmr[r] = -mean*rstd so that
-// the normalised value is fmaf(x, rstd, nmr).  `red`, `red2`: 8*(NT/32) floats each.
-// With refill_now, calls refill() between its first barrier and any later one (the caller
-// refills later when it still uses the quad's ring slots).
+// LayerNorm statistics of the four rows in xr.  The normalised value of x is
+// fmaf(x - sub[r], rstd[r], nmr[r]); returns whether any row of the quad needs the subtraction
+// (the same answer in every thread).  A row whose mean is small against its spread
+// (mean^2 <= var) takes the single-pass moments, sub = 0 and nmr = -mean*rstd.  Otherwise
+// (a large common offset, or a constant row) the single-pass variance cancels and the rounding
+// of -mean*rstd alone would move every value of the row together, so the row is redone from
+// d = x - m0 (m0 = sum / C, correctly rounded): sum(d) refines the mean to the pair
+// sub + lo (sub = fl(m0 + sum(d)/C)), var = sum(d^2)/C - (sum(d)/C)^2, nmr = -lo*rstd; x - sub
+// is exact for x near the mean, so the offset never meets a rounding.
+// `red`, `red2`: 8*(NT/32) floats each.  With refill_now, calls refill() between its first
+// barrier and any later one (the caller refills later when it still uses the quad's ring slots).
 template <typename T, int CPT, typename Pipe>
-__device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int NCH, float eps,
+__device__ __forceinline__ bool quad_stats(const uint4 (&xr)[4][CPT], int C, int NCH, float eps,
                                            float *red, float *red2, const Pipe &pipe, int64_t lq,
-                                           float (&rstd)[4], float (&nmr)[4], bool refill_now = true)
+                                           float (&rstd)[4], float (&nmr)[4], float (&sub)[4],
+                                           bool refill_now = true)
 {
     constexpr int VEC = Elem<T>::VEC;
     const int tid = threadIdx.x, NT = blockDim.x;
@@ -131,17 +139,23 @@ __device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int
     if (refill_now) pipe.refill(lq);
     const float invC = 1.0f / (float)C;
     float mean[4], var[4];
-    bool ill = false;
+    bool ill[4], any = false;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         mean[r] = v[r] * invC;
         var[r] = v[4 + r] * invC - mean[r] * mean[r];
-        ill |= !(mean[r] * mean[r] <= var[r]);
+        ill[r] = !(mean[r] * mean[r] <= var[r]);
+        any |= ill[r];
+        sub[r] = 0.f;
     }
-    if (ill) {  // same decision in every thread (identical reduced values)
-        float w[8];
+    if (any) {
+        float m0[4], w[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[i] = 0.f;
+        for (int r = 0; r < 4; ++r) {
+            m0[r] = __fdiv_rn(v[r], (float)C);
+            w[r] = 0.f;
+            w[4 + r] = 0.f;
+        }
 #pragma unroll
         for (int k = 0; k < CPT; ++k) {
             if (tid + k * NT < NCH) {
@@ -149,20 +163,55 @@ __device__ __forceinline__ void quad_stats(const uint4 (&xr)[4][CPT], int C, int
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) {
-                        const float d = Elem<T>::get(xr[r][k], e) - mean[r];
-                        w[r] = fmaf(d, d, w[r]);
+                        const float d = Elem<T>::get(xr[r][k], e) - m0[r];
+                        w[r] += d;
+                        w[4 + r] = fmaf(d, d, w[4 + r]);
                     }
             }
         }
         cta_sum8(w, red2);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) var[r] = w[r] * invC;
+        for (int r = 0; r < 4; ++r) {
+            if (!ill[r]) continue;
+            const float delta = w[r] * invC;
+            const float hi = m0[r] + delta;
+            mean[r] = delta - (hi - m0[r]);  // the low part of the mean pair (hi, mean)
+            sub[r] = hi;
+            var[r] = fmaf(-delta, delta, w[4 + r] * invC);
+        }
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
         rstd[r] = rsqrtf(fmaxf(var[r], 0.f) + eps);
         nmr[r] = -mean[r] * rstd[r];
     }
+    return any;
+}
+
+// LayerNorm statistics of one row held in shared memory (xs[0..C), every thread of the CTA,
+// `sum` = the CTA's reduced sum of the row): the mean as the pair hi + lo (hi = fl(m0 + delta),
+// m0 = sum / C, delta = sum(x - m0) / C) and the variance from the same deviations, so
+// fmaf(x - hi, rstd, nmr) with nmr = -lo*rstd stays exact for rows with a large common offset.
+// `red`: 64 floats, reused after a barrier.
+__device__ __forceinline__ void row_moments(const float *xs, int C, float sum, float eps, float *red,
+                                            float &hi, float &rstd, float &nmr)
+{
+    const float m0 = __fdiv_rn(sum, (float)C);
+    float sd = 0.f, ss = 0.f;
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        const float d = xs[c] - m0;
+        sd += d;
+        ss = fmaf(d, d, ss);
+    }
+    float w8[8] = {sd, ss, 0, 0, 0, 0, 0, 0};
+    __syncthreads();  // red is reused
+    cta_sum8(w8, red);
+    const float delta = w8[0] / (float)C;
+    hi = m0 + delta;
+    const float lo = delta - (hi - m0);
+    const float var = fmaf(-delta, delta, w8[1] / (float)C);
+    rstd = rsqrtf(fmaxf(var, 0.f) + eps);
+    nmr = -lo * rstd;
 }
 
 // Dynamic shared memory of a quad pipeline: ring + extra bytes, with 128-byte alignment.

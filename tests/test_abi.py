@@ -82,3 +82,24 @@ def test_host_validation_rejects_before_any_launch(rlib):
     # dequant: bad layout
     assert rlib.rptq_dequant(fake, 5, 4, 64, 0, 0, fake, fake, fake, 8, 3, fake, 0, None) == -1
     assert rlib.rptq_device_error(None, None) == -1
+
+
+def test_empty_problems_succeed_on_the_host(rlib):
+    """Empty problems are valid no-ops: they return before any CUDA call (this runs without a
+    GPU) and accept NULL data pointers, as an empty tensor provides."""
+    P = ctypes.c_void_p
+    fake = P(16 * 1024)  # tables: never dereferenced
+    # T = 0 rows, x / codes / ln_out NULL
+    assert rlib.rptq_ln_reorder_quant(None, 2, 0, 64, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
+                                      None, None, None) == 0
+    # S = 0 and B = 0 caches
+    assert rlib.rptq_kv_quant(None, None, 1, 2, 3, 0, 64, None, None, None, None, None, None, 4, 3,
+                              None, None, None) == 0
+    assert rlib.rptq_kv_quant(None, None, 1, 0, 3, 5, 64, None, None, None, None, None, None, 4, 3,
+                              None, None, None) == 0
+    # n0 = 0 rows; S = 0 positions of a BHSD cache
+    assert rlib.rptq_dequant(None, 0, 0, 64, 0, 0, fake, fake, fake, 8, 3, None, 0, None) == 0
+    assert rlib.rptq_dequant(None, 1, 2, 3, 0, 64, fake, fake, fake, 8, 3, None, 0, None) == 0
+    # ... but an empty problem with an invalid shape is still refused
+    assert rlib.rptq_ln_reorder_quant(None, 2, 0, 60, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
+                                      None, None, None) == -2
