@@ -220,6 +220,22 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
 }
+// Copy `bytes` (multiple of 16, both addresses 16-byte aligned) shared -> global as one bulk
+// asynchronous copy of the calling thread's current bulk group (never multicast).
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every bulk group of the thread but the newest N has finished READING its shared
+// source (the buffer may be rewritten), or has fully completed (wait_all).
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // One suspending try: the thread sleeps in hardware until the phase completes or a system
 // time limit passes (no busy polling that would take issue slots from working warps).
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity)

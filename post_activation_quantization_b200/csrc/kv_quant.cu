@@ -216,6 +216,136 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
+// Ring kernel (16-bit caches; D/8 a power of two <= 256; S a multiple of the stage rows 8192/D).
+// The work is cut into stages of 16 KB of the cache (8192/D whole rows of one (b, h) block,
+// contiguous in memory) and a stage's codes are 1024*BITS contiguous bytes of the output.
+// Stages are ordered (tensor, h, b, chunk) and every CTA of a one-wave grid takes a contiguous
+// range of them, so it crosses at most a couple of heads.  Thread 0 streams the stages into a
+// ring of KVR_NS shared-memory slots by bulk asynchronous copies (mbarrier completion, never
+// multicast); each thread turns its four 16-byte pieces (8 channels each; piece p of a stage
+// sits at p*16 in the slot and its codes at p*BITS in the code buffer, whatever D is) into
+// codes, and thread 0 writes the stage's codes with one bulk copy from one of two code buffers.
+constexpr int KVR_THREADS = 256;
+constexpr uint32_t KVR_STAGE = 16384;
+constexpr int KVR_PIECES = KVR_STAGE / 16;
+constexpr int KVR_PPT = KVR_PIECES / KVR_THREADS;
+constexpr int KVR_NS = 6;
+
+template <int BITS>
+constexpr size_t kv_ring_smem() { return (size_t)KVR_NS * KVR_STAGE + 2 * KVR_PIECES * BITS + 8 * KVR_NS; }
+
+// A stage's place in (tensor, h, b, chunk) order, advanced without divisions.
+struct KvStagePos {
+    int ti, h, b, chunk;
+    __device__ __forceinline__ void set(int64_t j, int64_t per_t, int B, int SPB)
+    {
+        ti = (int)(j / per_t);
+        int64_t r = j - ti * per_t;
+        const int64_t per_h = (int64_t)B * SPB;
+        h = (int)(r / per_h);
+        r -= h * per_h;
+        b = (int)(r / SPB);
+        chunk = (int)(r - (int64_t)b * SPB);
+    }
+    __device__ __forceinline__ void advance(int B, int H, int SPB)
+    {
+        if (++chunk == SPB) {
+            chunk = 0;
+            if (++b == B) {
+                b = 0;
+                if (++h == H) {
+                    h = 0;
+                    ++ti;
+                }
+            }
+        }
+    }
+    // stage number within its tensor in memory order (b, h, chunk)
+    __device__ __forceinline__ int64_t mem_index(int H, int SPB) const { return ((int64_t)b * H + h) * SPB + chunk; }
+};
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(KVR_THREADS, 2)
+    kv_quant_ring(KvTensors t, int nt, int sel0, int sel1, int B, int H, int SPB, int D, int g, int *err)
+{
+    constexpr uint32_t CBYTES = KVR_PIECES * BITS;  // codes of one stage
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_abort;
+    uint8_t *ring = smem;
+    uint8_t *cbuf = smem + (size_t)KVR_NS * KVR_STAGE;
+    const uint32_t bar0 = smem_u32(cbuf + 2 * CBYTES);
+    const int tid = threadIdx.x;
+    const int64_t per_t = (int64_t)B * H * SPB, total = per_t * nt;
+    const int64_t j0 = total * blockIdx.x / gridDim.x, j1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int n = (int)(j1 - j0);  // the grid has at least total / 2^31 CTAs
+    if (n <= 0) return;
+    KvStagePos prod;  // thread 0: the next stage to load
+    auto issue = [&](uint32_t s) {
+        const int tt = prod.ti ? sel1 : sel0;
+        const uint8_t *src = static_cast<const uint8_t *>(t.src[tt]) + prod.mem_index(H, SPB) * KVR_STAGE;
+        mbar_expect_tx(bar0 + 8u * s, KVR_STAGE);
+        bulk_g2s(smem_u32(ring + (size_t)s * KVR_STAGE), src, KVR_STAGE, bar0 + 8u * s);
+        prod.advance(B, H, SPB);
+    };
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < KVR_NS; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+        prod.set(j0, per_t, B, SPB);
+        for (int s = 0; s < KVR_NS && s < n; ++s) issue((uint32_t)s);
+    }
+    __syncthreads();
+    KvStagePos cur;
+    cur.set(j0, per_t, B, SPB);
+    const int col = tid & ((D >> 3) - 1);  // the thread's 8-channel group, the same in every piece
+    KvCoef<BITS, 8> cf;
+    int cf_key = -1;
+    uint32_t slot = 0, phase = 0;
+    for (int i = 0; i < n; ++i) {
+        const int tt = cur.ti ? sel1 : sel0;
+        if (cur.ti * H + cur.h != cf_key) {
+            cf.load(t.cl[tt], t.sc[tt], t.zp[tt], cur.h * D + col * 8, g, err);
+            cf_key = cur.ti * H + cur.h;
+        }
+        if (!mbar_wait_bounded(bar0 + 8u * slot, phase, err)) s_abort = 1;
+        const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)slot * KVR_STAGE);
+        uint4 xb[KVR_PPT];
+#pragma unroll
+        for (int k = 0; k < KVR_PPT; ++k) xb[k] = src[tid + k * KVR_THREADS];
+        uint8_t *cb = cbuf + (i & 1) * CBYTES;
+#pragma unroll
+        for (int k = 0; k < KVR_PPT; ++k) {
+            uint32_t grp[1];
+            kv_quant_row<T, BITS, 8>(&xb[k], cf, grp);
+            uint8_t *o = cb + (tid + k * KVR_THREADS) * BITS;
+            if constexpr (BITS == 4) {
+                *reinterpret_cast<uint32_t *>(o) = grp[0];
+            } else {
+                o[0] = (uint8_t)grp[0];
+                o[1] = (uint8_t)(grp[0] >> 8);
+                o[2] = (uint8_t)(grp[0] >> 16);
+            }
+        }
+        // the previous stage's code store has finished reading its buffer, which the stage
+        // after this one rewrites
+        if (tid == 0) bulk_wait_read<0>();
+        __syncthreads();  // slot read, codes complete
+        if (s_abort) break;
+        if (tid == 0) {
+            fence_proxy_async_smem();
+            bulk_s2g(t.dst[tt] + cur.mem_index(H, SPB) * CBYTES, smem_u32(cb), CBYTES);
+            bulk_commit();
+            if (i + KVR_NS < n) issue(slot);  // the slot just read, KVR_NS stages later
+        }
+        cur.advance(B, H, SPB);
+        if (++slot == KVR_NS) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+}
+
 // CTA kernel: blockIdx.x = b*H + h, blockIdx.y = tensor; the CTA streams all S rows of the block.
 template <typename T, int BITS, int DPT>
 __global__ void __launch_bounds__(256)
@@ -284,9 +414,46 @@ static cudaError_t launch_kv_cta(const KvArgs &a)
     return cudaGetLastError();
 }
 
+template <typename T, int BITS>
+static cudaError_t launch_kv_ring(const KvArgs &a)
+{
+    const KvTensors t{{a.k, a.v}, {a.kq, a.vq}, {a.ck, a.cv}, {a.sk, a.sv}, {a.zk, a.zv}};
+    int sel[2] = {0, 1}, nt = 0;
+    if (a.k) sel[nt++] = 0;
+    if (a.v) sel[nt++] = 1;
+    const int SPB = (int)(a.S / (8192 / a.D));
+    auto kern = kv_quant_ring<T, BITS>;
+    const size_t smem = kv_ring_smem<BITS>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t total = (int64_t)a.B * a.H * SPB * nt;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * a.num_sms, total);
+    kern<<<(unsigned)grid, KVR_THREADS, smem, a.stream>>>(t, nt, sel[0], sel[1], a.B, a.H, SPB, a.D, a.g, a.err);
+    return cudaGetLastError();
+}
+
+// The ring kernel's shape rule: 16-bit elements, D/8 a power of two dividing the 256 threads,
+// whole stages of 8192/D rows per (b, h) block, and a stage count the grid split keeps in int.
+static bool kv_ring_ok(const KvArgs &a, int esize)
+{
+    if (esize != 2 || a.D % 8 != 0 || a.D > 2048) return false;
+    const int npr = a.D / 8;
+    if ((npr & (npr - 1)) != 0) return false;
+    const int64_t sr = 8192 / a.D;
+    if (a.S % sr != 0) return false;
+    const int64_t per_t = (int64_t)a.B * a.H * (a.S / sr);
+    return per_t * 2 < 0x7fffffffLL && a.S / sr < 0x7fffffffLL;
+}
+
 template <typename T>
 static cudaError_t launch_kv_d(const KvArgs &a)
 {
+    if constexpr (sizeof(T) == 2)
+        if (kv_ring_ok(a, 2)) return a.bits == 4 ? launch_kv_ring<T, 4>(a) : launch_kv_ring<T, 3>(a);
     // warp kernel when the 8-channel groups of a row tile a warp evenly (D in 8, 16, ..., 256)
     if (a.D % 8 == 0 && a.D <= 256 && 32 % (a.D / 8) == 0 && a.S <= 0x7fffffffLL)
         return a.bits == 4 ? launch_kv_warp<T, 4>(a) : launch_kv_warp<T, 3>(a);

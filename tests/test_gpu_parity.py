@@ -225,7 +225,11 @@ def test_kv_calib_bit_exact(dtype, B, H, S, D):
 
 KV_CASES = [("f16", 2, 4, 33, 128, 6, 3), ("bf16", 1, 3, 17, 64, 5, 4), ("f32", 2, 2, 9, 128, 8, 4),
             ("f16", 1, 2, 11, 40, 4, 3), ("bf16", 3, 5, 7, 256, 7, 3), ("bf16", 2, 3, 300, 128, 6, 3),
-            ("f16", 1, 2, 5, 512, 4, 4), ("bf16", 2, 2, 130, 32, 5, 3), ("f32", 1, 3, 19, 8, 3, 4)]
+            ("f16", 1, 2, 5, 512, 4, 4), ("bf16", 2, 2, 130, 32, 5, 3), ("f32", 1, 3, 19, 8, 3, 4),
+            # whole 16 KB stages per (b, h) block (S a multiple of 8192 / D): the streaming-ring kernel
+            ("bf16", 2, 3, 128, 128, 6, 3), ("f16", 2, 3, 192, 128, 5, 4), ("bf16", 1, 4, 256, 64, 7, 4),
+            ("f16", 3, 2, 64, 256, 6, 3), ("bf16", 1, 2, 8, 2048, 4, 3), ("f16", 1, 3, 1024, 8, 3, 4),
+            ("bf16", 2, 5, 512, 32, 9, 3)]
 
 
 @pytest.mark.parametrize("dtype,B,H,S,D,g,bits", KV_CASES)
@@ -251,6 +255,8 @@ def test_kv_quant(dtype, B, H, S, D, g, bits):
     kq2, vq2 = rptq.rptq_kv_quant(k.to(DEV), None, pk["labels"], pk["scale"], pk["zero"], None, None,
                                   None, bits)
     assert vq2 is None and torch.equal(kq2, kq)
+    kq3, vq3 = rptq.rptq_kv_quant(None, v.to(DEV), None, None, None, pv["labels"], pv["scale"], pv["zero"], bits)
+    assert kq3 is None and torch.equal(vq3, vq)
 
 
 # ---------------------------------------------------------------- dequantization
