@@ -136,7 +136,7 @@ int rptq_kv_calib_minmax(const void *kv, int dtype, int B, int H, int64_t S, int
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
-    KvCalibArgs a{kv, dtype, B, H, S, D, ch_max, ch_min, accumulate, (cudaStream_t)stream, d.num_sms};
+    KvCalibArgs a{kv, dtype, B, H, S, D, ch_max, ch_min, accumulate, d.err, (cudaStream_t)stream, d.num_sms};
     return cuda_status(launch_kv_calib(a));
 }
 

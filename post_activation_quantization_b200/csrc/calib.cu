@@ -18,6 +18,7 @@
 // gamma < 0) is the same value as taking the max of the per-token fmaf results.
 #include <algorithm>
 
+#include "kv_stream.cuh"
 #include "launch.h"
 #include "row_pipeline.cuh"
 
@@ -221,6 +222,96 @@ __global__ void __launch_bounds__(256)
         atomic_max_f32(ch_max + h * D + d, m);
         atomic_min_f32(ch_min + h * D + d, n);
     }
+}
+
+// Ring form for 16-bit caches whose shape passes kv_ring_shape_ok (stages of kv_stream.cuh): the
+// eight pieces of a stage that a thread reads all hold its channel group, so it keeps one packed
+// running max / min; when the head changes (and at the end) the lanes sharing a channel group
+// are folded by shuffles and the result goes to the outputs with the same integer atomics.
+template <typename T>
+__device__ __forceinline__ void kv_calib_flush(const RawAcc<T> &acc, int h, int D, float *ch_max, float *ch_min)
+{
+    const int lane = threadIdx.x & 31, npr = D >> 3, col = threadIdx.x & (npr - 1);
+    float m[8], n[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        m[e] = acc.get_max(e);
+        n[e] = acc.get_min(e);
+    }
+    for (int o = npr; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            m[e] = fmaxf(m[e], __shfl_xor_sync(FULL, m[e], o));
+            n[e] = fminf(n[e], __shfl_xor_sync(FULL, n[e], o));
+        }
+    if (lane < npr || npr >= 32)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            atomic_max_f32(ch_max + h * D + col * 8 + e, m[e]);
+            atomic_min_f32(ch_min + h * D + col * 8 + e, n[e]);
+        }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(KVR_THREADS, 2)
+    kv_calib_ring(const T *__restrict__ x, int B, int H, int SPB, int D, float *ch_max, float *ch_min, int *err)
+{
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_abort;
+    uint8_t *ring = smem;
+    const uint32_t bar0 = smem_u32(smem + (size_t)KVR_NS * KVR_STAGE);
+    const int tid = threadIdx.x;
+    const int64_t total = (int64_t)B * H * SPB;
+    const int64_t j0 = total * blockIdx.x / gridDim.x, j1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int n = (int)(j1 - j0);
+    if (n <= 0) return;
+    KvStagePos prod;  // thread 0: the next stage to load
+    auto issue = [&](uint32_t s) {
+        const uint8_t *src = reinterpret_cast<const uint8_t *>(x) + prod.mem_index(H, SPB) * KVR_STAGE;
+        mbar_expect_tx(bar0 + 8u * s, KVR_STAGE);
+        bulk_g2s(smem_u32(ring + (size_t)s * KVR_STAGE), src, KVR_STAGE, bar0 + 8u * s);
+        prod.advance(B, H, SPB);
+    };
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < KVR_NS; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+        prod.set(j0, total, B, SPB);
+        for (int s = 0; s < KVR_NS && s < n; ++s) issue((uint32_t)s);
+    }
+    __syncthreads();
+    KvStagePos cur;
+    cur.set(j0, total, B, SPB);
+    RawAcc<T> acc;
+    acc.init();
+    int acc_h = cur.h;
+    uint32_t slot = 0, phase = 0;
+    for (int i = 0; i < n; ++i) {
+        if (cur.h != acc_h) {  // the same in every thread
+            kv_calib_flush<T>(acc, acc_h, D, ch_max, ch_min);
+            acc.init();
+            acc_h = cur.h;
+        }
+        if (!mbar_wait_bounded(bar0 + 8u * slot, phase, err)) s_abort = 1;
+        const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)slot * KVR_STAGE);
+        uint4 xb[KVR_PPT];
+#pragma unroll
+        for (int k = 0; k < KVR_PPT; ++k) xb[k] = src[tid + k * KVR_THREADS];
+#pragma unroll
+        for (int k = 0; k < KVR_PPT; ++k) acc.add(xb[k]);
+        __syncthreads();  // the slot has been read
+        if (s_abort) break;
+        if (tid == 0 && i + KVR_NS < n) {
+            fence_proxy_async_smem();
+            issue(slot);
+        }
+        cur.advance(B, H, SPB);
+        if (++slot == KVR_NS) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    kv_calib_flush<T>(acc, acc_h, D, ch_max, ch_min);
 }
 
 // ---- LayerNorm mode ------------------------------------------------------------------------
@@ -459,8 +550,29 @@ cudaError_t launch_calib(const CalibArgs &a)
 }
 
 template <typename T>
+static cudaError_t launch_kv_calib_ring(const KvCalibArgs &a)
+{
+    const int SPB = (int)(a.S / kv_ring_rows(a.D));
+    auto kern = kv_calib_ring<T>;
+    const size_t smem = (size_t)KVR_NS * KVR_STAGE + 8 * KVR_NS;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t total = (int64_t)a.B * a.H * SPB;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * a.num_sms, total);
+    kern<<<(unsigned)grid, KVR_THREADS, smem, a.stream>>>((const T *)a.x, a.B, a.H, SPB, a.D, a.ch_max, a.ch_min,
+                                                          a.err);
+    return cudaGetLastError();
+}
+
+template <typename T>
 static cudaError_t launch_kv_calib_t(const KvCalibArgs &a)
 {
+    if constexpr (sizeof(T) == 2)
+        if (kv_ring_shape_ok(a.B, a.H, a.S, a.D, 2)) return launch_kv_calib_ring<T>(a);
     const int nbh = a.B * a.H;
     int64_t gy = std::max<int64_t>(1, ((int64_t)a.num_sms * 6 + nbh - 1) / nbh);
     gy = std::min<int64_t>(gy, std::max<int64_t>(1, a.S / 64));

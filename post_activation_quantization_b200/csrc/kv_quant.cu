@@ -10,13 +10,14 @@
 // whole run of rows.  Per element: a correctly rounded x / s, the clamp, the rounding constant
 // 1.5*2^23 (which leaves the code in the low bits of the float), and a shifted sum of those bit
 // patterns minus a known constant is the packed word; rows are stored as whole words.
+// Ring kernel (16-bit caches cut into whole 32-KB stages, kv_stream.cuh): the default shape.
 // Warp kernel (D/DPT divides 32): a work unit is 64 rows of one (b, h) block; units are ordered
 // (h, b, chunk) and every warp of a one-wave grid takes a contiguous range of them, reloading its
 // coefficients only when the head changes.  CTA kernel
 // (other D): one CTA per (b, h) block.
 #include <algorithm>
 
-#include "common.cuh"
+#include "kv_stream.cuh"
 #include "launch.h"
 
 namespace rptq {
@@ -216,53 +217,12 @@ __global__ void __launch_bounds__(256, 2)
     }
 }
 
-// Ring kernel (16-bit caches; D/8 a power of two <= 256; S a multiple of the stage rows 8192/D).
-// The work is cut into stages of 16 KB of the cache (8192/D whole rows of one (b, h) block,
-// contiguous in memory) and a stage's codes are 1024*BITS contiguous bytes of the output.
-// Stages are ordered (tensor, h, b, chunk) and every CTA of a one-wave grid takes a contiguous
-// range of them, so it crosses at most a couple of heads.  Thread 0 streams the stages into a
-// ring of KVR_NS shared-memory slots by bulk asynchronous copies (mbarrier completion, never
-// multicast); each thread turns its four 16-byte pieces (8 channels each; piece p of a stage
-// sits at p*16 in the slot and its codes at p*BITS in the code buffer, whatever D is) into
-// codes, and thread 0 writes the stage's codes with one bulk copy from one of two code buffers.
-constexpr int KVR_THREADS = 256;
-constexpr uint32_t KVR_STAGE = 16384;
-constexpr int KVR_PIECES = KVR_STAGE / 16;
-constexpr int KVR_PPT = KVR_PIECES / KVR_THREADS;
-constexpr int KVR_NS = 6;
-
+// Ring kernel (16-bit caches whose shape passes kv_ring_shape_ok; stages of kv_stream.cuh).
+// Each thread turns its eight pieces into codes (piece p's codes sit at p*BITS in the code
+// buffer, whatever D is: a stage's codes are 2048*BITS contiguous bytes of the output), and
+// thread 0 writes them with one bulk copy from one of two code buffers.
 template <int BITS>
 constexpr size_t kv_ring_smem() { return (size_t)KVR_NS * KVR_STAGE + 2 * KVR_PIECES * BITS + 8 * KVR_NS; }
-
-// A stage's place in (tensor, h, b, chunk) order, advanced without divisions.
-struct KvStagePos {
-    int ti, h, b, chunk;
-    __device__ __forceinline__ void set(int64_t j, int64_t per_t, int B, int SPB)
-    {
-        ti = (int)(j / per_t);
-        int64_t r = j - ti * per_t;
-        const int64_t per_h = (int64_t)B * SPB;
-        h = (int)(r / per_h);
-        r -= h * per_h;
-        b = (int)(r / SPB);
-        chunk = (int)(r - (int64_t)b * SPB);
-    }
-    __device__ __forceinline__ void advance(int B, int H, int SPB)
-    {
-        if (++chunk == SPB) {
-            chunk = 0;
-            if (++b == B) {
-                b = 0;
-                if (++h == H) {
-                    h = 0;
-                    ++ti;
-                }
-            }
-        }
-    }
-    // stage number within its tensor in memory order (b, h, chunk)
-    __device__ __forceinline__ int64_t mem_index(int H, int SPB) const { return ((int64_t)b * H + h) * SPB + chunk; }
-};
 
 template <typename T, int BITS>
 __global__ void __launch_bounds__(KVR_THREADS, 2)
@@ -421,7 +381,7 @@ static cudaError_t launch_kv_ring(const KvArgs &a)
     int sel[2] = {0, 1}, nt = 0;
     if (a.k) sel[nt++] = 0;
     if (a.v) sel[nt++] = 1;
-    const int SPB = (int)(a.S / (8192 / a.D));
+    const int SPB = (int)(a.S / kv_ring_rows(a.D));
     auto kern = kv_quant_ring<T, BITS>;
     const size_t smem = kv_ring_smem<BITS>();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -436,24 +396,11 @@ static cudaError_t launch_kv_ring(const KvArgs &a)
     return cudaGetLastError();
 }
 
-// The ring kernel's shape rule: 16-bit elements, D/8 a power of two dividing the 256 threads,
-// whole stages of 8192/D rows per (b, h) block, and a stage count the grid split keeps in int.
-static bool kv_ring_ok(const KvArgs &a, int esize)
-{
-    if (esize != 2 || a.D % 8 != 0 || a.D > 2048) return false;
-    const int npr = a.D / 8;
-    if ((npr & (npr - 1)) != 0) return false;
-    const int64_t sr = 8192 / a.D;
-    if (a.S % sr != 0) return false;
-    const int64_t per_t = (int64_t)a.B * a.H * (a.S / sr);
-    return per_t * 2 < 0x7fffffffLL && a.S / sr < 0x7fffffffLL;
-}
-
 template <typename T>
 static cudaError_t launch_kv_d(const KvArgs &a)
 {
     if constexpr (sizeof(T) == 2)
-        if (kv_ring_ok(a, 2)) return a.bits == 4 ? launch_kv_ring<T, 4>(a) : launch_kv_ring<T, 3>(a);
+        if (kv_ring_shape_ok(a.B, a.H, a.S, a.D, 2)) return a.bits == 4 ? launch_kv_ring<T, 4>(a) : launch_kv_ring<T, 3>(a);
     // warp kernel when the 8-channel groups of a row tile a warp evenly (D in 8, 16, ..., 256)
     if (a.D % 8 == 0 && a.D <= 256 && 32 % (a.D / 8) == 0 && a.S <= 0x7fffffffLL)
         return a.bits == 4 ? launch_kv_warp<T, 4>(a) : launch_kv_warp<T, 3>(a);

@@ -48,6 +48,7 @@ struct KvCalibArgs {
     int D;
     float *ch_max, *ch_min;
     int accumulate;
+    int *err;
     cudaStream_t stream;
     int num_sms;
 };

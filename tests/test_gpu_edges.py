@@ -125,7 +125,7 @@ def test_calib_layernorm_constant_and_offset_rows(dtype, C, all_offset):
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 def test_kv_quant_huge_zero_point_integer_path(dtype, S):
     """Zero points beyond +-2^21 take the integer rounding path; codes are still exact (S = 40:
-    the warp kernel; S = 128: whole 16 KB stages, the streaming-ring kernel)."""
+    the warp kernel; S = 128: whole 32 KB stages, the streaming-ring kernel)."""
     B, H, D, g, bits = 2, 3, 128, 4, 3
     mk = synthetic.channel_model(H * D, 17, tag=1)
     k = synthetic.kv_cache(B, H, S, D, mk, 17, "k", dtype)

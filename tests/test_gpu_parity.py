@@ -208,7 +208,11 @@ def test_ln_reorder_is_ln_then_gather():
 
 # ---------------------------------------------------------------- K/V cache
 @pytest.mark.parametrize("dtype", DTYPES)
-@pytest.mark.parametrize("B,H,S,D", [(2, 3, 37, 128), (1, 2, 5, 40), (3, 1, 300, 8), (1, 4, 64, 256)])
+@pytest.mark.parametrize("B,H,S,D", [(2, 3, 37, 128), (1, 2, 5, 40), (3, 1, 300, 8), (1, 4, 64, 256),
+                                     # whole 32 KB stages (16-bit): the streaming-ring kernel; the
+                                     # last case has more stages than CTAs, so CTAs cross heads
+                                     (2, 3, 128, 128), (1, 2, 2048, 8), (2, 5, 512, 32), (1, 2, 8, 2048),
+                                     (2, 4, 16384, 128)])
 def test_kv_calib_bit_exact(dtype, B, H, S, D):
     m = synthetic.channel_model(H * D, S, tag=1)
     kv = synthetic.kv_cache(B, H, S, D, m, S, "k", dtype=dtype)
@@ -226,10 +230,11 @@ def test_kv_calib_bit_exact(dtype, B, H, S, D):
 KV_CASES = [("f16", 2, 4, 33, 128, 6, 3), ("bf16", 1, 3, 17, 64, 5, 4), ("f32", 2, 2, 9, 128, 8, 4),
             ("f16", 1, 2, 11, 40, 4, 3), ("bf16", 3, 5, 7, 256, 7, 3), ("bf16", 2, 3, 300, 128, 6, 3),
             ("f16", 1, 2, 5, 512, 4, 4), ("bf16", 2, 2, 130, 32, 5, 3), ("f32", 1, 3, 19, 8, 3, 4),
-            # whole 16 KB stages per (b, h) block (S a multiple of 8192 / D): the streaming-ring kernel
-            ("bf16", 2, 3, 128, 128, 6, 3), ("f16", 2, 3, 192, 128, 5, 4), ("bf16", 1, 4, 256, 64, 7, 4),
-            ("f16", 3, 2, 64, 256, 6, 3), ("bf16", 1, 2, 8, 2048, 4, 3), ("f16", 1, 3, 1024, 8, 3, 4),
-            ("bf16", 2, 5, 512, 32, 9, 3)]
+            # whole 32 KB stages per (b, h) block (S a multiple of 16384 / D): the streaming-ring kernel
+            ("bf16", 2, 3, 128, 128, 6, 3), ("f16", 2, 3, 384, 128, 5, 4), ("bf16", 1, 4, 256, 64, 7, 4),
+            ("f16", 3, 2, 64, 256, 6, 3), ("bf16", 1, 2, 8, 2048, 4, 3), ("f16", 1, 3, 2048, 8, 3, 4),
+            ("bf16", 2, 5, 512, 32, 9, 3), ("bf16", 1, 3, 192, 128, 5, 3),
+            ("bf16", 2, 4, 4096, 128, 6, 3)]  # more stages than CTAs: CTAs cross heads and tensors
 
 
 @pytest.mark.parametrize("dtype,B,H,S,D,g,bits", KV_CASES)
