@@ -13,12 +13,18 @@
 // bytes (A4: one word per lane) or 3 bytes (A3: 24 lanes load the warp's 96 bytes as words and
 // each lane assembles its 3 bytes with two shuffles and a funnel shift).  Rows layout: warp w
 // of a CTA owns the 256-channel spans w, w + WR, w + 2 WR, ... of every row it walks, with
-// their (s, 2^23 + z) in registers.  BHSD layout: one CTA per (b, h) block of S rows x D
-// channels (contiguous), a warp covers 256 / D consecutive rows per store, so a lane's channel
-// position is fixed.  Other shapes use the general kernel (DPT consecutive channels per thread).
+// their (s, 2^23 + z) in registers.  BHSD layout: a warp covers 256 / D consecutive rows per
+// store, so a lane's channel position is fixed; warps take contiguous ranges of (h, b, chunk)
+// units.  Other shapes use the general kernel (DPT consecutive channels per thread).
+//
+// Ring kernel (BHSD layout, 16-bit output, shapes that pass kv_ring_shape_ok): the stage
+// decomposition of kv_stream.cuh run in reverse.  A stage is 32 KB of output (2048 pieces of 8
+// channels) and 2048*BITS contiguous bytes of codes; thread 0 streams the codes into a ring of
+// shared slots, every thread decodes its eight pieces into one of two 32 KB staging buffers, and
+// thread 0 writes the stage with one bulk copy.
 #include <algorithm>
 
-#include "common.cuh"
+#include "kv_stream.cuh"
 #include "launch.h"
 
 namespace rptq {
@@ -316,6 +322,139 @@ __global__ void __launch_bounds__(NSPAN <= 2 ? 1024 : 512)
     }
 }
 
+// Eight fp32 values -> one 16-byte chunk of 16-bit values (round to nearest even).
+template <typename T> __device__ __forceinline__ uint4 pack8(const float (&v)[8]);
+template <> __device__ __forceinline__ uint4 pack8<__nv_bfloat16>(const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<const uint32_t *>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+template <> __device__ __forceinline__ uint4 pack8<__half>(const float (&v)[8])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const __half2 p = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<const uint32_t *>(&p);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int BITS>
+constexpr size_t dq_ring_smem() { return (size_t)KVR_NS * KVR_PIECES * BITS + 2 * (size_t)KVR_STAGE + 8 * KVR_NS; }
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(KVR_THREADS, 2)
+    dequant_bhsd_ring(const uint8_t *__restrict__ codes, int B, int H, int SPB, int D,
+                      const int32_t *__restrict__ cluster, const float *__restrict__ scale,
+                      const int32_t *__restrict__ zero, int g, T *__restrict__ out, int *err)
+{
+    constexpr uint32_t CBYTES = KVR_PIECES * BITS;  // codes of one stage
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int s_abort;
+    uint8_t *stage = smem;                                  // 2 x 32 KB of output
+    uint8_t *ring = smem + 2 * (size_t)KVR_STAGE;           // KVR_NS x CBYTES of codes
+    const uint32_t bar0 = smem_u32(ring + (size_t)KVR_NS * CBYTES);
+    const int tid = threadIdx.x;
+    const int64_t total = (int64_t)B * H * SPB;
+    const int64_t j0 = total * blockIdx.x / gridDim.x, j1 = total * (blockIdx.x + 1) / gridDim.x;
+    const int n = (int)(j1 - j0);
+    if (n <= 0) return;
+    KvStagePos prod;  // thread 0: the next stage whose codes to load
+    auto issue = [&](uint32_t s) {
+        mbar_expect_tx(bar0 + 8u * s, CBYTES);
+        bulk_g2s(smem_u32(ring + (size_t)s * CBYTES), codes + prod.mem_index(H, SPB) * CBYTES, CBYTES, bar0 + 8u * s);
+        prod.advance(B, H, SPB);
+    };
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < KVR_NS; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+        prod.set(j0, total, B, SPB);
+        for (int s = 0; s < KVR_NS && s < n; ++s) issue((uint32_t)s);
+    }
+    __syncthreads();
+    KvStagePos cur;
+    cur.set(j0, total, B, SPB);
+    const int col = tid & ((D >> 3) - 1);  // the thread's 8-channel group in every piece
+    float sc[8], nzf[8];
+    bool exact = true;
+    int cur_h = -1;
+    uint32_t slot = 0, phase = 0;
+    for (int i = 0; i < n; ++i) {
+        if (cur.h != cur_h) {
+            exact = true;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int k = checked_cluster(cluster, cur.h * D + col * 8 + e, g, err);
+                sc[e] = scale[k];
+                const int z = zero[k];
+                const bool ok = z > -(1 << 23) + 16 && z < (1 << 23) - 16;
+                exact &= ok;
+                nzf[e] = -(float)((1 << 23) + (ok ? z : 0));
+            }
+            cur_h = cur.h;
+        }
+        if (!mbar_wait_bounded(bar0 + 8u * slot, phase, err)) s_abort = 1;
+        const uint8_t *cs = ring + (size_t)slot * CBYTES;
+        uint4 *dst = reinterpret_cast<uint4 *>(stage + (size_t)(i & 1) * KVR_STAGE);
+#pragma unroll
+        for (int k = 0; k < KVR_PPT; ++k) {
+            const int p = tid + k * KVR_THREADS;
+            uint32_t grp;
+            if constexpr (BITS == 4) {
+                grp = *reinterpret_cast<const uint32_t *>(cs + 4 * p);
+            } else {  // 3 bytes at 3p: the aligned word holding the first, the next one only
+                      // when the bytes cross into it (never past the slot), and a funnel shift
+                const uint32_t *w = reinterpret_cast<const uint32_t *>(cs) + ((3 * p) >> 2);
+                const uint32_t sh = (uint32_t)((3 * p) & 3) * 8u;
+                grp = __funnelshift_r(w[0], sh > 8u ? w[1] : 0u, sh) & 0xffffffu;
+            }
+            float v[8];
+            if (exact) {
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const uint32_t q0 = (grp >> (BITS * e)) & ((1u << BITS) - 1), q1 = (grp >> (BITS * (e + 1))) & ((1u << BITS) - 1);
+                    const f32x2 x = add2(mk2(__uint_as_float(0x4B000000u | q0), __uint_as_float(0x4B000000u | q1)),
+                                         mk2(nzf[e], nzf[e + 1]));
+                    const f32x2 y = mul2(x, mk2(sc[e], sc[e + 1]));
+                    v[e] = lo2(y);
+                    v[e + 1] = hi2(y);
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int kc = checked_cluster(cluster, cur.h * D + col * 8 + e, g, err);
+                    v[e] = sc[e] * (float)((int)((grp >> (BITS * e)) & ((1u << BITS) - 1)) - zero[kc]);
+                }
+            }
+            dst[p] = pack8<T>(v);
+        }
+        // the previous stage's output copy has finished reading its buffer, which the stage after
+        // this one rewrites
+        if (tid == 0) bulk_wait_read<0>();
+        __syncthreads();  // codes slot read, the stage's output complete
+        if (s_abort) break;
+        if (tid == 0) {
+            fence_proxy_async_smem();
+            bulk_s2g(reinterpret_cast<uint8_t *>(out) + cur.mem_index(H, SPB) * KVR_STAGE, smem_u32(dst), KVR_STAGE);
+            bulk_commit();
+            if (i + KVR_NS < n) issue(slot);
+        }
+        cur.advance(B, H, SPB);
+        if (++slot == KVR_NS) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+}
+
 // BHSD layout, D % 8 == 0 and (D/8) divides 32.  A span is the RPW = 256/D consecutive rows one
 // warp-wide store covers; a work unit is up to 32 spans of one (b, h) block; units are ordered
 // (h, b, chunk) and every warp of a one-wave grid takes a contiguous range of them.  A lane's
@@ -454,9 +593,31 @@ static cudaError_t launch_rows_span(const DequantArgs &a, int WR)
 }
 
 template <typename T, int BITS>
+static cudaError_t launch_dq_ring(const DequantArgs &a)
+{
+    const int SPB = (int)(a.S / kv_ring_rows(a.D));
+    auto kern = dequant_bhsd_ring<T, BITS>;
+    const size_t smem = dq_ring_smem<BITS>();
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    const int64_t total = a.n0 * a.n1 * SPB;
+    const int64_t grid = std::min<int64_t>((int64_t)per_sm * a.num_sms, total);
+    kern<<<(unsigned)grid, KVR_THREADS, smem, a.stream>>>(a.codes, (int)a.n0, a.n1, SPB, a.D, a.cluster, a.scale,
+                                                          a.zero, a.g, (T *)a.out, a.err);
+    return cudaGetLastError();
+}
+
+template <typename T, int BITS>
 static cudaError_t launch_dq_b(const DequantArgs &a)
 {
     const bool aligned = ((uintptr_t)a.codes % 4 == 0) && ((uintptr_t)a.out % 16 == 0);
+    if constexpr (sizeof(T) == 2)  // bulk copies: both bases 16-byte aligned (checked by the caller)
+        if (a.layout == RPTQ_LAYOUT_BHSD && a.n0 <= 0x7fffffff && kv_ring_shape_ok((int)a.n0, a.n1, a.S, a.D, 2))
+            return launch_dq_ring<T, BITS>(a);
     if (a.layout == RPTQ_LAYOUT_BHSD) {
         // word loads need every (b, h) block of codes to start on a 4-byte boundary
         const bool blocks4 = ((int64_t)a.S * a.D * BITS / 8) % 4 == 0;

@@ -284,11 +284,16 @@ def test_dequant_rows_bit_exact(out_dtype, rows, C, bits):
     assert torch.equal(out.cpu(), ref)
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("B,H,S,D,bits", [(2, 3, 5, 128, 3), (1, 2, 4, 40, 4), (1, 4, 3, 64, 4), (2, 2, 67, 128, 3),
                                           (1, 3, 9, 256, 4), (2, 1, 35, 8, 3), (2, 1, 36, 8, 3), (1, 2, 13, 32, 3),
-                                          (1, 1, 16, 16, 4)])
+                                          (1, 1, 16, 16, 4),
+                                          # whole 32 KB output stages (16-bit outputs): the ring kernel;
+                                          # the last case has more stages than CTAs
+                                          (2, 3, 128, 128, 3), (1, 4, 256, 64, 4), (2, 2, 64, 256, 3),
+                                          (1, 2, 2048, 8, 4), (1, 2, 8, 2048, 3), (2, 4, 8192, 128, 3)])
 @pytest.mark.parametrize("huge_z", [False, True])
-def test_dequant_bhsd_bit_exact(B, H, S, D, bits, huge_z):
+def test_dequant_bhsd_bit_exact(B, H, S, D, bits, huge_z, out_dtype):
     rng = np.random.default_rng(B * H * S * D)
     g = 6
     labels = rng.integers(0, g, H * D).astype(np.int32)
@@ -300,9 +305,9 @@ def test_dequant_bhsd_bit_exact(B, H, S, D, bits, huge_z):
     packed = oracle.pack(q, bits).reshape(B, H, S, D * bits // 8)
     out = rptq.rptq_dequant(torch.from_numpy(packed).to(DEV), torch.from_numpy(labels).to(DEV),
                             torch.from_numpy(s).to(DEV), torch.from_numpy(z).to(DEV), bits,
-                            out_dtype=torch.float32, layout=rptq.RPTQ_LAYOUT_BHSD, D=D)
-    ref = oracle.kv_dequant(packed, D, labels, s, z, bits)
-    assert np.array_equal(out.cpu().numpy(), ref)
+                            out_dtype=out_dtype, layout=rptq.RPTQ_LAYOUT_BHSD, D=D)
+    ref = torch.from_numpy(oracle.kv_dequant(packed, D, labels, s, z, bits)).to(out_dtype)
+    assert torch.equal(out.cpu(), ref)
 
 
 # ---------------------------------------------------------------- device error word
