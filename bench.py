@@ -44,6 +44,7 @@ from post_activation_quantization_b200 import workloads as W  # noqa: E402
 
 METRIC = "fused LN+reorder+cluster-quant GB/s & Mtokens/s; % of B200 HBM peak"
 DEFAULT_WORKLOAD = "opt175b-12288"
+L2_BYTES = 126 * 2 ** 20
 HBM_FALLBACK_GBS = 6650.0
 
 
@@ -56,6 +57,11 @@ def peaks():
     return HBM_FALLBACK_GBS, "fallback"
 
 
+def has_act(w: W.Workload) -> bool:
+    """Whether the workload carries the activation path (the K/V-only workload does not)."""
+    return w.T > 0 and w.C > 0
+
+
 # ------------------------------------------------------------------------------------------
 class Step:
     """Device buffers of one rank and the sequence of library calls that makes a step."""
@@ -65,20 +71,22 @@ class Step:
         self.r = rptq
         self.w, self.dev = w, device
         self.kvw = w.kv
-        dt = synthetic.torch_dtype(w.dtype)
-        m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
-        g, b = synthetic.ln_params(w.C, w.seed)
-        self.gamma, self.beta = g.to(device), b.to(device)
-        # every rank draws its own tokens of the same model
-        self.xcal = synthetic.activations(w.T_cal or w.T, m, w.seed + 7919 * rank, dtype=w.dtype,
-                                          calibration=True, device=device)
-        self.x = synthetic.activations(w.T, m, w.seed + 7919 * rank, dtype=w.dtype, device=device)
-        self.mx = torch.empty(w.C, dtype=torch.float32, device=device)
-        self.mn = torch.empty_like(self.mx)
-        self.km = self._km_out(w.C, w.g)
-        self.ws = torch.empty(rptq.rptq_kmeans_workspace_size(w.C, w.g), dtype=torch.uint8, device=device)
-        self.codes = torch.empty((w.T, w.C * w.bits // 8), dtype=torch.uint8, device=device)
-        self.xhat = torch.empty((w.T, w.C), dtype=dt, device=device)
+        self.act = has_act(w)  # the K/V-only workload has no activation stages
+        if self.act:
+            dt = synthetic.torch_dtype(w.dtype)
+            m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
+            g, b = synthetic.ln_params(w.C, w.seed)
+            self.gamma, self.beta = g.to(device), b.to(device)
+            # every rank draws its own tokens of the same model
+            self.xcal = synthetic.activations(w.T_cal or w.T, m, w.seed + 7919 * rank, dtype=w.dtype,
+                                              calibration=True, device=device)
+            self.x = synthetic.activations(w.T, m, w.seed + 7919 * rank, dtype=w.dtype, device=device)
+            self.mx = torch.empty(w.C, dtype=torch.float32, device=device)
+            self.mn = torch.empty_like(self.mx)
+            self.km = self._km_out(w.C, w.g)
+            self.ws = torch.empty(rptq.rptq_kmeans_workspace_size(w.C, w.g), dtype=torch.uint8, device=device)
+            self.codes = torch.empty((w.T, w.C * w.bits // 8), dtype=torch.uint8, device=device)
+            self.xhat = torch.empty((w.T, w.C), dtype=dt, device=device)
         if self.kvw:
             k = self.kvw
             mk = synthetic.channel_model(k.channels, w.seed, k.outlier_frac, k.outlier_factor, tag=1)
@@ -114,16 +122,18 @@ class Step:
     # without `accumulate` is an init launch + the reduction; a KMeans call is two launches (the
     # workspace clear and the cooperative KMeans kernel).
     def stages(self):
-        w, k = self.w, self.kvw
+        w, k, a = self.w, self.kvw, self.act
         n = w.T * w.C
-        st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2)]
+        st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2)] if a else []
         if k:
             st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4)]
-        st += [("kmeans", 0, 2 * (3 if k else 1)),
-               ("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+        st += [("kmeans", 0, 2 * ((1 if a else 0) + (2 if k else 0)))]
+        if a:
+            st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
         if k:
             st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
-        st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
+        if a:
+            st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
         if k:
             st += [("dequant_kv", 2 * W.bytes_dequant(k.elems, k.dtype, k.bits), 2)]
         return st
@@ -140,10 +150,11 @@ class Step:
             if ev is not None:
                 ev[name][i].record(main)
 
-        mark("calib_ln", 0)
-        r.rptq_calib_minmax(self.xcal, self.gamma, self.beta, w.eps, ch_max=self.mx, ch_min=self.mn)
-        mark("calib_ln", 1)
-        pdist.allreduce_minmax(self.mx, self.mn)
+        if self.act:
+            mark("calib_ln", 0)
+            r.rptq_calib_minmax(self.xcal, self.gamma, self.beta, w.eps, ch_max=self.mx, ch_min=self.mn)
+            mark("calib_ln", 1)
+            pdist.allreduce_minmax(self.mx, self.mn)
         if k:
             mark("kv_calib", 0)
             r.rptq_kv_calib_minmax(self.k, ch_max=self.kst[0], ch_min=self.kst[1])
@@ -161,25 +172,28 @@ class Step:
             with torch.cuda.stream(self.side[1]):
                 r.rptq_kmeans(self.kst[2], self.kst[3], k.g, k.iters, k.bits, workspace=self.wsv, out=self.kmv,
                               stream=self.side[1])
-        r.rptq_kmeans(self.mx, self.mn, w.g, w.iters, w.bits, workspace=self.ws, out=self.km)
+        if self.act:
+            r.rptq_kmeans(self.mx, self.mn, w.g, w.iters, w.bits, workspace=self.ws, out=self.km)
         if k:
             for s in self.side:
                 main.wait_stream(s)
         mark("kmeans", 1)
-        mark("ln_reorder_quant", 0)
-        r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
-                                self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
-        mark("ln_reorder_quant", 1)
+        if self.act:
+            mark("ln_reorder_quant", 0)
+            r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
+                                    self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
+            mark("ln_reorder_quant", 1)
         if k:
             mark("kv_quant", 0)
             r.rptq_kv_quant(self.k, self.v, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],
                             self.kmv["labels"], self.kmv["scale"], self.kmv["zero"], k.bits,
                             k_codes=self.kq, v_codes=self.vq)
             mark("kv_quant", 1)
-        mark("dequant_act", 0)
-        r.rptq_dequant(self.codes, self.km["col_cluster"], self.km["scale"], self.km["zero"], w.bits,
-                       out=self.xhat)
-        mark("dequant_act", 1)
+        if self.act:
+            mark("dequant_act", 0)
+            r.rptq_dequant(self.codes, self.km["col_cluster"], self.km["scale"], self.km["zero"], w.bits,
+                           out=self.xhat)
+            mark("dequant_act", 1)
         if k:
             mark("dequant_kv", 0)
             r.rptq_dequant(self.kq, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"], k.bits,
@@ -325,7 +339,9 @@ def run_rptq(args):
         if b:
             kern[n]["gbs"] = round(b / (mean_ms * 1e-3) / 1e9, 1)
             kern[n]["frac_of_measured_hbm"] = round(b / (mean_ms * 1e-3) / 1e9 / hbm, 4)
-    kern["ln_reorder_quant"]["mtokens_per_s"] = round(w.T / (kern["ln_reorder_quant"]["ms_per_call"] * 1e-3) / 1e6, 2)
+    # tokens of the step: the activation batch, or the cache's B*S positions for the K/V-only workload
+    tok_stage, tokens = ("ln_reorder_quant", w.T) if step.act else ("kv_quant", w.kv.B * w.kv.S)
+    kern[tok_stage]["mtokens_per_s"] = round(tokens / (kern[tok_stage]["ms_per_call"] * 1e-3) / 1e6, 2)
     dom = max((n for n, b, _ in stages if b), key=lambda n: kern[n]["ms_per_call"])
     dom_bytes = kern[dom]["bytes_per_call"]
     ach = dom_bytes / (kern[dom]["ms_per_call"] * 1e-3) / 1e9
@@ -341,7 +357,7 @@ def run_rptq(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded per-channel uniform ranges with outlier channels)",
             "config": workload_config(w),
-            "mtokens_per_s": round(w.T * ws * args.steps / (ms * 1e-3) / 1e6, 3),
+            "mtokens_per_s": round(tokens * ws * args.steps / (ms * 1e-3) / 1e6, 3),
             "frac_of_measured_hbm": round(value / ws / hbm, 4),
             "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm,
                          "unit": "GB/s", "frac": round(ach / hbm, 4), "peak_kind": peak_kind,
@@ -373,9 +389,18 @@ def scaled_workload(args) -> W.Workload:
 
 
 def workload_config(w):
+    es = W.ESIZE
+    ins = [(w.T_cal or w.T) * w.C * es[w.dtype], w.T * w.C * es[w.dtype]] if has_act(w) else []
+    if w.kv:
+        ins += [w.kv.elems * es[w.kv.dtype]] * 2
+    streamed = sum(ins)
+    if min(ins) > L2_BYTES:
+        l2 = f"inputs larger than L2 (a step streams about {streamed / 1e9:.1f} GB of inputs), no flush needed"
+    else:
+        l2 = (f"some inputs fit in the 126 MB L2 (a step streams {streamed / 1e6:.0f} MB of inputs): "
+              "stage times are partly L2-warm, not HBM numbers")
     c = {"workload": w.name, "tokens": w.T, "channels": w.C, "calib_tokens": w.T_cal or w.T,
-         "g": w.g, "iters": w.iters, "bits": w.bits, "io_dtype": w.dtype,
-         "l2": "inputs larger than L2 (a step streams about 12 GB), no flush needed"}
+         "g": w.g, "iters": w.iters, "bits": w.bits, "io_dtype": w.dtype, "l2": l2}
     if w.kv:
         k = w.kv
         c["kv"] = {"B": k.B, "H": k.H, "S": k.S, "D": k.D, "dtype": k.dtype, "g": k.g,
@@ -386,9 +411,10 @@ def workload_config(w):
 def run_e2e(step: Step, args, dev, step_bytes, ws):
     """Same step through the public API with host inputs: each step copies its inputs from
     pinned host memory and reads the codes (and calibration results) back, inside the timing."""
-    ins = [step.xcal, step.x] + ([step.k, step.v] if step.kvw else [])
-    outs = [step.codes] + ([step.kq, step.vq] if step.kvw else []) + [step.km["R"], step.km["scale"],
-                                                                      step.km["zero"]]
+    ins = ([step.xcal, step.x] if step.act else []) + ([step.k, step.v] if step.kvw else [])
+    outs = ([step.codes] if step.act else []) + ([step.kq, step.vq] if step.kvw else [])
+    outs += [step.km["R"], step.km["scale"], step.km["zero"]] if step.act else \
+        [step.kmk["labels"], step.kmk["scale"], step.kmk["zero"]]
     h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
     for h, t in zip(h_in, ins):
         h.copy_(t)
@@ -435,19 +461,23 @@ class OracleSample:
         oracle.build()
         self.o, self.w = oracle, w
         gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
-        m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
-        self.gamma, self.beta = synthetic.ln_params(w.C, w.seed)
-        self.t_cal = max(4, int((w.T_cal or w.T) * frac))
-        self.t_x = max(4, int(w.T * frac))
-        self.xc = [oracle._f32(synthetic.activations(min(4096, self.t_cal - r0), m, w.seed + r0, dtype=w.dtype,
-                                                    calibration=True, device=gen_dev).cpu())
-                   for r0 in range(0, self.t_cal, 4096)]
-        self.x = oracle._f32(synthetic.activations(self.t_x, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
-        mx = mn = None
-        for xc in self.xc:
-            mx, mn = oracle.minmax_ln(xc, self.gamma, self.beta, w.eps, ch_max=mx, ch_min=mn)
-        self.mx, self.mn = mx, mn
-        self.desc = f"oracle (1 core) on {self.t_cal} calibration tokens and {self.t_x} tokens of the batch, full KMeans"
+        self.act = has_act(w)
+        self.desc = "oracle (1 core)"
+        if self.act:
+            m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
+            self.gamma, self.beta = synthetic.ln_params(w.C, w.seed)
+            self.t_cal = max(4, int((w.T_cal or w.T) * frac))
+            self.t_x = max(4, int(w.T * frac))
+            self.xc = [oracle._f32(synthetic.activations(min(4096, self.t_cal - r0), m, w.seed + r0, dtype=w.dtype,
+                                                        calibration=True, device=gen_dev).cpu())
+                       for r0 in range(0, self.t_cal, 4096)]
+            self.x = oracle._f32(synthetic.activations(self.t_x, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
+            mx = mn = None
+            for xc in self.xc:
+                mx, mn = oracle.minmax_ln(xc, self.gamma, self.beta, w.eps, ch_max=mx, ch_min=mn)
+            self.mx, self.mn = mx, mn
+            self.desc += f" on {self.t_cal} calibration tokens and {self.t_x} tokens of the batch"
+        self.desc += ", full KMeans"
         self.kv = []
         if w.kv:
             k = w.kv
@@ -461,13 +491,15 @@ class OracleSample:
                 self.kv.append((kvf, flat, kmx, kmn))
             self.desc += f", K and V with {self.s_s} of {k.S} sequence positions"
         self.desc += "; stage times scaled to the full step"
-        self.cal = oracle.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
+        self.cal = oracle.calibrate(self.mx, self.mn, w.g, w.iters, w.bits) if self.act else None
         self.kcal = [oracle.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits) for _, _, kmx, kmn in self.kv]
 
     def bytes_per_step(self) -> int:
         w = self.w
-        n = W.bytes_calib(w.T_cal or w.T, w.C, w.dtype) + W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits) \
-            + W.bytes_dequant(w.T * w.C, w.dtype, w.bits)
+        n = 0
+        if self.act:
+            n += W.bytes_calib(w.T_cal or w.T, w.C, w.dtype) + W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits) \
+                + W.bytes_dequant(w.T * w.C, w.dtype, w.bits)
         if w.kv:
             k = w.kv
             n += 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype) + \
@@ -477,7 +509,8 @@ class OracleSample:
     def time_kmeans(self) -> float:
         o, w = self.o, self.w
         t = time.perf_counter()
-        o.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
+        if self.act:
+            o.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
         for _, _, kmx, kmn in self.kv:
             o.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits)
         return time.perf_counter() - t
@@ -486,16 +519,17 @@ class OracleSample:
         """Seconds the token-parallel stages of a full step take, scaled from the sample."""
         o, w, cal = self.o, self.w, self.cal
         secs = 0.0
-        t = time.perf_counter()
-        for xc in self.xc:
-            o.minmax_ln(xc, self.gamma, self.beta, w.eps)
-        secs += (time.perf_counter() - t) / (self.t_cal / (w.T_cal or w.T))
-        t = time.perf_counter()
-        packed, _, _ = o.ln_reorder_quant(self.x, self.gamma, self.beta, cal["R"], cal["col_cluster"],
-                                          cal["scale"], cal["zero"], w.bits, eps=w.eps)
-        q = o.unpack(packed, w.C, w.bits)
-        o.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])
-        secs += (time.perf_counter() - t) / (self.t_x / w.T)
+        if self.act:
+            t = time.perf_counter()
+            for xc in self.xc:
+                o.minmax_ln(xc, self.gamma, self.beta, w.eps)
+            secs += (time.perf_counter() - t) / (self.t_cal / (w.T_cal or w.T))
+            t = time.perf_counter()
+            packed, _, _ = o.ln_reorder_quant(self.x, self.gamma, self.beta, cal["R"], cal["col_cluster"],
+                                              cal["scale"], cal["zero"], w.bits, eps=w.eps)
+            q = o.unpack(packed, w.C, w.bits)
+            o.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])
+            secs += (time.perf_counter() - t) / (self.t_x / w.T)
         if w.kv:
             k = w.kv
             t = time.perf_counter()

@@ -497,28 +497,60 @@ static cudaError_t launch_ln_simple(const CalibArgs &a)
     return cudaGetLastError();
 }
 
+template <typename T, int CPT>
+static int ln_calib_per_sm(int NT, size_t smem)
+{
+    int per_sm = 0;
+    if (cudaFuncSetAttribute(calib_ln_kernel<T, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_ln_kernel<T, CPT>, NT, smem) != cudaSuccess)
+        return 0;
+    return per_sm;
+}
+
 template <typename T>
 static cudaError_t launch_ln_d(const CalibArgs &a)
 {
     constexpr int VEC = Elem<T>::VEC;
     const int NCH = a.C / VEC;
-    int cpt = 0, nt = 0;
-    for (int k = 1; k <= 4; ++k) {
-        const int n = ((NCH + k - 1) / k + 31) / 32 * 32;
-        if (n <= 512) {
-            cpt = k;
-            nt = n;
-            break;
+    // fewest chunks per thread that keep the CTA within `lim` threads
+    auto pick = [&](int lim, int &cpt, int &nt) {
+        cpt = nt = 0;
+        for (int k = 1; k <= 4; ++k) {
+            const int n = ((NCH + k - 1) / k + 31) / 32 * 32;
+            if (n <= lim) {
+                cpt = k;
+                nt = n;
+                return;
+            }
         }
-    }
+    };
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
     int ns = 0;
-    for (int s = 8; s >= 4 && cpt; --s)
+    for (int s = 8; s >= 4; --s)
         if (quad_smem_layout(s, rowbytes, 2 * 8 * 32 * 4).total <= (size_t)a.max_smem) {
             ns = s;
             break;
         }
+    int cpt, nt;
+    pick(512, cpt, nt);
     if (!cpt || !ns) return launch_ln_simple<T>(a);
+    // Short rows are latency-bound: two CTAs of at most 256 threads (two independent row
+    // pipelines per SM) measured 49% -> 74% of the HBM copy rate at C = 4096 (fp16).  Taken only
+    // when the occupancy query confirms two CTAs per SM (at 4 chunks per thread the registers
+    // allow one, and one 256-thread CTA ran slower than one of 512).
+    int c2, n2;
+    pick(256, c2, n2);
+    if (c2 && c2 < 4) {
+        const size_t smem = quad_smem_layout(ns, rowbytes, 2 * 8 * 32 * 4).total;
+        const int per_sm = c2 == 1 ? ln_calib_per_sm<T, 1>(n2, smem)
+                           : c2 == 2 ? ln_calib_per_sm<T, 2>(n2, smem)
+                                     : ln_calib_per_sm<T, 3>(n2, smem);
+        if (per_sm >= 2) {
+            cpt = c2;
+            nt = n2;
+        }
+    }
     switch (cpt) {
     case 1: return launch_ln_t<T, 1>(a, nt, ns);
     case 2: return launch_ln_t<T, 2>(a, nt, ns);
