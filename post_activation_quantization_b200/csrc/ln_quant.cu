@@ -95,7 +95,24 @@ __device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int3
 {
     constexpr int VEC = Elem<T>::VEC;
     constexpr double QMAX = (double)((1 << BITS) - 1);
-    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC;
+    // every thread's share of R and col_cluster (int4 j4 = tid + u*NT; NT*CPT chunks cover the
+    // row, so NR int4 per thread suffice) is loaded first; thread 0 also pulls gamma and beta
+    // into L2 for the loads after the scatter
+    constexpr int NR = CPT * VEC / 4;
+    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC, C4 = C / 4;
+    if (tid == 0) {
+        prefetch_l2(gamma, (uint32_t)C * 4u);
+        prefetch_l2(beta, (uint32_t)C * 4u);
+    }
+    const int4 *R4 = reinterpret_cast<const int4 *>(R);
+    const int4 *K4 = reinterpret_cast<const int4 *>(col_cluster);
+    int4 r[NR], kk[NR];
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+        const int j4 = tid + u * NT;
+        r[u] = j4 < C4 ? R4[j4] : make_int4(-1, -1, -1, -1);
+        kk[u] = j4 < C4 ? K4[j4] : make_int4(0, 0, 0, 0);
+    }
     for (int c = tid; c < C; c += NT) {
         postab[c] = pbase;
         ctab[c] = 0;
@@ -106,33 +123,21 @@ __device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int3
         ctl[2 * k + 1] = (double)zero[k] / QMAX;
     }
     __syncthreads();
-    const int4 *R4 = reinterpret_cast<const int4 *>(R);
-    const int4 *K4 = reinterpret_cast<const int4 *>(col_cluster);
-    const int C4 = C / 4;
-    for (int b0 = tid; b0 < C4; b0 += 4 * NT) {  // four int4 of R and of col_cluster in flight
-        int4 r[4], kk[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j4 = b0 + u * NT;
-            r[u] = j4 < C4 ? R4[j4] : make_int4(-1, -1, -1, -1);
-            kk[u] = j4 < C4 ? K4[j4] : make_int4(0, 0, 0, 0);
-        }
+    for (int u = 0; u < NR; ++u) {
+        const int j4 = tid + u * NT;
+        if (j4 >= C4) continue;
+        const int rv[4] = {r[u].x, r[u].y, r[u].z, r[u].w}, kv[4] = {kk[u].x, kk[u].y, kk[u].z, kk[u].w};
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int j4 = b0 + u * NT;
-            if (j4 >= C4) continue;
-            const int rv[4] = {r[u].x, r[u].y, r[u].z, r[u].w}, kv[4] = {kk[u].x, kk[u].y, kk[u].z, kk[u].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = rv[i], k = kv[i];
-                if (c >= 0 && c < C) {
-                    postab[c] = pbase + codebuf_offset((uint32_t)(4 * j4 + i));
-                    ctab[c] = (uint16_t)((k >= 0 && k < g) ? k : 0);
-                } else {
-                    raise_error(err, RPTQ_DEVERR_REORDER);
-                }
-                if (k < 0 || k >= g) raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+        for (int i = 0; i < 4; ++i) {
+            const int c = rv[i], k = kv[i];
+            if (c >= 0 && c < C) {
+                postab[c] = pbase + codebuf_offset((uint32_t)(4 * j4 + i));
+                ctab[c] = (uint16_t)((k >= 0 && k < g) ? k : 0);
+            } else {
+                raise_error(err, RPTQ_DEVERR_REORDER);
             }
+            if (k < 0 || k >= g) raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
         }
     }
     __syncthreads();
