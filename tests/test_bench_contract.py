@@ -1,0 +1,41 @@
+"""The benchmark's JSON contract on the host: the reference arm (the oracle on a bounded sample)
+prints one line with the required keys for an activation workload and for the K/V-only one, and
+each workload's L2 statement follows its input sizes."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"}
+
+
+@pytest.mark.parametrize("workload", ["tiny-768", "kv-4096"])
+def test_reference_arm_line(workload):
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", workload, "--steps", "2",
+                          "--warmup", "1", "--ref-budget-s", "5"], cwd=ROOT, env=env, capture_output=True,
+                         text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert KEYS <= set(d)
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["value"] > 0 and d["e2e"]["value"] == d["value"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["config"]["workload"] == workload
+
+
+def test_l2_statement_follows_input_sizes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from post_activation_quantization_b200 import workloads as W
+    assert "larger than L2" in bench.workload_config(W.WORKLOADS["opt175b-12288"])["l2"]
+    assert "larger than L2" in bench.workload_config(W.WORKLOADS["kv-4096"])["l2"]
+    assert "fit in the 126 MB L2" in bench.workload_config(W.WORKLOADS["tiny-768"])["l2"]
+    assert "fit in the 126 MB L2" in bench.workload_config(W.WORKLOADS["opt6.7b-4096"])["l2"]
