@@ -3,8 +3,10 @@
 // Every entry point validates its arguments on the host, then enqueues kernels on the
 // caller's stream and returns without synchronising.  Nothing here allocates device memory:
 // the only library-owned device storage is the sticky error word below.
+#include <algorithm>
 #include <cstdio>
 #include <mutex>
+#include <unordered_map>
 
 #include "common.cuh"
 #include "launch.h"
@@ -24,6 +26,32 @@ struct DevInfo {
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
+
+// ---- launch settings, cached per kernel and device -------------------------------------
+struct SmemKey {
+    const void *f;
+    int dev;
+    bool operator==(const SmemKey &o) const { return f == o.f && dev == o.dev; }
+};
+struct OccKey {
+    const void *f;
+    int dev, threads;
+    size_t smem;
+    bool operator==(const OccKey &o) const
+    {
+        return f == o.f && dev == o.dev && threads == o.threads && smem == o.smem;
+    }
+};
+struct KeyHash {
+    size_t operator()(const SmemKey &k) const { return std::hash<const void *>()(k.f) * 31u + (size_t)k.dev; }
+    size_t operator()(const OccKey &k) const
+    {
+        return ((std::hash<const void *>()(k.f) * 31u + (size_t)k.dev) * 31u + (size_t)k.threads) * 31u + k.smem;
+    }
+};
+std::mutex g_launch_mu;
+std::unordered_map<SmemKey, size_t, KeyHash> g_smem_set;
+std::unordered_map<OccKey, int, KeyHash> g_occupancy;
 
 // Per-device facts, looked up once per device with that device current.
 int dev_info(DevInfo *out)
@@ -48,6 +76,48 @@ int dev_info(DevInfo *out)
 }
 
 }  // namespace
+
+cudaError_t kernel_smem(const void *func, size_t bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const SmemKey k{func, dev};
+    {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        auto it = g_smem_set.find(k);
+        if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+    }
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        size_t &v = g_smem_set[k];
+        v = std::max(v, bytes);
+    }
+    return e;
+}
+
+cudaError_t kernel_occupancy(int *per_sm, const void *func, int threads, size_t smem)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const OccKey k{func, dev, threads, smem};
+    {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        auto it = g_occupancy.find(k);
+        if (it != g_occupancy.end()) {
+            *per_sm = it->second;
+            return cudaSuccess;
+        }
+    }
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, func, threads, smem);
+    if (e == cudaSuccess) {
+        std::lock_guard<std::mutex> lock(g_launch_mu);
+        g_occupancy[k] = *per_sm;
+    }
+    return e;
+}
 
 int *device_error_word()
 {

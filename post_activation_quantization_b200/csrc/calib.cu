@@ -466,10 +466,10 @@ static cudaError_t launch_ln_t(const CalibArgs &a, int NT, int NS)
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
     const QuadSmem L = quad_smem_layout(NS, rowbytes, 2 * 8 * 32 * 4);
     auto kern = calib_ln_kernel<T, CPT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    cudaError_t e = kernel_smem((const void *)kern, L.total);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, L.total);
+    e = kernel_occupancy(&per_sm, (const void *)kern, NT, L.total);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t quads = (a.T + 3) / 4;
@@ -485,10 +485,10 @@ static cudaError_t launch_ln_simple(const CalibArgs &a)
     const size_t smem = (size_t)a.C * 12;
     if (smem > (size_t)a.max_smem) return cudaErrorInvalidValue;
     auto kern = calib_ln_simple_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, 256, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t grid = std::min<int64_t>(a.T, (int64_t)per_sm * a.num_sms);
@@ -501,9 +501,9 @@ template <typename T, int CPT>
 static int ln_calib_per_sm(int NT, size_t smem)
 {
     int per_sm = 0;
-    if (cudaFuncSetAttribute(calib_ln_kernel<T, CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+    if (kernel_smem((const void *)calib_ln_kernel<T, CPT>, smem) !=
             cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, calib_ln_kernel<T, CPT>, NT, smem) != cudaSuccess)
+        kernel_occupancy(&per_sm, (const void *)calib_ln_kernel<T, CPT>, NT, smem) != cudaSuccess)
         return 0;
     return per_sm;
 }
@@ -587,10 +587,10 @@ static cudaError_t launch_kv_calib_ring(const KvCalibArgs &a)
     const int SPB = (int)(a.S / kv_ring_rows(a.D));
     auto kern = kv_calib_ring<T>;
     const size_t smem = (size_t)KVR_NS * KVR_STAGE + 8 * KVR_NS;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, KVR_THREADS, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t total = (int64_t)a.B * a.H * SPB;

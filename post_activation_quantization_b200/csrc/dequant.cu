@@ -585,7 +585,7 @@ static cudaError_t launch_rows_span(const DequantArgs &a, int WR)
 {
     const int threads = WR * 32;
     int per_sm = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_rows_span<T, BITS, NSPAN>, threads, 0) !=
+    if (kernel_occupancy(&per_sm, (const void *)dequant_rows_span<T, BITS, NSPAN>, threads, 0) !=
             cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
@@ -601,10 +601,10 @@ static cudaError_t launch_dq_ring(const DequantArgs &a)
     const int SPB = (int)(a.S / kv_ring_rows(a.D));
     auto kern = dequant_bhsd_ring<T, BITS>;
     const size_t smem = dq_ring_smem<BITS>();
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, KVR_THREADS, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t total = a.n0 * a.n1 * SPB;
@@ -626,7 +626,7 @@ static cudaError_t launch_dq_b(const DequantArgs &a)
         const bool blocks4 = ((int64_t)a.S * a.D * BITS / 8) % 4 == 0;
         if (aligned && blocks4 && a.D % 8 == 0 && 32 % (a.D / 8) == 0 && a.D <= 256) {
             int per_sm = 1;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dequant_bhsd_span<T, BITS>, 256, 0) !=
+            if (kernel_occupancy(&per_sm, (const void *)dequant_bhsd_span<T, BITS>, 256, 0) !=
                     cudaSuccess ||
                 per_sm < 1)
                 per_sm = 1;

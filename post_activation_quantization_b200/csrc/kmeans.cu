@@ -711,7 +711,7 @@ cudaError_t launch_kmeans(const KmArgs &a)
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t sm = kmeans_smem_bytes(a.C, a.g);
-    e = cudaFuncSetAttribute(km_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    e = kernel_smem((const void *)km_fused, sm);
     if (e != cudaSuccess) return e;
     int C = a.C, g = a.g, iters = a.iters, bits = a.bits;
     KmWs wc = w;

@@ -356,7 +356,7 @@ static cudaError_t launch_kv_warp(const KvArgs &a)
     constexpr int DPT = 8;
     const KvTensors t{{a.k, a.v}, {a.kq, a.vq}, {a.ck, a.cv}, {a.sk, a.sv}, {a.zk, a.zv}};
     int per_sm = 1;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kv_quant_warp<T, BITS, DPT>, 256, 0) != cudaSuccess ||
+    if (kernel_occupancy(&per_sm, (const void *)kv_quant_warp<T, BITS, DPT>, 256, 0) != cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     const int64_t units = (int64_t)a.B * a.H * ((a.S + KV_ROWS_PER_UNIT - 1) / KV_ROWS_PER_UNIT);
@@ -384,10 +384,10 @@ static cudaError_t launch_kv_ring(const KvArgs &a)
     const int SPB = (int)(a.S / kv_ring_rows(a.D));
     auto kern = kv_quant_ring<T, BITS>;
     const size_t smem = kv_ring_smem<BITS>();
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, KVR_THREADS, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, KVR_THREADS, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t total = (int64_t)a.B * a.H * SPB * nt;

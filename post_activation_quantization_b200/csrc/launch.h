@@ -7,6 +7,12 @@
 
 namespace rptq {
 
+// Launch settings remembered per kernel and device (api.cu): the kernel's dynamic shared-memory
+// limit is raised once to the largest size asked for, and each (threads, bytes) occupancy
+// answer is looked up once, so a repeated launch makes no driver query.
+cudaError_t kernel_smem(const void *func, size_t bytes);
+cudaError_t kernel_occupancy(int *per_sm, const void *func, int threads, size_t smem);
+
 struct LnQuantArgs {
     const void *x;
     int dtype;

@@ -546,10 +546,10 @@ static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
     const bool db = a.C <= 9216 && db_smem <= (size_t)a.max_smem;
     const size_t smem = db ? db_smem : direct_smem_bytes(a.C, a.g);
     auto kern = db ? ln_quant_direct_kernel<T, BITS, CPT, MAXT, true> : ln_quant_direct_kernel<T, BITS, CPT, MAXT, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t quads = (a.T + 3) / 4;
@@ -565,10 +565,10 @@ static cudaError_t launch_fast_t(const LnQuantArgs &a, int NT, int NS, int alias
     const uint32_t rowbytes = (uint32_t)a.C * sizeof(T);
     const QuadSmem L = quad_smem_layout(NS, rowbytes, (alias ? 0 : (size_t)a.C * 4) + (size_t)a.C * 2 + 2 * 8 * 32 * 4);
     auto kern = ln_quant_fast_kernel<T, BITS, CPT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
+    cudaError_t e = kernel_smem((const void *)kern, L.total);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, NT, L.total);
+    e = kernel_occupancy(&per_sm, (const void *)kern, NT, L.total);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t quads = (a.T + 3) / 4;
@@ -673,10 +673,10 @@ static cudaError_t launch_simple_t(const LnQuantArgs &a)
 {
     const size_t smem = (size_t)a.C * 5;
     auto kern = ln_quant_simple_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, smem);
+    e = kernel_occupancy(&per_sm, (const void *)kern, 256, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t grid = std::min<int64_t>(a.T, (int64_t)per_sm * a.num_sms);
