@@ -103,3 +103,40 @@ def test_empty_problems_succeed_on_the_host(rlib):
     # ... but an empty problem with an invalid shape is still refused
     assert rlib.rptq_ln_reorder_quant(None, 2, 0, 60, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
                                       None, None, None) == -2
+
+
+def _prototypes():
+    """name -> list of C parameter types, parsed from the prototypes in include/rptq.h."""
+    src = open(os.path.join(ROOT, "include", "rptq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for m in re.finditer(r"(?:\bint\s+|\bsize_t\s+|\bconst char\s*\*\s*)(rptq_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(1)] = params
+    return out
+
+
+def _ctype_of(param: str):
+    t = re.sub(r"\s+", " ", param.rsplit(" ", 1)[0] if "*" not in param else param[: param.rindex("*") + 1])
+    if "*" in t or t.endswith("rptq_stream_t"):
+        return ctypes.c_void_p if "char" not in t else ctypes.c_char_p
+    return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "size_t": ctypes.c_size_t,
+            "float": ctypes.c_float}[t.replace("const ", "").strip()]
+
+
+def test_binding_argument_types_match_the_header():
+    """The Python binding's ctypes signature of every entry point has the header's parameter
+    count and, position by position, a ctypes type of the same size and kind."""
+    from post_activation_quantization_b200 import rptq
+    protos = _prototypes()
+    assert set(protos) == set(rptq.SIGNATURES)
+    for name, params in protos.items():
+        _, argtypes = rptq.SIGNATURES[name]
+        assert len(argtypes) == len(params), name
+        for i, (p, a) in enumerate(zip(params, argtypes)):
+            want = _ctype_of(p)
+            if want is ctypes.c_void_p:  # any pointer: void*, typed pointers, the stream handle
+                assert a is ctypes.c_void_p or hasattr(a, "_type_") and ctypes.sizeof(a) == ctypes.sizeof(ctypes.c_void_p), (name, i, p)
+            else:
+                assert a is want or ctypes.sizeof(a) == ctypes.sizeof(want) and a._type_ == want._type_, (name, i, p, a)
