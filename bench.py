@@ -62,6 +62,27 @@ def has_act(w: W.Workload) -> bool:
     return w.T > 0 and w.C > 0
 
 
+def stage_list(w: W.Workload):
+    """(name, algorithmic bytes per call, launches of this library's kernels per call) of the
+    step's stages, in order.  A calibration call without `accumulate` is an init launch + the
+    reduction; a KMeans call is two launches (the workspace clear and the cooperative kernel)."""
+    k, a = w.kv, has_act(w)
+    n = w.T * w.C
+    st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2)] if a else []
+    if k:
+        st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4)]
+    st += [("kmeans", 0, 2 * ((1 if a else 0) + (2 if k else 0)))]
+    if a:
+        st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+    if k:
+        st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
+    if a:
+        st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
+    if k:
+        st += [("dequant_kv", 2 * W.bytes_dequant(k.elems, k.dtype, k.bits), 2)]
+    return st
+
+
 # ------------------------------------------------------------------------------------------
 class Step:
     """Device buffers of one rank and the sequence of library calls that makes a step."""
@@ -118,25 +139,8 @@ class Step:
                     scale=torch.empty(g, dtype=torch.float32, device=d),
                     zero=torch.empty(g, dtype=torch.int32, device=d))
 
-    # (name, algorithmic bytes per call, launches of our kernels per call).  A calibration call
-    # without `accumulate` is an init launch + the reduction; a KMeans call is two launches (the
-    # workspace clear and the cooperative KMeans kernel).
     def stages(self):
-        w, k, a = self.w, self.kvw, self.act
-        n = w.T * w.C
-        st = [("calib_ln", W.bytes_calib(w.T_cal or w.T, w.C, w.dtype), 2)] if a else []
-        if k:
-            st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4)]
-        st += [("kmeans", 0, 2 * ((1 if a else 0) + (2 if k else 0)))]
-        if a:
-            st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
-        if k:
-            st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
-        if a:
-            st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
-        if k:
-            st += [("dequant_kv", 2 * W.bytes_dequant(k.elems, k.dtype, k.bits), 2)]
-        return st
+        return stage_list(self.w)
 
     def run(self, ev=None):
         """Enqueue one step on the current stream; ev: optional dict name -> (start, end).

@@ -39,3 +39,29 @@ def test_l2_statement_follows_input_sizes():
     assert "larger than L2" in bench.workload_config(W.WORKLOADS["kv-4096"])["l2"]
     assert "fit in the 126 MB L2" in bench.workload_config(W.WORKLOADS["tiny-768"])["l2"]
     assert "fit in the 126 MB L2" in bench.workload_config(W.WORKLOADS["opt6.7b-4096"])["l2"]
+
+
+def test_stage_accounting_per_workload():
+    """Stages, algorithmic bytes and launch counts of a step (the basis of `value` and of the
+    `gpu_launches` claim): by hand for the bench workload and the K/V-only one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from post_activation_quantization_b200 import workloads as W
+    st = bench.stage_list(W.WORKLOADS["opt175b-12288"])
+    assert [s[0] for s in st] == ["calib_ln", "kv_calib", "kmeans", "ln_reorder_quant", "kv_quant", "dequant_act",
+                                  "dequant_kv"]
+    b = dict((n, v) for n, v, _ in st)
+    T, C, Tc, kv = 32768, 12288, 262144, 8 * 96 * 2048 * 128
+    assert b["calib_ln"] == Tc * C * 2
+    assert b["kv_calib"] == 2 * kv * 2
+    assert b["ln_reorder_quant"] == T * C * 2 + T * C * 3 // 8
+    assert b["kv_quant"] == 2 * (kv * 2 + kv * 3 // 8)
+    assert b["dequant_act"] == T * C * 3 // 8 + T * C * 2
+    assert b["dequant_kv"] == 2 * (kv * 3 // 8 + kv * 2)
+    assert sum(l for _, _, l in st) == 17  # 2 + 4 + 6 + 1 + 1 + 1 + 2
+    st = bench.stage_list(W.WORKLOADS["kv-4096"])
+    assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "dequant_kv"]
+    assert sum(l for _, _, l in st) == 4 + 4 + 1 + 2
+    st = bench.stage_list(W.WORKLOADS["tiny-768"])
+    assert [s[0] for s in st] == ["calib_ln", "kmeans", "ln_reorder_quant", "dequant_act"]
+    assert sum(l for _, _, l in st) == 2 + 2 + 1 + 1
