@@ -97,3 +97,46 @@ def test_single_process_helpers_are_identity():
     assert a.tolist() == [1.0, -2.0] and b.tolist() == [0.5, -3.0]
     assert pdist.max_over_ranks(3.25) == 3.25
     assert pdist.sum_over_ranks(7.0) == 7.0
+
+
+def _rank_dies(rank: int, world: int, port: int, out_dir: str) -> None:
+    """Rank 1 leaves before the calibration exchange; rank 0 must get an error, not hang."""
+    import datetime
+    import time
+
+    import torch
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    from post_activation_quantization_b200 import dist as pdist
+    if rank == 1:
+        os._exit(0)  # the failing rank: gone between steps, nothing of it in flight
+    mx, mn = torch.zeros(16), torch.zeros(16)
+    t0 = time.time()
+    try:
+        pdist.allreduce_minmax(mx, mn)
+        res = "returned"
+    except Exception as e:  # the surviving rank learns of it from the collective
+        res = f"raised {type(e).__name__}"
+    with open(os.path.join(out_dir, "rank0.txt"), "w") as f:
+        f.write(f"{res} {time.time() - t0:.1f}")
+    os._exit(0)
+
+
+def test_a_lost_rank_ends_the_exchange_with_an_error(tmp_path):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    procs = [ctx.Process(target=_rank_dies, args=(r, WORLD, port, str(tmp_path))) for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+            pytest.fail("a rank hung after its peer left")
+    res = (tmp_path / "rank0.txt").read_text().split()
+    assert res[0] == "raised", res
+    assert float(res[-1]) < 60.0
