@@ -28,6 +28,11 @@
  *    R entry outside [0, C), a bounded wait that ran out) set a sticky device error word and
  *    the kernel carries on with safe values; read and clear it with rptq_device_error().
  *  - Calls that touch the same output buffers must not overlap on the GPU.
+ *  - Per-device facts are looked up at a device's first call and kept for the process: the SM
+ *    count, the shared-memory limit, the error word's address, each kernel's raised
+ *    shared-memory limit and its occupancy.  A process that resets a device (cudaDeviceReset)
+ *    must not call the library on that device afterwards.
+ *  - Empty problems (no rows, no positions) are valid: nothing is launched (see each call).
  *
  * Notation: T tokens, C channels, g clusters, b = bits (3 or 4), qmax = 2^b - 1.
  *
