@@ -8,29 +8,29 @@ A step is one pass of the whole path over one synthetic batch of the workload:
   4. K/V calibration statistics, KMeans for K and for V                   (rptq_kv_calib_minmax, rptq_kmeans)
   5. K/V cache quantization                                               (rptq_kv_quant)
   6. dequantization of the activation codes and of the K/V codes         (rptq_dequant)
-`value` is the whole-job algorithmic GB/s: the bytes every stage must move (see
-post_activation_quantization_b200/workloads.py) summed over ranks, divided by the slowest
-rank's device time for the K timed steps.  Inputs are larger than the 126 MB L2, so no flush
-is needed between steps.
+`value` is the metric's own kernel, measured inside those steps: the algorithmic GB/s of the
+fused LN-reorder-quant (read x, write the packed codes), its bytes summed over ranks and its
+device time the slowest rank's (the K/V quantizer for the K/V-only workload).  `step` gives
+the same for the whole step, `kernels` every stage (see
+post_activation_quantization_b200/workloads.py for the byte counts).  Inputs are larger than
+the 126 MB L2, so no flush is needed between steps.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl rptq|reference]
-Multi-GPU: launched by torchrun, one process per GPU, weak scaling (every rank its own batch);
-the calibration statistics are combined with one MAX/MIN all-reduce (NCCL).
+Multi-GPU: one process per GPU (run under torchrun, or `--gpus N` starts N ranks itself), weak
+scaling (every rank its own batch); the calibration statistics are combined with one MAX/MIN
+all-reduce (NCCL).
 """
 from __future__ import annotations
 
 import argparse
-import csv
 import dataclasses
 import datetime
 import hashlib
-import io
 import json
 import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -209,55 +209,70 @@ class Step:
 
 # ------------------------------------------------------------------------------------------
 class Clocks:
-    """nvidia-smi samples every 100 ms; only those taken inside the timed region are kept."""
-    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons sampled every `period_s` by a thread (NVML, in
+    process) while the timed region runs; only samples taken between start() and end() are kept.
+    Falls back to `nvidia-smi -lms 100` when NVML cannot be opened."""
+    REASONS = (("hw_slowdown", "HwSlowdown"), ("hw_thermal_slowdown", "HwThermalSlowdown"),
+               ("sw_thermal_slowdown", "SwThermalSlowdown"), ("sw_power_cap", "SwPowerCap"),
+               ("hw_power_brake", "HwPowerBrakeSlowdown"))
 
-    def __init__(self, gpu_index: int):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    def __init__(self, device, period_s: float = 0.002):
+        import threading
+        self.period, self.rows, self.on = period_s, [], False
         self.t0 = self.t1 = None
+        self.stop_ev = threading.Event()
+        self.how = "nvml"
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "100"],
-                                      stdout=self.f, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.p = None
+            import pynvml as nv
+            nv.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.nv = nv
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.bits = {name: getattr(nv, "nvmlClocksEventReason" + suffix, 0) for name, suffix in self.REASONS}
+            self.th = threading.Thread(target=self._loop, daemon=True)
+            self.th.start()
+        except Exception as e:  # noqa: BLE001 -- any NVML failure falls back to nvidia-smi
+            self.how, self.nv, self.err = "unavailable", None, str(e)
+
+    def _loop(self):
+        nv, h = self.nv, self.h
+        while not self.stop_ev.is_set():
+            if self.on:
+                t = time.time()
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                except Exception:  # noqa: BLE001
+                    mhz, rs, pw = None, 0, None
+                self.rows.append((t, mhz, rs, pw))
+            time.sleep(self.period)
 
     def start(self):
         self.t0 = time.time()
+        self.on = True
 
     def end(self):
+        self.on = False
         self.t1 = time.time()
 
     def stop(self) -> dict:
-        if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.p.terminate()
-        try:
-            self.p.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.p.kill()
-        self.f.flush()
-        self.f.seek(0)
-        rows = []
-        for r in csv.reader(io.StringIO(self.f.read())):
-            if len(r) < 10:
-                continue
-            try:
-                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
-            except ValueError:
-                continue
-            if self.t0 is not None and self.t0 <= ts <= self.t1:
-                rows.append([x.strip() for x in r[1:]])
-        os.unlink(self.f.name)
-        num = lambda v: v.replace(".", "", 1).isdigit()  # noqa: E731
-        sm = [float(r[1]) for r in rows if num(r[1])]
-        mx = [float(r[2]) for r in rows if num(r[2])]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v and "Not" not in v})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "samples": len(rows), "reasons": reasons}
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": ["clock sampling unavailable"],
+                    "how": self.how}
+        self.stop_ev.set()
+        self.th.join(timeout=2)
+        rows = [r for r in self.rows if r[1] is not None and self.t0 <= r[0] <= self.t1]
+        sm = [r[1] for r in rows]
+        reasons = sorted({n for r in rows for n, b in self.bits.items() if b and (r[2] & b)})
+        bins = {}
+        for v in sm:
+            bins[str(int(v))] = bins.get(str(int(v)), 0) + 1
+        pw = [r[3] for r in rows if r[3] is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "samples": len(rows), "period_ms": self.period * 1e3, "reasons": reasons,
+                "sm_mhz_bins": bins, "power_w_max": round(max(pw), 1) if pw else None, "how": "nvml in-process"}
 
 
 def _traffic(kernel: str):
@@ -278,12 +293,22 @@ def _traffic(kernel: str):
 
 
 # ------------------------------------------------------------------------------------------
+def headline_stage(w: W.Workload) -> str:
+    """The stage the metric names: the fused LN-reorder-quant, or the K/V quantizer for the
+    K/V-only workload."""
+    return "ln_reorder_quant" if has_act(w) else "kv_quant"
+
+
+def headline_tokens(w: W.Workload) -> int:
+    return w.T if has_act(w) else w.kv.B * w.kv.S
+
+
 def run_rptq(args):
     rank, ws, local = pdist.world()
     if ws > 1:
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", device_id=torch.device("cuda", local),
-                                             timeout=__import__("datetime").timedelta(seconds=120))
+                                             timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local if ws > 1 else 0)
     torch.cuda.set_device(dev)
     from post_activation_quantization_b200 import build, rptq
@@ -301,15 +326,11 @@ def run_rptq(args):
     torch.cuda.synchronize()
     tw = (time.perf_counter() - tw) / max(1, args.warmup)
     assert rptq.rptq_device_error() == 0, "device error word set during warm-up"
-    # untimed steps while the clock sampler starts (every rank runs the same number)
-    n_pre = int(pdist.max_over_ranks(min(2000, int(0.5 / max(tw, 1e-4)) + 1), dev))
 
     ev = {n: [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
           for n, _, _ in stages}
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = Clocks(dev.index) if rank == 0 else None
-    for _ in range(n_pre if args.clock_warmup else 0):  # the sampler starts while these run
-        step.run()
+    clk = Clocks(dev) if rank == 0 else None
     torch.cuda.synchronize()
     if ws > 1:
         torch.distributed.barrier()
@@ -326,11 +347,8 @@ def run_rptq(args):
     if ws > 1:
         torch.distributed.barrier()
     clocks = clk.stop() if clk else None
-    ms_rank = t0.elapsed_time(t1)
-    ms = pdist.max_over_ranks(ms_rank, dev)
-    step_bytes = sum(b * 1 for _, b, _ in stages)
-    total_bytes = pdist.sum_over_ranks(step_bytes * args.steps, dev)
-    value = total_bytes / (ms * 1e-3) / 1e9
+    ms = pdist.max_over_ranks(t0.elapsed_time(t1), dev)
+    step_bytes = sum(b for _, b, _ in stages)
     assert rptq.rptq_device_error() == 0, "device error word set during the timed steps"
 
     hbm, peak_kind = peaks()
@@ -338,20 +356,28 @@ def run_rptq(args):
     for n, b, launches in stages:
         per = [ev[n][i][0].elapsed_time(ev[n][i][1]) for i in range(args.steps)]
         mean_ms = sum(per) / len(per)
-        kern[n] = {"ms_per_call": round(mean_ms, 4), "bytes_per_call": b,
-                   "gpu_launches_per_call": launches}
+        kern[n] = {"ms_per_call": round(mean_ms, 4), "bytes_per_call": b, "gpu_launches_per_call": launches}
         if b:
             kern[n]["gbs"] = round(b / (mean_ms * 1e-3) / 1e9, 1)
             kern[n]["frac_of_measured_hbm"] = round(b / (mean_ms * 1e-3) / 1e9 / hbm, 4)
-    # tokens of the step: the activation batch, or the cache's B*S positions for the K/V-only workload
-    tok_stage, tokens = ("ln_reorder_quant", w.T) if step.act else ("kv_quant", w.kv.B * w.kv.S)
-    kern[tok_stage]["mtokens_per_s"] = round(tokens / (kern[tok_stage]["ms_per_call"] * 1e-3) / 1e6, 2)
+    # the headline: the metric's own kernel, its device time summed over the timed steps (the
+    # slowest rank's), its bytes summed over ranks
+    head = headline_stage(w)
+    head_bytes = kern[head]["bytes_per_call"]
+    head_ms = pdist.max_over_ranks(kern[head]["ms_per_call"] * args.steps, dev)
+    value = pdist.sum_over_ranks(head_bytes * args.steps, dev) / (head_ms * 1e-3) / 1e9
+    tokens = headline_tokens(w)
+    kern[head]["mtokens_per_s"] = round(tokens / (kern[head]["ms_per_call"] * 1e-3) / 1e6, 2)
     dom = max((n for n, b, _ in stages if b), key=lambda n: kern[n]["ms_per_call"])
-    dom_bytes = kern[dom]["bytes_per_call"]
-    ach = dom_bytes / (kern[dom]["ms_per_call"] * 1e-3) / 1e9
-    launches = sum(l for _, _, l in stages) * args.steps
 
-    e2e = run_e2e(step, args, dev, step_bytes, ws) if args.e2e_steps > 0 else None
+    def roof(n):
+        ach = kern[n]["bytes_per_call"] / (kern[n]["ms_per_call"] * 1e-3) / 1e9
+        return {"bound": "hbm", "kernel": n, "achieved": round(ach, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(ach / hbm, 4), "peak_kind": peak_kind, "traffic": _traffic(n),
+                "algorithmic_bytes_per_launch": kern[n]["bytes_per_call"]}
+
+    launches = sum(l for _, _, l in stages) * args.steps
+    e2e = run_e2e(step, args, dev, ws) if args.e2e_steps > 0 else None
 
     if rank == 0:
         cpu = cpu_baseline(w, args) if (ws == 1 and not args.no_cpu_baseline) else None
@@ -361,11 +387,16 @@ def run_rptq(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (seeded per-channel uniform ranges with outlier channels)",
             "config": workload_config(w),
-            "mtokens_per_s": round(tokens * ws * args.steps / (ms * 1e-3) / 1e6, 3),
+            "headline_kernel": head,
+            "mtokens_per_s": round(tokens * ws * args.steps / (head_ms * 1e-3) / 1e6, 3),
             "frac_of_measured_hbm": round(value / ws / hbm, 4),
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(ach / hbm, 4), "peak_kind": peak_kind,
-                         "traffic": _traffic(dom), "algorithmic_bytes_per_launch": dom_bytes},
+            "step": {"what": "every stage of the path once (calibration, KMeans, quantization, dequantization)",
+                     "ms": round(ms / args.steps, 4),
+                     "gbs": round(pdist.sum_over_ranks(step_bytes * args.steps, dev) / (ms * 1e-3) / 1e9, 1),
+                     "frac_of_measured_hbm": round(step_bytes * args.steps / (ms * 1e-3) / 1e9 / hbm, 4),
+                     "bytes": step_bytes},
+            "roofline": roof(head),
+            "roofline_step_dominant": roof(dom),
             "kernels": kern,
             "gpu_launches": launches,
             "clocks": clocks,
@@ -412,13 +443,25 @@ def workload_config(w):
     return c
 
 
-def run_e2e(step: Step, args, dev, step_bytes, ws):
-    """Same step through the public API with host inputs: each step copies its inputs from
-    pinned host memory and reads the codes (and calibration results) back, inside the timing."""
-    ins = ([step.xcal, step.x] if step.act else []) + ([step.k, step.v] if step.kvw else [])
-    outs = ([step.codes] if step.act else []) + ([step.kq, step.vq] if step.kvw else [])
-    outs += [step.km["R"], step.km["scale"], step.km["zero"]] if step.act else \
-        [step.kmk["labels"], step.kmk["scale"], step.kmk["zero"]]
+def run_e2e(step: Step, args, dev, ws):
+    """The headline call through the public API with host buffers: every step copies its input
+    from pinned host memory, runs the call, and reads its codes back, all inside the timing
+    (the calibration results of the timed steps are the call's tables)."""
+    r, w = step.r, step.w
+    if step.act:
+        ins, outs = [step.x], [step.codes]
+
+        def call():
+            r.rptq_ln_reorder_quant(step.x, step.gamma, step.beta, step.km["R"], step.km["col_cluster"],
+                                    step.km["scale"], step.km["zero"], w.bits, eps=w.eps, codes=step.codes)
+    else:
+        k = step.kvw
+        ins, outs = [step.k, step.v], [step.kq, step.vq]
+
+        def call():
+            r.rptq_kv_quant(step.k, step.v, step.kmk["labels"], step.kmk["scale"], step.kmk["zero"],
+                            step.kmv["labels"], step.kmv["scale"], step.kmv["zero"], k.bits,
+                            k_codes=step.kq, v_codes=step.vq)
     h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
     for h, t in zip(h_in, ins):
         h.copy_(t)
@@ -429,7 +472,7 @@ def run_e2e(step: Step, args, dev, step_bytes, ws):
     def one():
         for h, t in zip(h_in, ins):
             t.copy_(h, non_blocking=True)
-        step.run()
+        call()
         for h, t in zip(h_out, outs):
             h.copy_(t, non_blocking=True)
 
@@ -445,149 +488,134 @@ def run_e2e(step: Step, args, dev, step_bytes, ws):
     b.record()
     torch.cuda.synchronize()
     ms = pdist.max_over_ranks(a.elapsed_time(b), dev)
-    total = pdist.sum_over_ranks(step_bytes * args.e2e_steps, dev)
+    nbytes = stage_bytes(w, headline_stage(w))
+    total = pdist.sum_over_ranks(nbytes * args.e2e_steps, dev)
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": args.e2e_steps,
-            "ms_per_step": round(ms / args.e2e_steps, 3), "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo}
+            "what": f"{headline_stage(w)} through the C ABI with host buffers",
+            "ms_per_step": round(ms / args.e2e_steps, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+
+
+def stage_bytes(w: W.Workload, name: str) -> int:
+    return dict((n, b) for n, b, _ in stage_list(w))[name]
 
 
 # ------------------------------------------------------------------------------------------
-class OracleSample:
-    """The CPU oracle on a bounded sample of one step: `frac` of the tokens of every
-    token-parallel stage (inputs generated once, outside the timing), the three KMeans problems
-    in full.  `time_tokens()` times the token-parallel stages once; `time_kmeans()` the KMeans
-    problems (deterministic: the same inputs give the same work every time)."""
+def host_cpu() -> dict:
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
-    def __init__(self, w: W.Workload, frac: float):
-        import numpy as np
 
+class OracleHeadline:
+    """The CPU oracle on a bounded sample of the headline stage: the fused LN-reorder-quant of
+    `n` tokens of the workload's batch (the oracle's own calibration on a small calibration
+    sample gives its R, clusters, s and z), or the K/V quantization of `n` sequence positions of
+    the K and V caches (calibrated on that sample).  Inputs are generated once, outside the
+    timing; `run()` times one pass and returns the seconds."""
+
+    def __init__(self, w: W.Workload, n: int):
         import oracle
         oracle.build()
         self.o, self.w = oracle, w
         gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
-        self.act = has_act(w)
-        self.desc = "oracle (1 core)"
-        if self.act:
+        if has_act(w):
+            self.n = n = max(1, min(n, w.T))
             m = synthetic.channel_model(w.C, w.seed, w.outlier_frac, w.outlier_factor)
             self.gamma, self.beta = synthetic.ln_params(w.C, w.seed)
-            self.t_cal = max(4, int((w.T_cal or w.T) * frac))
-            self.t_x = max(4, int(w.T * frac))
-            self.xc = [oracle._f32(synthetic.activations(min(4096, self.t_cal - r0), m, w.seed + r0, dtype=w.dtype,
-                                                        calibration=True, device=gen_dev).cpu())
-                       for r0 in range(0, self.t_cal, 4096)]
-            self.x = oracle._f32(synthetic.activations(self.t_x, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
-            mx = mn = None
-            for xc in self.xc:
-                mx, mn = oracle.minmax_ln(xc, self.gamma, self.beta, w.eps, ch_max=mx, ch_min=mn)
-            self.mx, self.mn = mx, mn
-            self.desc += f" on {self.t_cal} calibration tokens and {self.t_x} tokens of the batch"
-        self.desc += ", full KMeans"
-        self.kv = []
-        if w.kv:
+            xc = oracle._f32(synthetic.activations(256, m, w.seed, dtype=w.dtype, calibration=True,
+                                                   device=gen_dev).cpu())
+            mx, mn = oracle.minmax_ln(xc, self.gamma, self.beta, w.eps)
+            self.cal = oracle.calibrate(mx, mn, w.g, w.iters, w.bits)
+            self.x = oracle._f32(synthetic.activations(n, m, w.seed, dtype=w.dtype, device=gen_dev).cpu())
+            self.nbytes = W.bytes_ln_quant(n, w.C, w.dtype, w.bits)
+            self.desc = (f"oracle fused LN-reorder-quant (LayerNorm, gather through R, quantize, pack) of {n} of "
+                         f"the {w.T} tokens, single-threaded")
+        else:
             k = w.kv
-            self.s_s = max(1, int(k.S * frac))
+            self.n = n = max(1, min(n, k.S))
+            self.kv = []
             for tag, which in ((1, "k"), (2, "v")):
                 mk = synthetic.channel_model(k.channels, w.seed, k.outlier_frac, k.outlier_factor, tag=tag)
-                kvf = oracle._f32(synthetic.kv_cache(k.B, k.H, self.s_s, k.D, mk, w.seed, which, k.dtype,
+                kvf = oracle._f32(synthetic.kv_cache(k.B, k.H, n, k.D, mk, w.seed, which, k.dtype,
                                                     device=gen_dev).cpu())
-                flat = np.ascontiguousarray(kvf.transpose(0, 2, 1, 3).reshape(-1, k.channels))
-                kmx, kmn = oracle.minmax(flat)
-                self.kv.append((kvf, flat, kmx, kmn))
-            self.desc += f", K and V with {self.s_s} of {k.S} sequence positions"
-        self.desc += "; stage times scaled to the full step"
-        self.cal = oracle.calibrate(self.mx, self.mn, w.g, w.iters, w.bits) if self.act else None
-        self.kcal = [oracle.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits) for _, _, kmx, kmn in self.kv]
+                flat = kvf.transpose(0, 2, 1, 3).reshape(-1, k.channels)
+                mx, mn = oracle.minmax(flat)
+                self.kv.append((kvf, oracle.calibrate(mx, mn, k.g, k.iters, k.bits)))
+            self.nbytes = W.bytes_kv_quant(k.B * k.H * n * k.D, k.dtype, k.bits)
+            self.desc = f"oracle K/V quantization of {n} of the {k.S} sequence positions of K and V, single-threaded"
 
-    def bytes_per_step(self) -> int:
-        w = self.w
-        n = 0
-        if self.act:
-            n += W.bytes_calib(w.T_cal or w.T, w.C, w.dtype) + W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits) \
-                + W.bytes_dequant(w.T * w.C, w.dtype, w.bits)
-        if w.kv:
-            k = w.kv
-            n += 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype) + \
-                W.bytes_kv_quant(k.elems, k.dtype, k.bits) + 2 * W.bytes_dequant(k.elems, k.dtype, k.bits)
-        return n
-
-    def time_kmeans(self) -> float:
+    def run(self) -> float:
         o, w = self.o, self.w
         t = time.perf_counter()
-        if self.act:
-            o.calibrate(self.mx, self.mn, w.g, w.iters, w.bits)
-        for _, _, kmx, kmn in self.kv:
-            o.calibrate(kmx, kmn, w.kv.g, w.kv.iters, w.kv.bits)
+        if has_act(w):
+            c = self.cal
+            o.ln_reorder_quant(self.x, self.gamma, self.beta, c["R"], c["col_cluster"], c["scale"], c["zero"],
+                               w.bits, eps=w.eps)
+        else:
+            for kvf, c in self.kv:
+                o.kv_quant(kvf, c["labels"], c["scale"], c["zero"], w.kv.bits)
         return time.perf_counter() - t
 
-    def time_tokens(self) -> float:
-        """Seconds the token-parallel stages of a full step take, scaled from the sample."""
-        o, w, cal = self.o, self.w, self.cal
-        secs = 0.0
-        if self.act:
-            t = time.perf_counter()
-            for xc in self.xc:
-                o.minmax_ln(xc, self.gamma, self.beta, w.eps)
-            secs += (time.perf_counter() - t) / (self.t_cal / (w.T_cal or w.T))
-            t = time.perf_counter()
-            packed, _, _ = o.ln_reorder_quant(self.x, self.gamma, self.beta, cal["R"], cal["col_cluster"],
-                                              cal["scale"], cal["zero"], w.bits, eps=w.eps)
-            q = o.unpack(packed, w.C, w.bits)
-            o.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])
-            secs += (time.perf_counter() - t) / (self.t_x / w.T)
-        if w.kv:
-            k = w.kv
-            t = time.perf_counter()
-            for (kvf, flat, _, _), kc in zip(self.kv, self.kcal):
-                o.minmax(flat)
-                pk = o.kv_quant(kvf, kc["labels"], kc["scale"], kc["zero"], k.bits)
-                o.kv_dequant(pk, k.D, kc["labels"], kc["scale"], kc["zero"], k.bits)
-            secs += (time.perf_counter() - t) / (self.s_s / k.S)
-        return secs
+
+def oracle_units_for(w: W.Workload, seconds: float) -> int:
+    """Sample size (tokens, or K/V positions) the oracle processes in about `seconds`."""
+    probe = OracleHeadline(w, 16)
+    probe.run()
+    per = probe.run() / probe.n
+    full = w.T if has_act(w) else w.kv.S
+    return int(max(1, min(full, seconds / max(per, 1e-9))))
 
 
 def cpu_baseline(w, args):
-    smp = OracleSample(w, args.cpu_frac)
-    secs = smp.time_tokens() + smp.time_kmeans()
-    return {"value": round(smp.bytes_per_step() / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": smp.desc, "seconds_per_step_extrapolated": round(secs, 2)}
+    smp = OracleHeadline(w, oracle_units_for(w, args.cpu_seconds))
+    secs = smp.run()
+    return {"value": round(smp.nbytes / secs / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": smp.desc, "seconds": round(secs, 2), **host_cpu()}
 
 
 def run_reference(args):
-    """The reference arm: the oracle on the host, one bounded sample per step.  The sample size
-    keeps the whole --steps K --warmup W run near `--ref-budget-s` seconds; the three KMeans
-    problems (deterministic, the same work each step) are timed once and counted in every step."""
+    """The reference arm: the oracle on the host cores, each step one bounded sample of the
+    headline stage, sized so the whole --steps K --warmup W run takes about --ref-budget-s."""
     rank, ws, _ = pdist.world()
     if rank != 0:
         return  # under torchrun only rank 0 runs the CPU reference
     w = W.WORKLOADS[args.workload]
-    probe = OracleSample(w, 1 / 256)
-    t0 = time.perf_counter()
-    probe.time_tokens()
-    per_frac = (time.perf_counter() - t0) * 256  # seconds of token work per full-step fraction 1
     per_step = args.ref_budget_s / max(1, args.steps + args.warmup)
-    frac = min(args.ref_frac, max(1 / 4096, per_step / max(per_frac, 1e-9)))
-    smp = OracleSample(w, frac)
-    km_secs = smp.time_kmeans()
+    smp = OracleHeadline(w, oracle_units_for(w, per_step))
     for _ in range(args.warmup):
-        smp.time_tokens()
-    vals = []
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        vals.append(smp.bytes_per_step() / (smp.time_tokens() + km_secs) / 1e9)
-    wall = time.perf_counter() - t0
-    value = statistics.mean(vals)
-    nbytes = smp.bytes_per_step()
+        smp.run()
+    secs = [smp.run() for _ in range(args.steps)]
+    total = sum(secs)
+    value = smp.nbytes * args.steps / total / 1e9
     line = {"metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(nbytes / (value * 1e9) * 1e3, 1), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w), "impl": "reference",
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(w), "impl": "reference",
+            "headline_kernel": headline_stage(w),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                             "sample": smp.desc + f" (token fraction {frac:.5f}; KMeans timed once)",
-                             "wall_s": round(wall, 1)},
+                             "sample": smp.desc + " per step", **host_cpu()},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def relaunch(n: int) -> int:
+    """Run this command again as n ranks under torchrun (one process per GPU) and return its
+    exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -597,19 +625,30 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["rptq", "reference"], default="rptq")
     ap.add_argument("--workload", choices=W.ORDER, default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=2)
-    ap.add_argument("--cpu-frac", type=float, default=1 / 2,
-                    help="fraction of the tokens the CPU oracle processes for its baseline")
-    ap.add_argument("--ref-frac", type=float, default=1 / 32,
-                    help="largest fraction of the tokens per step of the --impl reference arm")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="about how long the CPU oracle's baseline sample runs")
     ap.add_argument("--ref-budget-s", type=float, default=120.0,
                     help="target seconds of host work for the whole --impl reference run")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-clock-warmup", dest="clock_warmup", action="store_false",
-                    help="skip the untimed steps that let the clock sampler start (profiling runs)")
     ap.add_argument("--token-scale", type=float, default=1.0,
                     help="shrink the token counts (a small case for ncu captures; not a bench config)")
+    ap.add_argument("--no-clock-warmup", action="store_true",
+                    help="no effect (the in-process clock sampler needs no warm-up steps)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="print this rank's place in the launch and exit (checks the multi-process plumbing)")
     args = ap.parse_args()
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        sys.exit(relaunch(args.gpus))  # one process per GPU
+    rank, ws, local = pdist.world()
+    if ws != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but the launcher started {ws} ranks", file=sys.stderr)
+        sys.exit(2)
+    if args.dry_run:
+        print(json.dumps({"rank": rank, "world_size": ws, "local_rank": local, "impl": args.impl}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -329,7 +329,8 @@ __global__ void __launch_bounds__(512, 1)
     const QuadSmem L = quad_smem_layout(NS, rowbytes, 2 * 8 * 32 * 4);
     float *red = reinterpret_cast<float *>(smem + L.extra_off);
     float *red2 = red + 8 * 32;
-    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
+    __shared__ int s_abort;
+    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err, &s_abort};
     pipe.start();
     __syncthreads();
 
@@ -348,6 +349,10 @@ __global__ void __launch_bounds__(512, 1)
         pipe.load(nrows, xr);
         float rstd[4], nmr[4], sub[4];
         const bool offs = quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, sub);
+        if (pipe.aborted()) {  // a row never arrived: stop here (the error word is set)
+            pipe.drain(lq);
+            return;
+        }
         if (nrows == 4 && !offs) {  // normalised values of tokens (0, 1) and (2, 3) two lanes at a time
             const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
             const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);

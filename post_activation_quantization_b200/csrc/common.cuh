@@ -57,6 +57,36 @@ template <> struct Elem<__half> {
     }
 };
 
+// Element e of a 16-byte chunk plus nsub, in fp32 with one rounding.  16-bit inputs use the
+// sm_100 mixed-precision add, which widens and adds in one instruction; nsub = -0.0 gives the
+// element exactly, and x - m for x near m is exact (Sterbenz), so the same code serves rows with
+// and without a subtracted offset.
+template <typename T> __device__ __forceinline__ float elem_plus(const uint4 &v, int e, float nsub);
+template <> __device__ __forceinline__ float elem_plus<__nv_bfloat16>(const uint4 &v, int e, float nsub)
+{
+    const uint32_t w = (&v.x)[e >> 1];
+    float r;
+    if (e & 1)
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n add.rn.f32.bf16 %0, hi, %2;\n}" : "=f"(r) : "r"(w), "f"(nsub));
+    else
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n add.rn.f32.bf16 %0, lo, %2;\n}" : "=f"(r) : "r"(w), "f"(nsub));
+    return r;
+}
+template <> __device__ __forceinline__ float elem_plus<__half>(const uint4 &v, int e, float nsub)
+{
+    const uint32_t w = (&v.x)[e >> 1];
+    float r;
+    if (e & 1)
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n add.rn.f32.f16 %0, hi, %2;\n}" : "=f"(r) : "r"(w), "f"(nsub));
+    else
+        asm("{\n .reg .b16 lo, hi;\n mov.b32 {lo, hi}, %1;\n add.rn.f32.f16 %0, lo, %2;\n}" : "=f"(r) : "r"(w), "f"(nsub));
+    return r;
+}
+template <> __device__ __forceinline__ float elem_plus<float>(const uint4 &v, int e, float nsub)
+{
+    return __uint_as_float((&v.x)[e]) + nsub;
+}
+
 // Moments of a 16-byte chunk: s += sum(x), q += sum(x^2).  16-bit inputs use the sm_100
 // mixed-precision add/fma (16-bit sources, fp32 accumulator, one rounding; identical to widening
 // first), so no separate conversion instruction is spent on them.
@@ -271,10 +301,12 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
 
 // ---- CTA-wide sum of 8 floats per thread, every thread receives the 8 totals -----------
 // `red` is shared scratch of 8 * (blockDim.x / 32) floats.  Deterministic (fixed order).
-// Contains one __syncthreads().
-__device__ __forceinline__ void cta_sum8(float (&v)[8], float *red)
+// Contains one __syncthreads().  nwarps_: the CTA's warp count when the caller knows it at
+// compile time (0: read it from blockDim).
+__device__ __forceinline__ void cta_sum8(float (&v)[8], float *red, int nwarps_ = 0)
 {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarps = nwarps_ ? nwarps_ : (int)(blockDim.x >> 5);
     const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {

@@ -173,23 +173,25 @@ __device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int3
 }
 
 // Codes of the quad's four tokens for every channel of the thread -> one word per channel at
-// its stored position in the code buffer.  SUB: subtract sub[r] before the normalising fma (the
-// quad holds a row with a large offset or no spread; see quad_stats).
-template <typename T, int BITS, int CPT, bool ABS, bool SUB>
+// its stored position in the code buffer.  The normalised value of x is fmaf(x - sub[r], rstd[r],
+// nmr[r]) (sub = 0 except for rows with a large offset, see quad_stats); x - sub is formed by the
+// widening mixed-precision add, so both kinds of row share this code and cost no extra
+// instruction.  NT_: the CTA's thread count when known at compile time (0: blockDim.x).
+template <typename T, int BITS, int CPT, bool ABS>
 __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const float (&rstd)[4], const float (&nmr)[4],
                                               const float (&sub)[4],
                                               const float (&pA)[CPT][Elem<T>::VEC],
                                               const float (&pB)[CPT][Elem<T>::VEC], const void *postab,
-                                              uint8_t *codebuf, int NCH, uint32_t boff = 0)
+                                              uint8_t *codebuf, int NCH, uint32_t boff = 0, int NT_ = 0)
 {
     // ABS: postab holds 32-bit shared-memory addresses (stored directly, no extraction);
     // otherwise 16-bit offsets into codebuf, two per word
     constexpr int VEC = Elem<T>::VEC;
     constexpr float QMAX = (float)((1 << BITS) - 1);
-    const int tid = threadIdx.x, NT = blockDim.x;
+    const int tid = threadIdx.x, NT = NT_ ? NT_ : (int)blockDim.x;
     const f32x2 rs01 = mk2(rstd[0], rstd[1]), rs23 = mk2(rstd[2], rstd[3]);
     const f32x2 nm01 = mk2(nmr[0], nmr[1]), nm23 = mk2(nmr[2], nmr[3]);
-    const f32x2 ms01 = mk2(-sub[0], -sub[1]), ms23 = mk2(-sub[2], -sub[3]);
+    const float ms[4] = {-sub[0], -sub[1], -sub[2], -sub[3]};
     const f32x2 qm2 = mk2(QMAX, QMAX), mg2 = mk2(MAGIC_RINT, MAGIC_RINT);
 #pragma unroll
     for (int k = 0; k < CPT; ++k) {
@@ -213,12 +215,8 @@ __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const f
 #pragma unroll
         for (int e = 0; e < VEC; ++e) {
             // normalised values of channel e for tokens (0,1) and (2,3), two lanes at a time
-            f32x2 x01 = mk2(Elem<T>::get(xr[0][k], e), Elem<T>::get(xr[1][k], e));
-            f32x2 x23 = mk2(Elem<T>::get(xr[2][k], e), Elem<T>::get(xr[3][k], e));
-            if constexpr (SUB) {
-                x01 = add2(x01, ms01);
-                x23 = add2(x23, ms23);
-            }
+            const f32x2 x01 = mk2(elem_plus<T>(xr[0][k], e, ms[0]), elem_plus<T>(xr[1][k], e, ms[1]));
+            const f32x2 x23 = mk2(elem_plus<T>(xr[2][k], e, ms[2]), elem_plus<T>(xr[3][k], e, ms[3]));
             const f32x2 t01 = fma2(x01, rs01, nm01);
             const f32x2 t23 = fma2(x23, rs23, nm23);
             const float A = pA[k][e], Bc = pB[k][e];
@@ -242,9 +240,10 @@ __device__ __forceinline__ void quant_scatter(const uint4 (&xr)[4][CPT], const f
 // rows 4*gq .. 4*gq + nrows - 1.
 template <int BITS>
 __device__ __forceinline__ void pack_store(const uint8_t *codebuf, uint8_t *codes, int64_t gq, int64_t pitch, int nrows,
-                                           int NU)
+                                           int NU, int NT_ = 0)
 {
-    for (int u = threadIdx.x; u < NU; u += blockDim.x) {
+    const int NT = NT_ ? NT_ : (int)blockDim.x;
+    for (int u = threadIdx.x; u < NU; u += NT) {
         uint32_t o[4][4];  // [group m of 8 positions][token r]
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
@@ -300,7 +299,8 @@ __global__ void __launch_bounds__(512, 1)
     float *red = reinterpret_cast<float *>(postab + C);                      // 8*32 floats
     float *red2 = red + 8 * 32;
 
-    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err};
+    __shared__ int s_abort;
+    QuadRows<T, CPT> pipe{x, T_, C, NCH, NS, rowbytes, smem, smem_u32(smem + L.bar_off), err, &s_abort};
     pipe.start();
     float pA[CPT][VEC], pB[CPT][VEC];
     quant_tables<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, 0u, pA, pB, err);
@@ -313,12 +313,13 @@ __global__ void __launch_bounds__(512, 1)
         uint4 xr[4][CPT];
         pipe.load(nrows, xr);
         float rstd[4], nmr[4], sub[4];
-        const bool offs = quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, sub, !alias);
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, pipe, lq, rstd, nmr, sub, !alias);
+        if (pipe.aborted()) {  // a row never arrived (the error word is set): stop, no refill
+            pipe.drain(lq);
+            return;
+        }
         if (alias) codebuf = smem + (size_t)pipe.slot * rowbytes;  // this quad's slots
-        if (offs)
-            quant_scatter<T, BITS, CPT, false, true>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
-        else
-            quant_scatter<T, BITS, CPT, false, false>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
+        quant_scatter<T, BITS, CPT, false>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH);
         __syncthreads();
         pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU);
         if (alias) {  // the quad's slots held its codes until now
@@ -340,10 +341,10 @@ struct NoRefill {
 
 template <typename T, int CPT>
 __device__ __forceinline__ void load_quad_direct(const T *x, int64_t T_, int C, int64_t gq, bool exact,
-                                                 uint4 (&xr)[4][CPT])
+                                                 uint4 (&xr)[4][CPT], int NT_ = 0)
 {
     constexpr int VEC = Elem<T>::VEC;
-    const int tid = threadIdx.x, NT = blockDim.x, NCH = C / VEC;
+    const int tid = threadIdx.x, NT = NT_ ? NT_ : (int)blockDim.x, NCH = C / VEC;
     const T *src = x + 4 * gq * (int64_t)C + tid * VEC;
     if (exact && 4 * gq + 4 <= T_) {  // a full quad and every chunk inside the row: no predicates
 #pragma unroll
@@ -386,15 +387,21 @@ __host__ __device__ inline size_t direct_db_off(int C, int g) { return (direct_s
 // remains: stats(q) [barrier] -> scatter(q) into buffer q%2 -> loads of q+1 -> pack(q-1) from
 // buffer (q-1)%2.  The scatter of q+1 rewrites buffer (q-1)%2 only after the barrier of q+1,
 // which every thread reaches after its pack(q-1).
-template <typename T, int BITS, int CPT, int MAXT, bool DB>
+// CC: the channel count fixed at compile time (0: the runtime argument).  With it the thread
+// count (CC / VEC / CPT, the exact split) and every loop bound, row pitch and load offset are
+// constants, which removes most of the per-quad address, bound and branch instructions; the
+// launcher instantiates it for the common hidden sizes.
+template <typename T, int BITS, int CPT, int MAXT, bool DB, int CC = 0>
 __global__ void __launch_bounds__(MAXT, 1)
-    ln_quant_direct_kernel(const T *__restrict__ x, int64_t T_, int C, const float *__restrict__ gamma,
+    ln_quant_direct_kernel(const T *__restrict__ x, int64_t T_, int C_, const float *__restrict__ gamma,
                            const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
                            const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
                            const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int *err)
 {
     constexpr int VEC = Elem<T>::VEC;
     extern __shared__ __align__(128) uint8_t smem[];
+    const int C = CC ? CC : C_;
+    const int NT = CC ? CC / VEC / CPT : (int)blockDim.x;
     const int NCH = C / VEC;
     const uint32_t rowbytes = (uint32_t)C * sizeof(T);
     uint8_t *codebuf = smem;                                                    // 4*C bytes
@@ -404,14 +411,14 @@ __global__ void __launch_bounds__(MAXT, 1)
     double *ctl = reinterpret_cast<double *>(red2 + 8 * 32);                   // 2*g doubles
     uint16_t *ctab = reinterpret_cast<uint16_t *>(ctl + 2 * g);                // C u16
     const int64_t G = gridDim.x;
-    const bool exact = NCH == CPT * (int)blockDim.x;  // the chunks split evenly over the threads
+    const bool exact = NCH == CPT * NT;  // the chunks split evenly over the threads
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x);
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x + G);
     float pA[CPT][VEC], pB[CPT][VEC];
     quant_tables_direct<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, ctab, ctl,
                                       smem_u32(codebuf), pA, pB, err);
     uint4 xr[4][CPT];
-    load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr);  // the L2 prefetch above is in flight
+    load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr, NT);  // the L2 prefetch above is in flight
 
     const int64_t pitch = (int64_t)C * BITS / 8;
     const int NU = C >> 5;
@@ -424,28 +431,26 @@ __global__ void __launch_bounds__(MAXT, 1)
         const int nrows = (int)(T_ - 4 * gq < 4 ? T_ - 4 * gq : 4);
         float rstd[4], nmr[4], sub[4];
         const uint32_t off = (DB && (it & 1)) ? boff : 0u;
-        if (quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, none, 0, rstd, nmr, sub, false))
-            quant_scatter<T, BITS, CPT, true, true>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH, off);
-        else
-            quant_scatter<T, BITS, CPT, true, false>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH, off);
+        quad_stats<T, CPT>(xr, C, NCH, eps, red, red2, none, 0, rstd, nmr, sub, false, NT);
+        quant_scatter<T, BITS, CPT, true>(xr, rstd, nmr, sub, pA, pB, postab, codebuf, NCH, off, NT);
         // the rows are dead: next quad's loads fly during the pack, and one more quad to L2
-        load_quad_direct<T, CPT>(x, T_, C, gq + G, exact, xr);
+        load_quad_direct<T, CPT>(x, T_, C, gq + G, exact, xr, NT);
         prefetch_quad_l2(x, T_, rowbytes, gq + 2 * G);
         if constexpr (DB) {
-            if (pgq >= 0) pack_store<BITS>((it & 1) ? codebuf : codebuf1, codes, pgq, pitch, prows, NU);
+            if (pgq >= 0) pack_store<BITS>((it & 1) ? codebuf : codebuf1, codes, pgq, pitch, prows, NU, NT);
             pgq = gq;
             prows = nrows;
             ++it;
         } else {
             __syncthreads();
-            pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU);
+            pack_store<BITS>(codebuf, codes, gq, pitch, nrows, NU, NT);
             // the next quad's scatter overwrites the code buffer only after the barrier inside
             // its LayerNorm statistics, which every thread reaches after this pack
         }
     }
     if (DB && pgq >= 0) {  // the last quad (number it - 1) and its buffer
         __syncthreads();
-        pack_store<BITS>((it & 1) ? codebuf : codebuf1, codes, pgq, pitch, prows, NU);
+        pack_store<BITS>((it & 1) ? codebuf : codebuf1, codes, pgq, pitch, prows, NU, NT);
     }
 }
 
@@ -539,13 +544,27 @@ __global__ void __launch_bounds__(256)
 template <typename T, int BITS, int CPT, int MAXT>
 static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
 {
-    // two code buffers (one barrier per quad) when they fit, for rows up to 9216 channels:
-    // measured on bf16 A3, 59% -> 62% of the HBM copy rate at C = 9216 but 72.5% -> 70.4% at
-    // C = 12288
+    // two code buffers (one barrier per quad) whenever they fit: with the thread split fixed at
+    // compile time, bf16 A3 measured 0.685 -> 0.706 of the HBM copy rate at C = 12288 (one
+    // buffer was faster there with a runtime split) and 0.59 -> 0.62 at C = 9216
     const size_t db_smem = direct_db_off(a.C, a.g) + (size_t)4 * a.C;
-    const bool db = a.C <= 9216 && db_smem <= (size_t)a.max_smem;
+    const bool db = db_smem <= (size_t)a.max_smem;
     const size_t smem = db ? db_smem : direct_smem_bytes(a.C, a.g);
     auto kern = db ? ln_quant_direct_kernel<T, BITS, CPT, MAXT, true> : ln_quant_direct_kernel<T, BITS, CPT, MAXT, false>;
+    // the hidden sizes of OPT-6.7B, -66B and -175B with 16-bit inputs, compiled for their exact
+    // thread split (the plan below picks 512 x 1, 384 x 3 and 384 x 4 chunks)
+    if constexpr (sizeof(T) == 2 && CPT == 1 && MAXT == 512) {
+        if (a.C == 4096 && NT == 4096 / 8)
+            kern = db ? ln_quant_direct_kernel<T, BITS, 1, 512, true, 4096> : ln_quant_direct_kernel<T, BITS, 1, 512, false, 4096>;
+    }
+    if constexpr (sizeof(T) == 2 && CPT == 3 && MAXT == 384) {
+        if (a.C == 9216 && NT == 9216 / 8 / 3)
+            kern = db ? ln_quant_direct_kernel<T, BITS, 3, 384, true, 9216> : ln_quant_direct_kernel<T, BITS, 3, 384, false, 9216>;
+    }
+    if constexpr (sizeof(T) == 2 && CPT == 4 && MAXT == 384) {
+        if (a.C == 12288 && NT == 12288 / 8 / 4)
+            kern = db ? ln_quant_direct_kernel<T, BITS, 4, 384, true, 12288> : ln_quant_direct_kernel<T, BITS, 4, 384, false, 12288>;
+    }
     cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

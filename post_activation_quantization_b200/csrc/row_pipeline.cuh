@@ -29,6 +29,7 @@ struct QuadRows {
     uint8_t *ring;      // NS * rowbytes, 128-byte aligned
     uint32_t bar0;      // shared address of NS consecutive 8-byte mbarriers
     int *err;
+    int *abort;         // shared flag: a wait of this CTA ran out (set in load, read after a barrier)
     // ring position of the current quad's first row, kept incrementally (no divisions):
     // slot = (4 lq) mod NS and phase parity = ((4 lq) / NS) mod 2
     uint32_t slot = 0, phase = 0;
@@ -52,6 +53,7 @@ struct QuadRows {
     __device__ __forceinline__ void start() const
     {
         if (threadIdx.x == 0) {
+            *abort = 0;
             for (int s = 0; s < NS; ++s) mbar_init(bar0 + 8u * s, 1);
             fence_mbar_init();
             for (int s = 0; s < NS; ++s) issue(s, (uint32_t)s);
@@ -75,7 +77,7 @@ struct QuadRows {
         for (int r = 0; r < 4; ++r) {
             uint32_t s, ph;
             where(r, s, ph);
-            if (r < nrows) mbar_wait_bounded(bar0 + 8u * s, ph, err);
+            if (r < nrows && !mbar_wait_bounded(bar0 + 8u * s, ph, err)) *abort = 1;
             const uint4 *src = reinterpret_cast<const uint4 *>(ring + (size_t)s * rowbytes);
 #pragma unroll
             for (int k = 0; k < CPT; ++k) {
@@ -84,11 +86,28 @@ struct QuadRows {
             }
         }
     }
+    // Whether a wait of the current quad ran out: the same answer in every thread once a barrier
+    // separates it from load().  The caller then stops (after drain()) instead of refilling.
+    __device__ __forceinline__ bool aborted() const { return *(volatile int *)abort != 0; }
+    // thread 0 after an abort: wait (bounded) for the copies still in flight into the ring, the
+    // rows of the current quad and the NS - 4 rows after them, so none lands after the CTA exits
+    __device__ __forceinline__ void drain(int64_t lq) const
+    {
+        if (threadIdx.x != 0) return;
+        uint32_t s = slot, ph = phase;
+        for (int i = 0; i < NS; ++i) {
+            if (row_of(4 * lq + i) < T_) mbar_wait_bounded(bar0 + 8u * s, ph, err);
+            if (++s == (uint32_t)NS) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+    }
     // thread 0 after the quad's last read of its slots r0 .. r1-1: refill them with the rows NS
-    // ahead
+    // ahead (nothing once the CTA has aborted)
     __device__ __forceinline__ void refill(int64_t lq, int r0 = 0, int r1 = 4) const
     {
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0 && !aborted()) {
             fence_proxy_async_smem();
             for (int r = r0; r < r1; ++r) {
                 uint32_t s, ph;
@@ -119,14 +138,15 @@ struct QuadRows {
 // is exact for x near the mean, so the offset never meets a rounding.
 // `red`, `red2`: 8*(NT/32) floats each.  With refill_now, calls refill() between its first
 // barrier and any later one (the caller refills later when it still uses the quad's ring slots).
+// NT_: the CTA's thread count when the caller knows it at compile time (0: blockDim.x).
 template <typename T, int CPT, typename Pipe>
 __device__ __forceinline__ bool quad_stats(const uint4 (&xr)[4][CPT], int C, int NCH, float eps,
                                            float *red, float *red2, const Pipe &pipe, int64_t lq,
                                            float (&rstd)[4], float (&nmr)[4], float (&sub)[4],
-                                           bool refill_now = true)
+                                           bool refill_now = true, int NT_ = 0)
 {
     constexpr int VEC = Elem<T>::VEC;
-    const int tid = threadIdx.x, NT = blockDim.x;
+    const int tid = threadIdx.x, NT = NT_ ? NT_ : (int)blockDim.x;
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;
@@ -135,7 +155,7 @@ __device__ __forceinline__ bool quad_stats(const uint4 (&xr)[4][CPT], int C, int
     for (int k = 0; k < CPT; ++k)
 #pragma unroll
         for (int r = 0; r < 4; ++r) chunk_moments<T>(xr[r][k], v[r], v[4 + r]);
-    cta_sum8(v, red);  // every thread is past its reads of this quad's ring slots
+    cta_sum8(v, red, NT >> 5);  // every thread is past its reads of this quad's ring slots
     if (refill_now) pipe.refill(lq);
     const float invC = 1.0f / (float)C;
     float mean[4], var[4];
@@ -169,7 +189,7 @@ __device__ __forceinline__ bool quad_stats(const uint4 (&xr)[4][CPT], int C, int
                     }
             }
         }
-        cta_sum8(w, red2);
+        cta_sum8(w, red2, NT >> 5);
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             if (!ill[r]) continue;

@@ -123,7 +123,12 @@ LN_CASES = [  # (dtype, T, C, g, bits)
     ("f32", 512, 768, 8, 4), ("f32", 7, 768, 8, 3), ("f16", 203, 4096, 32, 4),
     ("bf16", 130, 9216, 64, 3), ("bf16", 65, 12288, 64, 3), ("bf16", 1, 12288, 64, 4),
     ("f16", 6, 256, 5, 3), ("bf16", 33, 2048, 16, 4), ("f32", 9, 4096, 16, 3),
-    ("bf16", 1203, 12288, 64, 3), ("f16", 97, 16384, 512, 4), ("bf16", 70, 8192, 300, 3)]
+    ("bf16", 1203, 12288, 64, 3), ("f16", 97, 16384, 512, 4), ("bf16", 70, 8192, 300, 3),
+    # several quads of four rows per CTA (148 CTAs): the double code buffer in turn, the kernels
+    # compiled for fixed channel counts (4096, 9216, 12288), the generic 4-chunk split (8192)
+    # and ragged last quads
+    ("bf16", 2001, 9216, 64, 3), ("f16", 1779, 9216, 64, 4), ("bf16", 1802, 8192, 300, 3),
+    ("f16", 2501, 4096, 32, 4), ("bf16", 1777, 12288, 64, 4), ("bf16", 3000, 5120, 40, 3)]
 
 
 @pytest.mark.parametrize("dtype,T,C,g,bits", LN_CASES)
