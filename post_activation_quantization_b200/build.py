@@ -28,7 +28,7 @@ def nvcc() -> str:
 
 def _deps(src: str) -> list[str]:
     return [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
-        os.path.join(ROOT, "include", "rptq.h"), src]
+        os.path.join(ROOT, "include", "rptq.h"), os.path.join(ROOT, "include", "rptq_testing.h"), src]
 
 
 def _stale(out: str, deps: list[str]) -> bool:

@@ -38,6 +38,7 @@
 //   Every wait is bounded (2 s, then the device error word and no further waiting).
 #include <algorithm>
 
+#include "../../include/rptq_testing.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -237,10 +238,16 @@ __device__ __forceinline__ void ll_get1(const uint64_t *p, uint64_t &w)
 }
 __device__ __forceinline__ bool ll_ok(uint64_t w, uint32_t flag) { return (uint32_t)(w >> 32) == flag; }
 
+// Limit of every exchange wait and grid barrier of the KMeans kernel (2 s), and the CTA that
+// leaves out its first Lloyd record (-1: none).  Both change only through the testing hook
+// rptq_testing_kmeans_wait (include/rptq_testing.h), so that a test can make a wait run out.
+static __device__ unsigned long long g_km_wait_ns = 2000000000ull;
+static __device__ int g_km_withhold = -1;
+
 // Read cells p[b * stride], b < n (n <= N), until both words of each carry `flag`: all reads
 // are issued together and only the cells still stale are read again, all together.  Bounded by
-// 2 s, after which the device error word is set and `abort` makes every later wait of the CTA
-// give up at once.
+// the wait limit, after which the device error word is set and `abort` makes every later wait
+// of the CTA give up at once.
 template <int N>
 __device__ __forceinline__ void ll_gather2(const uint4 *p, size_t stride, int n, uint32_t flag, uint64_t (&v0)[N],
                                            uint64_t (&v1)[N], int *err, volatile int *abort)
@@ -262,7 +269,7 @@ __device__ __forceinline__ void ll_gather2(const uint4 *p, size_t stride, int n,
 #pragma unroll
         for (int b = 0; b < N; ++b)
             if (((pend >> b) & 1u) && ll_ok(v0[b], flag) && ll_ok(v1[b], flag)) pend &= ~(1u << b);
-        if (pend && global_ns() - t0 > 2000000000ull) {
+        if (pend && global_ns() - t0 > g_km_wait_ns) {
             raise_error(err, RPTQ_DEVERR_TIMEOUT);
             *abort = 1;
         }
@@ -289,7 +296,7 @@ __device__ __forceinline__ void ll_gather1(const uint64_t *p, size_t stride, int
 #pragma unroll
         for (int b = 0; b < N; ++b)
             if (((pend >> b) & 1u) && ll_ok(v[b], flag)) pend &= ~(1u << b);
-        if (pend && global_ns() - t0 > 2000000000ull) {
+        if (pend && global_ns() - t0 > g_km_wait_ns) {
             raise_error(err, RPTQ_DEVERR_TIMEOUT);
             *abort = 1;
         }
@@ -297,11 +304,13 @@ __device__ __forceinline__ void ll_gather1(const uint64_t *p, size_t stride, int
 }
 
 // Grid-wide barrier for a cooperative launch: arrival counter + generation word.  The wait is
-// bounded by wall time; on expiry the device error word is set and the CTA goes on.
-__device__ __forceinline__ void km_grid_barrier(unsigned *bar, int *err)
+// bounded by the wait limit; on expiry the device error word and `abort` are set, and a CTA
+// that has aborted no longer waits at all (its later exchange waits give up at once too), so
+// one straggler costs at most one limit per CTA.
+__device__ __forceinline__ void km_grid_barrier(unsigned *bar, int *err, volatile int *abort)
 {
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && !*abort) {
         unsigned g0;
         asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(bar + 1) : "memory");
         unsigned prior;
@@ -316,8 +325,9 @@ __device__ __forceinline__ void km_grid_barrier(unsigned *bar, int *err)
                 unsigned gv;
                 asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(gv) : "l"(bar + 1) : "memory");
                 if (gv != g0) break;
-                if ((++spin & 255u) == 0 && global_ns() - t0 > 2000000000ull) {
+                if ((++spin & 255u) == 0 && global_ns() - t0 > g_km_wait_ns) {
                     raise_error(err, RPTQ_DEVERR_TIMEOUT);
+                    *abort = 1;
                     break;
                 }
             }
@@ -409,7 +419,7 @@ __global__ void __launch_bounds__(KM_THREADS, 1)
             rank[j] = p;  // keys of the own segment below this one
         }
         __threadfence();
-        km_grid_barrier(w.bar, err);
+        km_grid_barrier(w.bar, err, abort);
         for (int i = tid; i < C; i += KM_THREADS) allk[i] = __ldcg(w.keys + i);
         __syncthreads();
         // rank = own-segment position + keys below (other segments); equal keys: a lower
@@ -513,10 +523,12 @@ __global__ void __launch_bounds__(KM_THREADS, 1)
                 __syncwarp();
             }
             const int nchg = __syncthreads_count(changed);
-            // publish this CTA's record: warps folded in warp order
+            // publish this CTA's record: warps folded in warp order (a CTA named by the testing
+            // hook leaves out its first record, so the other CTAs' gathers run out)
             const uint32_t flag = (uint32_t)it + 1u;
             uint4 *out = w.sums + ((size_t)(it & 1) * nb + me) * rec;
-            for (int q = tid; q < rec; q += KM_THREADS) {
+            const bool publish = !(it == 0 && me == g_km_withhold);
+            for (int q = tid; q < rec && publish; q += KM_THREADS) {
                 if (q < 2 * g) {
                     double a = 0.0;
 #pragma unroll
@@ -810,6 +822,21 @@ extern "C" int rptq_kmeans_noalloc(const float *ch_max, const float *ch_min, int
                    scale, zero, d.scratch, (cudaStream_t)stream, d.num_sms, d.max_smem, err};
     const cudaError_t e = rptq::launch_kmeans(a);
     if (e != cudaSuccess) {
+        cudaGetLastError();
+        return RPTQ_ERR_CUDA;
+    }
+    return RPTQ_OK;
+}
+
+// ==========================================================================================
+// Testing hook (include/rptq_testing.h): the exchange wait limit and the CTA that leaves out its
+// first Lloyd record, on the current device.
+extern "C" int rptq_testing_kmeans_wait(unsigned long long limit_ns, int withhold_cta)
+{
+    const unsigned long long lim = limit_ns ? limit_ns : 2000000000ull;
+    if (withhold_cta < -1) return RPTQ_ERR_INVALID_ARG;
+    if (cudaMemcpyToSymbol(rptq::g_km_wait_ns, &lim, sizeof(lim)) != cudaSuccess ||
+        cudaMemcpyToSymbol(rptq::g_km_withhold, &withhold_cta, sizeof(withhold_cta)) != cudaSuccess) {
         cudaGetLastError();
         return RPTQ_ERR_CUDA;
     }

@@ -17,6 +17,7 @@
 // (other D): one CTA per (b, h) block.
 #include <algorithm>
 
+#include "../../include/rptq_testing.h"
 #include "kv_stream.cuh"
 #include "launch.h"
 
@@ -25,15 +26,26 @@ namespace rptq {
 // Correctly rounded x / s from r = RN(1/s): q0 = RN(x r), the residual x - q0 s is exact in
 // one fused multiply-add, and q0 + residual * r rounds to RN(x / s) (P. Markstein, "IA-64 and
 // Elementary Functions", 2000, division by a reciprocal with one correction).  Quotients that
-// are exact half-integers therefore stay exact and round half-to-even like the reference.
-__device__ __forceinline__ float div_rn(float x, float s, float r)
+// are exact half-integers therefore stay exact and round half-to-even like the reference.  The
+// residual is exact as long as it is not subnormal: for |x| >= 2^-100 the quotient of every
+// finite bf16 or fp16 x is the IEEE one (checked exhaustively by the tests); below, the code is
+// decided by rint of a quotient far below 1/2 and does not depend on its last bit.
+// The quantizer forms x / (s 2^24) with s' = s 2^24 and r' = RN(1/s) 2^-24 (powers of two: the
+// same significands), so that x r' stays finite for every finite x when s >= 2^-24 (no
+// inf - inf in the correction), and scales back by 2^24 inside the rounding fma.
+__device__ __forceinline__ f32x2 div_rn2(f32x2 x2, f32x2 ns2, f32x2 r2)
 {
-    const float q0 = x * r;
-    const float res = fmaf(-q0, s, x);
-    return fmaf(res, r, q0);
+    const f32x2 q0 = mul2(x2, r2);
+    return fma2(fma2(q0, ns2, x2), r2, q0);
 }
 
 constexpr int KV_ROWS_PER_UNIT = 64;
+constexpr float KV_QSCALE = 16777216.0f;            // 2^24
+constexpr float KV_QSCALE_INV = 5.9604644775390625e-08f;  // 2^-24
+
+// Scales s for which the scaled quotient above is exact (no overflow of x r', no overflow or
+// subnormal r'); other clusters take the IEEE division.
+__device__ __forceinline__ bool kv_fast_scale(float s) { return s >= 0x1p-24f && s <= 0x1p+102f; }
 
 // Coefficients of a thread's DPT channels (h*D + d0 + i) for one head.
 template <int BITS, int DPT>
@@ -41,15 +53,15 @@ struct KvCoef {
     static constexpr int NG = DPT / 8;
     static constexpr int QMAX = (1 << BITS) - 1;
     static constexpr uint32_t MAGIC_BITS = 0x4B400000u;
-    f32x2 ns2[DPT / 2], r2[DPT / 2];  // -s and RN(1/s), two channels per pair
-    float lo_[DPT], hi_[DPT];         // code-domain clamp [-z, qmax - z]
+    f32x2 ns2[DPT / 2], r2[DPT / 2];  // -s 2^24 and RN(1/s) 2^-24, two channels per pair
+    int32_t lo_[DPT], hi_[DPT];       // clamp of the rounded bit pattern: MAGIC_BITS - z .. + qmax
     uint32_t bias[NG];                // sum_i (MAGIC_BITS - z_i) << (BITS*i): removes the rounding constant
-    bool small_z;                     // |z| < 2^21 keeps q + 1.5*2^23 inside one binade (exact rounding)
+    bool fast;                        // every channel: |z| < 2^21 (q + 1.5*2^23 inside one binade) and a fast scale
 
     __device__ __forceinline__ void load(const int32_t *cl, const float *sc, const int32_t *zp, int c0, int g,
                                          int *err)
     {
-        small_z = true;
+        fast = true;
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) bias[gi] = 0;
 #pragma unroll
@@ -62,13 +74,14 @@ struct KvCoef {
                     raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
                     kc = 0;
                 }
-                sv2[h2] = sc[kc];
-                rv2[h2] = __frcp_rn(sv2[h2]);
+                const float sv = sc[kc];
+                sv2[h2] = sv * KV_QSCALE;
+                rv2[h2] = __frcp_rn(sv) * KV_QSCALE_INV;
                 const int z = zp[kc];
-                lo_[i + h2] = (float)(-z);
-                hi_[i + h2] = (float)(QMAX - z);
+                lo_[i + h2] = (int32_t)(MAGIC_BITS - (uint32_t)z);
+                hi_[i + h2] = (int32_t)(MAGIC_BITS + (uint32_t)QMAX - (uint32_t)z);
                 bias[(i + h2) / 8] += (MAGIC_BITS - (uint32_t)z) << (BITS * ((i + h2) % 8));
-                small_z &= (z > -(1 << 21)) && (z < (1 << 21));
+                fast &= (z > -(1 << 21)) && (z < (1 << 21)) && kv_fast_scale(sv);
             }
             ns2[i / 2] = mk2(-sv2[0], -sv2[1]);
             r2[i / 2] = mk2(rv2[0], rv2[1]);
@@ -76,45 +89,53 @@ struct KvCoef {
     }
 };
 
+// One code from an IEEE quotient, exactly as the definition: clamp(rint(x / s) + z, 0, qmax)
+// (the sum in fp64 is exact for every finite quotient, and an infinite one clamps).
+template <int QMAX>
+__device__ __forceinline__ uint32_t kv_code_ieee(float x, float s, int z)
+{
+    const double q = (double)rintf(__fdiv_rn(x, s)) + (double)z;
+    return (uint32_t)fmin(fmax(q, 0.0), (double)QMAX);
+}
+
 // Codes of one row's DPT channels (x in VEC-element 16-byte chunks) -> NG packed 8-code groups.
 template <typename T, int BITS, int DPT>
 __device__ __forceinline__ void kv_quant_row(const uint4 *xb, const KvCoef<BITS, DPT> &cf, uint32_t *grp)
 {
     constexpr int VEC = Elem<T>::VEC;
     constexpr int NG = DPT / 8;
-    const f32x2 magic2 = mk2(MAGIC_RINT, MAGIC_RINT);
-    if (cf.small_z) {
+    const f32x2 magic2 = mk2(MAGIC_RINT, MAGIC_RINT), up2 = mk2(KV_QSCALE, KV_QSCALE);
+    if (cf.fast) {
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) {
             uint32_t acc = 0;
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
                 const int i = gi * 8 + j;
-                // correctly rounded x/s for two channels (reciprocal + one correction)
+                // correctly rounded x / (s 2^24) for two channels, then rint(x / s) + 1.5*2^23:
+                // the bit pattern is MAGIC_BITS + rint(x / s) while |x / s| < 2^22; beyond, and
+                // for an infinite quotient, it falls outside [lo, hi] on the side of its sign,
+                // so the integer clamp below is clamp(rint(x/s), -z, qmax - z) + MAGIC_BITS
                 const f32x2 x2 = pair_of<T>(xb[i / VEC], (i % VEC) / 2);
-                const f32x2 q0 = mul2(x2, cf.r2[i / 2]);
-                const f32x2 q1 = fma2(fma2(q0, cf.ns2[i / 2], x2), cf.r2[i / 2], q0);
-                // clamp(rint(q) + z) == rint(clamp(q, -z, qmax - z)) + z
-                const f32x2 qc = mk2(fminf(fmaxf(lo2(q1), cf.lo_[i]), cf.hi_[i]),
-                                     fminf(fmaxf(hi2(q1), cf.lo_[i + 1]), cf.hi_[i + 1]));
-                const f32x2 b2 = add2(qc, magic2);
-                acc += __float_as_uint(lo2(b2)) << (BITS * j);
-                acc += __float_as_uint(hi2(b2)) << (BITS * (j + 1));
+                const f32x2 b2 = fma2(div_rn2(x2, cf.ns2[i / 2], cf.r2[i / 2]), up2, magic2);
+                const int32_t l0 = min(max((int32_t)__float_as_uint(lo2(b2)), cf.lo_[i]), cf.hi_[i]);
+                const int32_t l1 = min(max((int32_t)__float_as_uint(hi2(b2)), cf.lo_[i + 1]), cf.hi_[i + 1]);
+                acc += (uint32_t)l0 << (BITS * j);
+                acc += (uint32_t)l1 << (BITS * (j + 1));
             }
             grp[gi] = acc - cf.bias[gi];
         }
-    } else {  // a huge zero point: integer rounding and clamping
+    } else {  // a huge zero point or an extreme scale: the IEEE division and the definition
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) {
             uint32_t acc = 0;
+#pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const int i = gi * 8 + j;
-                const float xf = Elem<T>::get(xb[i / VEC], i % VEC);
-                const float si = (i & 1) ? -hi2(cf.ns2[i / 2]) : -lo2(cf.ns2[i / 2]);
-                const float ri = (i & 1) ? hi2(cf.r2[i / 2]) : lo2(cf.r2[i / 2]);
-                const float q = rintf(div_rn(xf, si, ri));
-                const float c = fminf(fmaxf(q, cf.lo_[i]), cf.hi_[i]) - cf.lo_[i];
-                acc |= (uint32_t)c << (BITS * j);
+                // s and z back from the coefficients (exact: a power-of-two scale, an integer)
+                const float sv = -((i & 1) ? hi2(cf.ns2[i / 2]) : lo2(cf.ns2[i / 2])) * KV_QSCALE_INV;
+                const int z = (int)(KvCoef<BITS, DPT>::MAGIC_BITS - (uint32_t)cf.lo_[i]);
+                acc |= kv_code_ieee<KvCoef<BITS, DPT>::QMAX>(Elem<T>::get(xb[i / VEC], i % VEC), sv, z) << (BITS * j);
             }
             grp[gi] = acc;
         }
@@ -419,3 +440,38 @@ cudaError_t launch_kv_quant(const KvArgs &a)
 }
 
 }  // namespace rptq
+
+// ==========================================================================================
+// Testing hook (include/rptq_testing.h): the K/V quantizer's quotient x / s for n values, in the
+// packed form the kernels use (even n) and the scalar form of the integer path (last value of
+// an odd n).
+namespace rptq {
+__global__ void kv_quotient_kernel(const float *x, int64_t n, float s, float *q)
+{
+    const bool fast = kv_fast_scale(s);
+    const float r = __frcp_rn(s) * KV_QSCALE_INV, sp = s * KV_QSCALE;
+    const f32x2 ns2 = mk2(-sp, -sp), r2 = mk2(r, r), up2 = mk2(KV_QSCALE, KV_QSCALE);
+    for (int64_t i = 2 * ((int64_t)blockIdx.x * blockDim.x + threadIdx.x); i < n; i += 2 * (int64_t)gridDim.x * blockDim.x) {
+        const float x1 = i + 1 < n ? x[i + 1] : 0.f;
+        f32x2 v;
+        if (fast)
+            v = mul2(div_rn2(mk2(x[i], x1), ns2, r2), up2);
+        else
+            v = mk2(__fdiv_rn(x[i], s), __fdiv_rn(x1, s));
+        q[i] = lo2(v);
+        if (i + 1 < n) q[i + 1] = hi2(v);
+    }
+}
+}  // namespace rptq
+
+extern "C" int rptq_testing_kv_quotient(const float *x, int64_t n, float s, float *q, rptq_stream_t stream)
+{
+    if (n < 0 || !(s > 0.0f) || !(s < INFINITY)) return RPTQ_ERR_INVALID_ARG;
+    if (n == 0) return RPTQ_OK;
+    if (!x || !q) return RPTQ_ERR_INVALID_ARG;
+    const int64_t pairs = (n + 1) / 2;
+    const unsigned grid = (unsigned)std::min<int64_t>((pairs + 255) / 256, 4096);
+    rptq::kv_quotient_kernel<<<grid, 256, 0, (cudaStream_t)stream>>>(x, n, s, q);
+    if (cudaGetLastError() != cudaSuccess) return RPTQ_ERR_CUDA;
+    return RPTQ_OK;
+}

@@ -49,6 +49,9 @@ SIGNATURES = {
     "rptq_ln_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_quant": (_I, [_P, _P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
+    # include/rptq_testing.h
+    "rptq_testing_kv_quotient": (_I, [_P, _I64, _F, _P, _P]),
+    "rptq_testing_kmeans_wait": (_I, [ctypes.c_ulonglong, _I]),
 }
 
 _lib = None
@@ -238,3 +241,20 @@ def rptq_dequant(codes: torch.Tensor, cluster, scale, zero, bits: int, out_dtype
                             _stream(stream))
     _check(st, "rptq_dequant")
     return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Test hooks (include/rptq_testing.h)
+def rptq_testing_kv_quotient(x: torch.Tensor, s: float, q=None, stream=None) -> torch.Tensor:
+    """The K/V quantizer's quotient x / s for every value of the fp32 tensor x."""
+    assert x.dtype == torch.float32
+    if q is None:
+        q = torch.empty_like(x)
+    _check(lib().rptq_testing_kv_quotient(_ptr(x), x.numel(), float(s), _ptr(q), _stream(stream)),
+           "rptq_testing_kv_quotient")
+    return q
+
+
+def rptq_testing_kmeans_wait(limit_ns: int = 0, withhold_cta: int = -1) -> None:
+    """KMeans exchange wait limit (0: the default) and a CTA that leaves out its first record."""
+    _check(lib().rptq_testing_kmeans_wait(int(limit_ns), int(withhold_cta)), "rptq_testing_kmeans_wait")

@@ -5,10 +5,13 @@ Tolerances (each follows from the arithmetic of the two sides):
     bit-exact;
   * centroids: relative 1e-6 (the GPU sums cluster members in a different fixed order);
   * codes: identical except +-1 at rounding boundaries, on at most 1e-4 of the elements;
-  * LayerNorm output (fp32): |gpu - y| <= 1e-5 * (|gamma| * (1 + |xhat|) + |beta|), y and xhat
-    from the oracle's fp64 LayerNorm (the mean's rounding shifts every normalised value by an
-    amount relative to the row's spread, hence the unit floor on |xhat|); a bf16 output adds
-    one round-to-nearest of 8 significant bits, at most 2^-8 |y|; fp16 adds 2^-11 |y| + 2^-25.
+  * LayerNorm output (fp32): |gpu - y| <= 1e-5 |y| + 2.5e-7, y from the oracle's fp64
+    LayerNorm.  Measured on a B200 over the suite's 58 fp32 comparisons (dense outputs and
+    LayerNorm-mode calibration statistics, all three input types, offset rows included): the
+    worst error is within 1e-5 |y| + 6.6e-8, so the floor keeps a factor of about 4; where
+    |y| ~ 1e-3 the relative error alone reaches 2.5e-5 (the fp32 rounding of the mean and of
+    rstd moves y by a few 1e-8 absolute).  A bf16 output adds one round-to-nearest of 8
+    significant bits, at most 2^-8 |y|; fp16 adds 2^-11 |y| + 2^-25.
 """
 import numpy as np
 import torch
@@ -26,20 +29,37 @@ def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().numpy()
 
 
+# measured agreement of every comparison in this session (written out by conftest.py when
+# RPTQ_PARITY_REPORT names a file): codes -> off-by-one fraction, LN -> worst errors
+REPORT = {"codes": {}, "ln": {}}
+
+
 def compare_codes(gpu_packed: np.ndarray, ref_packed: np.ndarray, C: int, bits: int, what=""):
     """Unpack both and apply the codes bar; returns the off-by-one fraction."""
     g = oracle.unpack(gpu_packed.reshape(-1, C * bits // 8), C, bits).astype(np.int16)
     r = oracle.unpack(ref_packed.reshape(-1, C * bits // 8), C, bits).astype(np.int16)
     d = np.abs(g - r)
-    assert d.max(initial=0) <= 1, f"{what}: code differs by {d.max()} (> 1)"
     frac = float((d == 1).mean()) if d.size else 0.0
+    REPORT["codes"][_key(REPORT["codes"], what)] = {"elements": int(d.size), "off_by_one": int((d == 1).sum()), "fraction": frac,
+                             "max_diff": int(d.max(initial=0))}
+    assert d.max(initial=0) <= 1, f"{what}: code differs by {d.max()} (> 1)"
     assert frac <= CODE_OFF_BY_ONE_MAX, f"{what}: off-by-one fraction {frac:.2e}"
     return frac
 
 
-def ln_tol32(y64: np.ndarray, gamma_s: np.ndarray, beta_s: np.ndarray) -> np.ndarray:
-    xhat = (y64 - beta_s) / gamma_s
-    return 1e-5 * (np.abs(gamma_s) * (1.0 + np.abs(xhat)) + np.abs(beta_s))
+LN_REL32, LN_ABS32 = 1e-5, 2.5e-7
+
+
+def ln_tol32(y64: np.ndarray, gamma_s=None, beta_s=None) -> np.ndarray:
+    return LN_REL32 * np.abs(y64) + LN_ABS32
+
+
+def _key(table: dict, what: str) -> str:
+    k, n = what, 1
+    while k in table:
+        n += 1
+        k = f"{what} #{n}"
+    return k
 
 
 def compare_ln(gpu: np.ndarray, y64: np.ndarray, gamma_s, beta_s, dtype: str, what=""):
@@ -49,6 +69,12 @@ def compare_ln(gpu: np.ndarray, y64: np.ndarray, gamma_s, beta_s, dtype: str, wh
     elif dtype == "f16":
         tol = tol + 2.0 ** -11 * np.abs(y64) * (1 + 1e-5) + 2.0 ** -25
     err = np.abs(gpu.astype(np.float64) - y64)
+    ay = np.abs(y64)
+    rel = err[ay > 1e-3] / ay[ay > 1e-3]
+    REPORT["ln"][_key(REPORT["ln"], f"{what} ({dtype})")] = {
+        "values": int(err.size), "max_abs": float(err.max(initial=0)),
+        "max_rel_where_abs_y_gt_1e-3": float(rel.max(initial=0)),
+        "max_excess_over_1e-5_rel": float((err - 1e-5 * ay).max(initial=0))}
     bad = err > tol
     assert not bad.any(), f"{what}: {bad.sum()} LN values out of tolerance, worst {(err - tol).max():.3e}"
 

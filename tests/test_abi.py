@@ -10,9 +10,13 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def _declared_functions():
-    src = open(os.path.join(ROOT, "include", "rptq.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(rptq_[a-z_0-9]+)\s*\(", src)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(rptq_[a-z_0-9]+)\s*\(", src))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -106,8 +110,9 @@ def test_empty_problems_succeed_on_the_host(rlib):
 
 
 def _prototypes():
-    """name -> list of C parameter types, parsed from the prototypes in include/rptq.h."""
-    src = open(os.path.join(ROOT, "include", "rptq.h")).read()
+    """name -> list of C parameter types, parsed from the prototypes in include/*.h."""
+    src = "".join(open(os.path.join(ROOT, "include", h)).read()
+                  for h in sorted(os.listdir(os.path.join(ROOT, "include"))) if h.endswith(".h"))
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
     src = re.sub(r"//[^\n]*", "", src)
     out = {}
@@ -122,7 +127,7 @@ def _ctype_of(param: str):
     if "*" in t or t.endswith("rptq_stream_t"):
         return ctypes.c_void_p if "char" not in t else ctypes.c_char_p
     return {"int": ctypes.c_int, "int64_t": ctypes.c_int64, "size_t": ctypes.c_size_t,
-            "float": ctypes.c_float}[t.replace("const ", "").strip()]
+            "float": ctypes.c_float, "unsigned long long": ctypes.c_ulonglong}[t.replace("const ", "").strip()]
 
 
 def test_binding_argument_types_match_the_header():

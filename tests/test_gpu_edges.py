@@ -141,3 +141,35 @@ def test_kv_quant_huge_zero_point_integer_path(dtype, S):
                                torch.from_numpy(cal["scale"]).to(DEV), torch.from_numpy(z).to(DEV), None, None,
                                None, bits)
     assert np.array_equal(to_np(kq), pk)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("S", [40, 128])
+def test_kv_quant_extreme_scales_and_overflowing_quotients(dtype, S):
+    """Clusters with a scale below 2^-24 (the IEEE-division path) and values whose quotient x / s
+    overflows fp32 (a positive overflow must give qmax, a negative one 0, as in the definition):
+    codes are exact in both K/V kernels (S = 40: warp kernel; S = 128: streaming ring)."""
+    B, H, D, g, bits = 2, 3, 128, 4, 3
+    mk = synthetic.channel_model(H * D, 19, tag=1)
+    k = synthetic.kv_cache(B, H, S, D, mk, 19, "k", dtype)
+    kf = oracle._f32(k)
+    flat = np.ascontiguousarray(kf.transpose(0, 2, 1, 3).reshape(-1, H * D))
+    kmx, kmn = oracle.minmax(flat)
+    cal = oracle.calibrate(kmx, kmn, g, 5, bits)
+    s = cal["scale"].copy()
+    big = 60000.0 if dtype == "f16" else 3.0e38
+    s[0] = np.float32(2.0 ** -30)        # below the fast range
+    s[1] = np.float32(1e-3 if dtype == "f16" else 1e-20)  # big values overflow x / s
+    k2 = k.clone()
+    lab = cal["labels"].reshape(H, D)
+    for h in range(H):
+        cols = np.nonzero(lab[h] == 1)[0]
+        if len(cols):
+            k2[:, h, ::3, cols[0]] = big
+            k2[:, h, 1::3, cols[0]] = -big
+    kf2 = oracle._f32(k2)
+    pk = oracle.kv_quant(kf2, cal["labels"], s, cal["zero"], bits)
+    kq, _ = rptq.rptq_kv_quant(k2.to(DEV), None, torch.from_numpy(cal["labels"]).to(DEV),
+                               torch.from_numpy(s).to(DEV), torch.from_numpy(cal["zero"]).to(DEV), None, None,
+                               None, bits)
+    assert np.array_equal(to_np(kq), pk)
