@@ -65,3 +65,23 @@ def test_stage_accounting_per_workload():
     st = bench.stage_list(W.WORKLOADS["tiny-768"])
     assert [s[0] for s in st] == ["calib_ln", "kmeans", "ln_reorder_quant", "dequant_act"]
     assert sum(l for _, _, l in st) == 2 + 2 + 1 + 1
+
+
+def test_gpus_n_starts_n_ranks():
+    """`--gpus 2` outside a launcher starts two ranks under torchrun (checked without a GPU:
+    --dry-run makes each rank report its place and exit)."""
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    env.pop("WORLD_SIZE", None)
+    out = subprocess.run([sys.executable, "bench.py", "--gpus", "2", "--dry-run"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    ranks = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert sorted(r["rank"] for r in ranks) == [0, 1]
+    assert all(r["world_size"] == 2 for r in ranks)
+
+
+def test_world_size_mismatch_is_refused():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, "bench.py", "--gpus", "4", "--dry-run"], cwd=ROOT, env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert out.returncode != 0 and "--gpus 4" in out.stderr
