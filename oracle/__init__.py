@@ -240,6 +240,37 @@ def kv_dequant(packed, D, col_cluster, s, z, bits):
     return out
 
 
+def kv_append(cache, new, s_begin, col_cluster, s, z, bits):
+    """Decode-time append ([RPTQ-art] results paragraph: the K/V cache is quantized per cluster;
+    closing paragraph: the cache dominates memory at large batch x sequence).  A copy of the
+    packed cache [B, H, S_max, D*bits/8] whose positions s_begin .. s_begin + s_len - 1 hold the
+    codes of the new tokens [B, H, s_len, D] (quantized exactly as kv_quant does); every other
+    position is unchanged.  Definition written out: quantize the new rows, store them in place."""
+    out = np.array(cache, dtype=np.uint8, copy=True)
+    n = np.asarray(new).shape[2]
+    assert 0 <= s_begin and s_begin + n <= out.shape[2]
+    out[:, :, s_begin:s_begin + n] = kv_quant(new, col_cluster, s, z, bits)
+    return out
+
+
+def kv_decode_attention(q, k_codes, v_codes, L, D, clk, sk, zk, clv, sv, zv, bits, scale=None):
+    """One decode step of attention reading the packed caches (the consumer of the K/V codes;
+    [RPTQ-art] results paragraph and closing memory paragraph).  For every (b, h):
+    K, V = the fp32 dequantized rows 0 .. L-1 (exactly kv_dequant), scores = (q . K_s) * scale
+    (scale = 1/sqrt(D) by default), p = softmax over the L positions, out = sum_s p_s V_s; the
+    products, sums and the softmax in fp64.  q [B, H, D]; returns fp64 [B, H, D] and the fp64
+    scores [B, H, L] (for error bounds)."""
+    q = np.asarray(_f32(q), dtype=np.float64)
+    K = kv_dequant(np.ascontiguousarray(k_codes[:, :, :L]), D, clk, sk, zk, bits).astype(np.float64)
+    V = kv_dequant(np.ascontiguousarray(v_codes[:, :, :L]), D, clv, sv, zv, bits).astype(np.float64)
+    sc = (1.0 / np.sqrt(D)) if scale is None else float(scale)
+    scores = np.einsum("bhd,bhsd->bhs", q, K) * sc
+    m = scores.max(axis=2, keepdims=True)
+    e = np.exp(scores - m)
+    p = e / e.sum(axis=2, keepdims=True)
+    return np.einsum("bhs,bhsd->bhd", p, V), scores
+
+
 def calibrate(ch_max, ch_min, g, iters, bits):
     """The whole offline chain on given statistics: KMeans -> reorder -> cluster params."""
     labels, cent = kmeans(ch_max, ch_min, g, iters)
