@@ -80,6 +80,9 @@ def stage_list(w: W.Workload):
         st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
     if k:
         st += [("dequant_kv", 2 * W.bytes_dequant(k.elems, k.dtype, k.bits), 2)]
+        # one decode step: a token appended to K and V, then attention over the whole cache
+        st += [("kv_append", W.bytes_kv_append(k.B, k.H, k.D, k.dtype, k.bits), 1),
+               ("kv_decode_attention", W.bytes_kv_attention(k.B, k.H, k.S, k.D, k.bits), 1)]
     return st
 
 
@@ -126,6 +129,13 @@ class Step:
             kvdt = synthetic.torch_dtype(k.dtype)
             self.khat = torch.empty((k.B, k.H, k.S, k.D), dtype=kvdt, device=device)
             self.vhat = torch.empty_like(self.khat)
+            # the decode step's new token and query
+            self.knew = synthetic.kv_cache(k.B, k.H, 1, k.D, mk, w.seed + 7919 * rank + 1, "k", k.dtype, device)
+            self.vnew = synthetic.kv_cache(k.B, k.H, 1, k.D, mv, w.seed + 7919 * rank + 1, "v", k.dtype, device)
+            gq = torch.Generator(device=device)
+            gq.manual_seed(w.seed * 31 + rank)
+            self.q = torch.randn((k.B, k.H, k.D), generator=gq, device=device, dtype=torch.float32) * 0.05
+            self.attn = torch.empty((k.B, k.H, k.D), dtype=torch.float32, device=device)
         # the three KMeans problems are independent: they run concurrently on their own streams
         self.side = [torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)]
 
@@ -205,6 +215,16 @@ class Step:
             r.rptq_dequant(self.vq, self.kmv["labels"], self.kmv["scale"], self.kmv["zero"], k.bits,
                            layout=r.RPTQ_LAYOUT_BHSD, out=self.vhat)
             mark("dequant_kv", 1)
+            mark("kv_append", 0)
+            r.rptq_kv_append(self.knew, self.vnew, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],
+                             self.kmv["labels"], self.kmv["scale"], self.kmv["zero"], k.bits,
+                             k_cache=self.kq, v_cache=self.vq, s_begin=k.S - 1)
+            mark("kv_append", 1)
+            mark("kv_decode_attention", 0)
+            r.rptq_kv_decode_attention(self.q, self.kq, self.vq, k.S, self.kmk["labels"], self.kmk["scale"],
+                                       self.kmk["zero"], self.kmv["labels"], self.kmv["scale"], self.kmv["zero"],
+                                       k.bits, out=self.attn)
+            mark("kv_decode_attention", 1)
 
 
 # ------------------------------------------------------------------------------------------

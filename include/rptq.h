@@ -225,6 +225,46 @@ int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t
                   int bits, uint8_t *k_codes, uint8_t *v_codes, rptq_stream_t stream);
 
 /*
+ * Decode-time K/V append: the new tokens of one step quantized into preallocated caches.
+ * [RPTQ-art] results paragraph (K/V cache quantized per cluster: W4A4KV / W4A3KV / W3A3KV) and
+ * closing memory paragraph (the cache dominates memory at large batch x sequence).
+ *   k_new, v_new  [B, H, s_len, D] of `dtype` (either may be NULL, not both), channel c = h*D + d.
+ *   k_cache, v_cache  uint8 [B, H, S_max, D*bits/8] packed caches (rptq_kv_quant's layout);
+ *                positions s_begin .. s_begin + s_len - 1 of every (b, h) receive the codes of
+ *                the new tokens, computed exactly as rptq_kv_quant computes them; every other
+ *                byte is left as it is.
+ *   cluster_*, scale_*, zero_*: as in rptq_kv_quant (the calibration of that tensor).
+ * s_begin + s_len must not exceed S_max (RPTQ_ERR_INVALID_ARG).  D must be a multiple of 8,
+ * H*D <= RPTQ_MAX_CHANNELS.  B == 0 or s_len == 0 is valid: nothing is launched and no pointer
+ * is read.
+ */
+int rptq_kv_append(const void *k_new, const void *v_new, int dtype, int B, int H, int64_t s_len,
+                   int D, int64_t S_max, int64_t s_begin, const int32_t *cluster_k,
+                   const float *scale_k, const int32_t *zero_k, const int32_t *cluster_v,
+                   const float *scale_v, const int32_t *zero_v, int g, int bits,
+                   uint8_t *k_cache, uint8_t *v_cache, rptq_stream_t stream);
+
+/*
+ * One decode step of attention over the packed caches, dequantizing every code in registers
+ * as it is read (value = s_k * (q - z_k) in fp32, the value rptq_dequant writes): the consumer
+ * of the quantized K/V cache ([RPTQ-art] results and closing memory paragraphs).  For every
+ * (b, h): score_s = scale * sum_d q[b,h,d] K[b,h,s,d] for s < L, p = softmax(score),
+ * out[b,h,d] = sum_s p_s V[b,h,s,d].
+ *   q    fp32 [B, H, D] (one query per (b, h)).   out  fp32 [B, H, D].
+ *   k_cache, v_cache  uint8 [B, H, S_max, D*bits/8]; positions 0 .. L-1 are read.
+ *   cluster_*, scale_*, zero_*: the caches' calibrations (channel c = h*D + d).
+ *   scale  > 0, or 0 for 1 / sqrt(D).
+ * D must be a power of two in [8, 256]; 1 <= L <= S_max and L <= 16384 (the scores of a (b, h)
+ * stay in shared memory).  Arithmetic in fp32 (fma dot products, expf, the sums in a fixed
+ * order).  B == 0 is valid: nothing is launched.
+ */
+int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t *k_cache,
+                             const uint8_t *v_cache, int64_t S_max, int64_t L,
+                             const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
+                             const int32_t *cluster_v, const float *scale_v, const int32_t *zero_v,
+                             int g, int bits, float scale, float *out, rptq_stream_t stream);
+
+/*
  * Dequantization, [Basics] section 1.3: value = s_k * (q - z_k), computed in fp32 (one
  * rounding) and rounded to out_dtype.
  *   layout RPTQ_LAYOUT_ROWS: codes [n0, n1*bits/8] with n0 = rows, n1 = C; cluster[j] is the

@@ -287,6 +287,61 @@ int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t
     return cuda_status(launch_kv_quant(a));
 }
 
+int rptq_kv_append(const void *k_new, const void *v_new, int dtype, int B, int H, int64_t s_len, int D,
+                   int64_t S_max, int64_t s_begin, const int32_t *cluster_k, const float *scale_k,
+                   const int32_t *zero_k, const int32_t *cluster_v, const float *scale_v,
+                   const int32_t *zero_v, int g, int bits, uint8_t *k_cache, uint8_t *v_cache,
+                   rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (D <= 0 || D % 8 != 0 || D > 2048 || H <= 0 || (int64_t)H * D > RPTQ_MAX_CHANNELS)
+        return RPTQ_ERR_UNSUPPORTED;
+    if (B < 0 || s_len < 0 || S_max < 0 || s_begin < 0 || g <= 0) return RPTQ_ERR_INVALID_ARG;
+    if (s_begin + s_len > S_max) return RPTQ_ERR_INVALID_ARG;  // past the end of the cache
+    if (B == 0 || s_len == 0) return RPTQ_OK;  // nothing to append: no pointer is read
+    if (!k_new && !v_new) return RPTQ_ERR_INVALID_ARG;
+    if (k_new && (!cluster_k || !scale_k || !zero_k || !k_cache || !aligned16(k_new) || !aligned16(k_cache)))
+        return RPTQ_ERR_INVALID_ARG;
+    if (v_new && (!cluster_v || !scale_v || !zero_v || !v_cache || !aligned16(v_new) || !aligned16(v_cache)))
+        return RPTQ_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    KvAppendArgs a{k_new, v_new, dtype, B, H, s_len, D, S_max, s_begin, cluster_k, scale_k, zero_k,
+                   cluster_v, scale_v, zero_v, g, bits, k_cache, v_cache, d.err, (cudaStream_t)stream,
+                   d.num_sms};
+    return cuda_status(launch_kv_append(a));
+}
+
+int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t *k_cache,
+                             const uint8_t *v_cache, int64_t S_max, int64_t L,
+                             const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
+                             const int32_t *cluster_v, const float *scale_v, const int32_t *zero_v,
+                             int g, int bits, float scale, float *out, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (D < 8 || D > 256 || (D & (D - 1)) != 0 || H <= 0 || (int64_t)H * D > RPTQ_MAX_CHANNELS)
+        return RPTQ_ERR_UNSUPPORTED;
+    if (L > KV_ATTN_MAX_L) return RPTQ_ERR_UNSUPPORTED;
+    if (B < 0 || L < 1 || L > S_max || g <= 0 || !(scale >= 0.0f) || !(scale < INFINITY))
+        return RPTQ_ERR_INVALID_ARG;
+    if (B == 0) return RPTQ_OK;
+    if (!q || !k_cache || !v_cache || !out || !cluster_k || !scale_k || !zero_k || !cluster_v ||
+        !scale_v || !zero_v)
+        return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out))
+        return RPTQ_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    KvAttnArgs a{q, B, H, D, k_cache, v_cache, S_max, L, cluster_k, scale_k, zero_k, cluster_v,
+                 scale_v, zero_v, g, bits, scale, out, d.err, (cudaStream_t)stream, d.max_smem};
+    return cuda_status(launch_kv_attention(a));
+}
+
 int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,
                  const int32_t *cluster, const float *scale, const int32_t *zero, int g,
                  int bits, void *out, int out_dtype, rptq_stream_t stream)

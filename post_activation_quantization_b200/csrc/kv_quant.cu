@@ -429,6 +429,63 @@ static cudaError_t launch_kv_d(const KvArgs &a)
     return a.bits == 4 ? launch_kv_cta<T, 4, 8>(a) : launch_kv_cta<T, 3, 8>(a);
 }
 
+// ------------------------------------------------------------------------------------------
+// Decode-time append: the new tokens [B, H, s_len, D] of one step, quantized exactly as above,
+// written at positions s_begin .. s_begin + s_len - 1 of the packed caches [B, H, S_max, D*b/8].
+// One thread per 8-channel chunk of a new row (s_len is 1 in decode, so the work is B*H*D/8
+// chunks: launch latency and the coefficient gathers dominate, not bandwidth).
+template <typename T, int BITS>
+__global__ void __launch_bounds__(256)
+    kv_append_kernel(KvTensors t, int B, int H, int64_t s_len, int D, int64_t S_max, int64_t s_begin, int g,
+                     int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;
+    const int tensor = blockIdx.y;
+    if (!t.src[tensor]) return;
+    const int cpr = D / 8;  // chunks per row
+    const int64_t total = (int64_t)B * H * s_len * cpr;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int c8 = (int)(i % cpr);
+        const int64_t row = i / cpr;  // ((b * H + h) * s_len + s)
+        const int64_t s = row % s_len, bh = row / s_len;
+        const int h = (int)(bh % H);
+        KvCoef<BITS, 8> cf;
+        cf.load(t.cl[tensor], t.sc[tensor], t.zp[tensor], h * D + c8 * 8, g, err);
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(t.src[tensor]) + row * D + c8 * 8);
+        uint4 xb[8 / VEC];
+#pragma unroll
+        for (int k = 0; k < 8 / VEC; ++k) xb[k] = ldg_stream(src + k);
+        uint32_t grp[1];
+        kv_quant_row<T, BITS, 8>(xb, cf, grp);
+        uint8_t *o = t.dst[tensor] + (bh * S_max + s_begin + s) * (int64_t)(D * BITS / 8) + c8 * BITS;
+        kv_store_row<BITS, 8>(o, grp);
+    }
+}
+
+template <typename T>
+static cudaError_t launch_kv_append_t(const KvAppendArgs &a)
+{
+    KvTensors t{{a.k, a.v}, {a.kq, a.vq}, {a.ck, a.cv}, {a.sk, a.sv}, {a.zk, a.zv}};
+    const int64_t total = (int64_t)a.B * a.H * a.s_len * (a.D / 8);
+    const unsigned grid = (unsigned)std::min<int64_t>((total + 255) / 256, (int64_t)a.num_sms * 8);
+    const dim3 gd(grid, 2);
+    if (a.bits == 4)
+        kv_append_kernel<T, 4><<<gd, 256, 0, a.stream>>>(t, a.B, a.H, a.s_len, a.D, a.S_max, a.s_begin, a.g, a.err);
+    else
+        kv_append_kernel<T, 3><<<gd, 256, 0, a.stream>>>(t, a.B, a.H, a.s_len, a.D, a.S_max, a.s_begin, a.g, a.err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kv_append(const KvAppendArgs &a)
+{
+    if (a.s_len == 0 || a.B == 0) return cudaSuccess;
+    switch (a.dtype) {
+    case RPTQ_F32: return launch_kv_append_t<float>(a);
+    case RPTQ_F16: return launch_kv_append_t<__half>(a);
+    default: return launch_kv_append_t<__nv_bfloat16>(a);
+    }
+}
+
 cudaError_t launch_kv_quant(const KvArgs &a)
 {
     if (a.S == 0 || a.B == 0 || a.H == 0) return cudaSuccess;

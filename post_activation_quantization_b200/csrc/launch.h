@@ -77,6 +77,44 @@ struct KvArgs {
     int num_sms;
 };
 
+struct KvAppendArgs {
+    const void *k, *v;
+    int dtype, B, H;
+    int64_t s_len;
+    int D;
+    int64_t S_max, s_begin;
+    const int32_t *ck;
+    const float *sk;
+    const int32_t *zk;
+    const int32_t *cv;
+    const float *sv;
+    const int32_t *zv;
+    int g, bits;
+    uint8_t *kq, *vq;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+};
+
+struct KvAttnArgs {
+    const float *q;
+    int B, H, D;
+    const uint8_t *kq, *vq;
+    int64_t S_max, L;
+    const int32_t *ck;
+    const float *sk;
+    const int32_t *zk;
+    const int32_t *cv;
+    const float *sv;
+    const int32_t *zv;
+    int g, bits;
+    float scale;
+    float *out;
+    int *err;
+    cudaStream_t stream;
+    int max_smem;
+};
+
 struct DequantArgs {
     const uint8_t *codes;
     int layout;
@@ -117,6 +155,11 @@ cudaError_t launch_calib(const CalibArgs &a);
 cudaError_t launch_kv_calib(const KvCalibArgs &a);
 cudaError_t launch_kv_quant(const KvArgs &a);
 cudaError_t launch_dequant(const DequantArgs &a);
+cudaError_t launch_kv_append(const KvAppendArgs &a);
+cudaError_t launch_kv_attention(const KvAttnArgs &a);
+// largest number of cache positions one decode-attention call reads (its scores stay in shared
+// memory)
+constexpr int64_t KV_ATTN_MAX_L = 16384;
 cudaError_t launch_kmeans(const KmArgs &a);
 size_t kmeans_ws_bytes(int C, int g);
 // (C, g) within the limits and the fused KMeans kernel's shared memory within max_smem

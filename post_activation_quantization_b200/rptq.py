@@ -49,6 +49,8 @@ SIGNATURES = {
     "rptq_ln_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_quant": (_I, [_P, _P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
+    "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
+    "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
     # include/rptq_testing.h
     "rptq_testing_kv_quotient": (_I, [_P, _I64, _F, _P, _P]),
     "rptq_testing_kmeans_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -240,6 +242,36 @@ def rptq_dequant(codes: torch.Tensor, cluster, scale, zero, bits: int, out_dtype
                             _ptr(zero), scale.numel(), bits, _ptr(out), _DT[out.dtype],
                             _stream(stream))
     _check(st, "rptq_dequant")
+    return out
+
+
+def rptq_kv_append(k_new, v_new, cluster_k, scale_k, zero_k, cluster_v, scale_v, zero_v, bits: int,
+                   k_cache=None, v_cache=None, s_begin: int = 0, stream=None):
+    """Quantize the new tokens [B, H, s_len, D] into positions s_begin.. of the packed caches
+    [B, H, S_max, D*bits/8] (in place)."""
+    t = k_new if k_new is not None else v_new
+    B, H, s_len, D = t.shape
+    cache = k_cache if k_cache is not None else v_cache
+    S_max = cache.shape[2]
+    g = (scale_k if scale_k is not None else scale_v).numel()
+    st = lib().rptq_kv_append(_ptr(k_new), _ptr(v_new), _DT[t.dtype], B, H, s_len, D, S_max, s_begin,
+                              _ptr(cluster_k), _ptr(scale_k), _ptr(zero_k), _ptr(cluster_v), _ptr(scale_v),
+                              _ptr(zero_v), g, bits, _ptr(k_cache), _ptr(v_cache), _stream(stream))
+    _check(st, "rptq_kv_append")
+    return k_cache, v_cache
+
+
+def rptq_kv_decode_attention(q, k_cache, v_cache, L: int, cluster_k, scale_k, zero_k, cluster_v, scale_v,
+                             zero_v, bits: int, scale: float = 0.0, out=None, stream=None):
+    """Softmax attention of q [B, H, D] (fp32) over positions 0..L-1 of the packed caches."""
+    B, H, D = q.shape
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    st = lib().rptq_kv_decode_attention(_ptr(q), B, H, D, _ptr(k_cache), _ptr(v_cache), k_cache.shape[2], L,
+                                        _ptr(cluster_k), _ptr(scale_k), _ptr(zero_k), _ptr(cluster_v),
+                                        _ptr(scale_v), _ptr(zero_v), scale_k.numel(), bits, float(scale),
+                                        _ptr(out), _stream(stream))
+    _check(st, "rptq_kv_decode_attention")
     return out
 
 

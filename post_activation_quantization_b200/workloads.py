@@ -105,3 +105,14 @@ def bytes_dequant(n_elems: int, out_dtype: str, bits: int) -> int:
 def kv_cache_bytes(layers: int, batch: int, seq: int, hidden: int, bits: int) -> int:
     """Size of a K+V cache: two tensors of layers x batch x seq x hidden values of `bits` bits."""
     return 2 * layers * batch * seq * hidden * bits // 8
+
+
+def bytes_kv_append(B: int, H: int, D: int, dtype: str, bits: int) -> int:
+    """One decode step's append: read one new token of K and of V, write its packed codes."""
+    return 2 * (B * H * D * ESIZE[dtype] + B * H * D * bits // 8)
+
+
+def bytes_kv_attention(B: int, H: int, L: int, D: int, bits: int) -> int:
+    """Decode attention over L positions: read the packed K and V rows once, the fp32 query,
+    write the fp32 output."""
+    return 2 * B * H * L * D * bits // 8 + 2 * B * H * D * 4

@@ -49,7 +49,7 @@ def test_stage_accounting_per_workload():
     from post_activation_quantization_b200 import workloads as W
     st = bench.stage_list(W.WORKLOADS["opt175b-12288"])
     assert [s[0] for s in st] == ["calib_ln", "kv_calib", "kmeans", "ln_reorder_quant", "kv_quant", "dequant_act",
-                                  "dequant_kv"]
+                                  "dequant_kv", "kv_append", "kv_decode_attention"]
     b = dict((n, v) for n, v, _ in st)
     T, C, Tc, kv = 32768, 12288, 262144, 8 * 96 * 2048 * 128
     assert b["calib_ln"] == Tc * C * 2
@@ -58,10 +58,12 @@ def test_stage_accounting_per_workload():
     assert b["kv_quant"] == 2 * (kv * 2 + kv * 3 // 8)
     assert b["dequant_act"] == T * C * 3 // 8 + T * C * 2
     assert b["dequant_kv"] == 2 * (kv * 3 // 8 + kv * 2)
-    assert sum(l for _, _, l in st) == 17  # 2 + 4 + 6 + 1 + 1 + 1 + 2
+    assert b["kv_append"] == 2 * (8 * 96 * 128 * 2 + 8 * 96 * 128 * 3 // 8)
+    assert b["kv_decode_attention"] == 2 * kv * 3 // 8 + 2 * 8 * 96 * 128 * 4
+    assert sum(l for _, _, l in st) == 19  # 2 + 4 + 6 + 1 + 1 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["kv-4096"])
-    assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "dequant_kv"]
-    assert sum(l for _, _, l in st) == 4 + 4 + 1 + 2
+    assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "dequant_kv", "kv_append", "kv_decode_attention"]
+    assert sum(l for _, _, l in st) == 4 + 4 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["tiny-768"])
     assert [s[0] for s in st] == ["calib_ln", "kmeans", "ln_reorder_quant", "dequant_act"]
     assert sum(l for _, _, l in st) == 2 + 2 + 1 + 1
