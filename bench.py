@@ -74,6 +74,8 @@ def stage_list(w: W.Workload):
     st += [("kmeans", 0, 2 * ((1 if a else 0) + (2 if k else 0)))]
     if a:
         st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+        # the unfused pipeline the fused kernel replaces (a measurement baseline, same results)
+        st += [("explicit_reorder_baseline", W.bytes_explicit_reorder(w.T, w.C, w.dtype, w.bits), 3)]
     if k:
         st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
     if a:
@@ -110,6 +112,9 @@ class Step:
             self.km = self._km_out(w.C, w.g)
             self.ws = torch.empty(rptq.rptq_kmeans_workspace_size(w.C, w.g), dtype=torch.uint8, device=device)
             self.codes = torch.empty((w.T, w.C * w.bits // 8), dtype=torch.uint8, device=device)
+            self.xr_y = torch.empty((w.T, w.C), dtype=torch.float32, device=device)
+            self.xr_yr = torch.empty_like(self.xr_y)
+            self.xr_codes = torch.empty_like(self.codes)
             self.xhat = torch.empty((w.T, w.C), dtype=dt, device=device)
         if self.kvw:
             k = self.kvw
@@ -197,6 +202,11 @@ class Step:
             r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
                                     self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
             mark("ln_reorder_quant", 1)
+            mark("explicit_reorder_baseline", 0)
+            r.rptq_baseline_explicit_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
+                                                   self.km["scale"], self.km["zero"], w.bits, eps=w.eps,
+                                                   y=self.xr_y, y_reordered=self.xr_yr, codes=self.xr_codes)
+            mark("explicit_reorder_baseline", 1)
         if k:
             mark("kv_quant", 0)
             r.rptq_kv_quant(self.k, self.v, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librptq.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["api.cu", "calib.cu", "kmeans.cu", "ln_quant.cu", "kv_quant.cu", "dequant.cu", "kv_attention.cu"]
+SOURCES = ["api.cu", "calib.cu", "kmeans.cu", "ln_quant.cu", "kv_quant.cu", "dequant.cu", "kv_attention.cu", "explicit_reorder.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -28,7 +28,8 @@ def nvcc() -> str:
 
 def _deps(src: str) -> list[str]:
     return [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
-        os.path.join(ROOT, "include", "rptq.h"), os.path.join(ROOT, "include", "rptq_testing.h"), src]
+        os.path.join(ROOT, "include", "rptq.h"), os.path.join(ROOT, "include", "rptq_testing.h"),
+        os.path.join(ROOT, "include", "rptq_baseline.h"), src]
 
 
 def _stale(out: str, deps: list[str]) -> bool:

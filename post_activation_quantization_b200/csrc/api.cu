@@ -8,6 +8,7 @@
 #include <mutex>
 #include <unordered_map>
 
+#include "../../include/rptq_baseline.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -340,6 +341,32 @@ int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t 
     KvAttnArgs a{q, B, H, D, k_cache, v_cache, S_max, L, cluster_k, scale_k, zero_k, cluster_v,
                  scale_v, zero_v, g, bits, scale, out, d.err, (cudaStream_t)stream, d.max_smem};
     return cuda_status(launch_kv_attention(a));
+}
+
+int rptq_baseline_explicit_reorder_quant(const void *x, int dtype, int64_t T, int C,
+                                         const float *gamma, const float *beta, float eps,
+                                         const int32_t *R, const int32_t *col_cluster,
+                                         const float *scale, const int32_t *zero, int g, int bits,
+                                         float *y, float *y_reordered, uint8_t *codes,
+                                         rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (T < 0 || g <= 0 || g > C || !(eps >= 0.0f)) return RPTQ_ERR_INVALID_ARG;
+    if (!gamma || !beta || !R || !col_cluster || !scale || !zero) return RPTQ_ERR_INVALID_ARG;
+    if (T == 0) return RPTQ_OK;
+    if (!x || !y || !y_reordered || !codes) return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(y_reordered) || !aligned16(codes) || !aligned16(R) ||
+        !aligned16(col_cluster) || !aligned16(gamma) || !aligned16(beta))
+        return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if ((size_t)C * 8 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    XrArgs a{x, dtype, T, C, gamma, beta, eps, R, col_cluster, scale, zero, g, bits, y, y_reordered,
+             codes, d.err, (cudaStream_t)stream, d.num_sms};
+    return cuda_status(launch_explicit_reorder(a));
 }
 
 int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,

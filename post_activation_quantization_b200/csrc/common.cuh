@@ -161,6 +161,12 @@ __device__ __forceinline__ uint4 ldg_stream(const void *p)
     return v;
 }
 
+__device__ __forceinline__ float4 ldg_f4(const void *p)
+{
+    const uint4 v = ldg_stream(p);
+    return make_float4(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w));
+}
+
 __device__ __forceinline__ float fma_sat(float a, float b, float c)
 {
     float d;

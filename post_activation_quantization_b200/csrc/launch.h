@@ -115,6 +115,24 @@ struct KvAttnArgs {
     int max_smem;
 };
 
+struct XrArgs {
+    const void *x;
+    int dtype;
+    int64_t T;
+    int C;
+    const float *gamma, *beta;
+    float eps;
+    const int32_t *R, *col_cluster;
+    const float *scale;
+    const int32_t *zero;
+    int g, bits;
+    float *y, *yr;
+    uint8_t *codes;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+};
+
 struct DequantArgs {
     const uint8_t *codes;
     int layout;
@@ -156,6 +174,7 @@ cudaError_t launch_kv_calib(const KvCalibArgs &a);
 cudaError_t launch_kv_quant(const KvArgs &a);
 cudaError_t launch_dequant(const DequantArgs &a);
 cudaError_t launch_kv_append(const KvAppendArgs &a);
+cudaError_t launch_explicit_reorder(const XrArgs &a);
 cudaError_t launch_kv_attention(const KvAttnArgs &a);
 // largest number of cache positions one decode-attention call reads (its scores stay in shared
 // memory)

@@ -51,6 +51,9 @@ SIGNATURES = {
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
+    # include/rptq_baseline.h
+    "rptq_baseline_explicit_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P,
+                                                  _P]),
     # include/rptq_testing.h
     "rptq_testing_kv_quotient": (_I, [_P, _I64, _F, _P, _P]),
     "rptq_testing_kmeans_wait": (_I, [ctypes.c_ulonglong, _I]),
@@ -273,6 +276,27 @@ def rptq_kv_decode_attention(q, k_cache, v_cache, L: int, cluster_k, scale_k, ze
                                         _ptr(out), _stream(stream))
     _check(st, "rptq_kv_decode_attention")
     return out
+
+
+# ---------------------------------------------------------------------------------------------
+# Measurement baselines (include/rptq_baseline.h)
+def rptq_baseline_explicit_reorder_quant(x, gamma, beta, R, col_cluster, scale, zero, bits: int, eps: float = 1e-5,
+                                         y=None, y_reordered=None, codes=None, stream=None):
+    """The unfused LayerNorm -> explicit gather through R -> quantize pipeline (fp32
+    intermediates in HBM); returns (codes, y, y_reordered)."""
+    T, C = x.shape
+    if y is None:
+        y = torch.empty((T, C), dtype=torch.float32, device=x.device)
+    if y_reordered is None:
+        y_reordered = torch.empty((T, C), dtype=torch.float32, device=x.device)
+    if codes is None:
+        codes = torch.empty((T, C * bits // 8), dtype=torch.uint8, device=x.device)
+    st = lib().rptq_baseline_explicit_reorder_quant(_ptr(x), _DT[x.dtype], T, C, _ptr(gamma), _ptr(beta), eps,
+                                                    _ptr(R), _ptr(col_cluster), _ptr(scale), _ptr(zero),
+                                                    scale.numel(), bits, _ptr(y), _ptr(y_reordered), _ptr(codes),
+                                                    _stream(stream))
+    _check(st, "rptq_baseline_explicit_reorder_quant")
+    return codes, y, y_reordered
 
 
 # ---------------------------------------------------------------------------------------------

@@ -116,3 +116,10 @@ def bytes_kv_attention(B: int, H: int, L: int, D: int, bits: int) -> int:
     """Decode attention over L positions: read the packed K and V rows once, the fp32 query,
     write the fp32 output."""
     return 2 * B * H * L * D * bits // 8 + 2 * B * H * D * 4
+
+
+def bytes_explicit_reorder(T: int, C: int, dtype: str, bits: int) -> int:
+    """The unfused pipeline: read x, write the fp32 LayerNorm output, read it and write the fp32
+    reordered copy, read that and write the packed codes."""
+    n = T * C
+    return n * ESIZE[dtype] + 4 * n * 4 + n * bits // 8

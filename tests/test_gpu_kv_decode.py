@@ -4,11 +4,14 @@ packed caches, and decode attention reading those caches (codes dequantized in r
 Append: byte-exact against oracle.kv_append (the untouched positions of a cache pre-filled with
 random bytes must survive), and token-by-token appends reproduce the whole-cache quantization.
 Attention: against oracle.kv_decode_attention (fp64 on the same dequantized values), with a
-bar derived from the kernel's fp32 arithmetic: a row's dot product is 8 fused multiply-adds per
-lane and a log2(D/8)-level shuffle tree, so |d score| <= (8 + log2(D/8) + 2) u scale sum|q K|
-(u = 2^-24); a weight moves by at most p (2 max|d score| + the relative error of its exp and of
-the sums); the output is a fixed-order sum of ceil(L / (8 * 32/(D/8))) products per lane, a
-shuffle tree and 8 warp partials.  Everything is bounded by a multiple of sum_s p_s |V_s,d|."""
+bar derived from the kernel's fp32 arithmetic.  A lane owns CPL = min(32, D) channels; a row's
+score is two interleaved sums of CPL/2 fused multiply-adds of (q_d s_d scale) (q - z), one add,
+and a log2(D/CPL)-level shuffle tree, and q_d s_d scale and s (q - z) differ from the oracle's
+products by a rounding each, so |d score| <= (CPL/2 + 4 + log2(D/CPL)) u scale sum|q K|
+(u = 2^-24); a weight moves by at most p (2 max|d score| + the relative error of its exp and
+of the sums); the output is a fixed-order sum of ceil(L / (8 * rows per warp step)) products
+per lane, a shuffle tree, 8 warp partials and two final products.  Everything is bounded by a
+multiple of sum_s p_s |V_s,d|."""
 import math
 
 import numpy as np
@@ -98,14 +101,15 @@ def test_kv_append_rejects_positions_past_the_end():
 def _attn_bound(q, Kd, Vd, L, D, scale):
     """Per-output bound on |gpu - fp64| for the kernel's fp32 evaluation order (module docstring)."""
     q64, K, V = q.astype(np.float64), Kd[:, :, :L].astype(np.float64), Vd[:, :, :L].astype(np.float64)
-    lpp = D // 8
+    cpl = min(32, D)
+    lpp = D // cpl
     ppw = 32 // lpp
-    dscore = (8 + math.log2(lpp) + 2) * U * scale * np.einsum("bhd,bhsd->bhs", np.abs(q64), np.abs(K))
+    dscore = (cpl / 2 + 4 + math.log2(lpp)) * U * scale * np.einsum("bhd,bhsd->bhs", np.abs(q64), np.abs(K))
     sc = np.einsum("bhd,bhsd->bhs", q64, K) * scale
     p = np.exp(sc - sc.max(axis=2, keepdims=True))
     p /= p.sum(axis=2, keepdims=True)
     n_sum = math.ceil(L / 256) + 5 + 8
-    n_out = math.ceil(L / (8 * ppw)) + math.log2(ppw) + 8
+    n_out = math.ceil(L / (8 * ppw)) + math.log2(ppw) + 8 + 1 + 3
     rel = 2 * dscore.max(axis=2) + (n_sum + n_out + 8) * U
     mag = np.einsum("bhs,bhsd->bhd", p, np.abs(V))
     return 2 * rel[..., None] * mag + 1e-30
@@ -113,7 +117,8 @@ def _attn_bound(q, Kd, Vd, L, D, scale):
 
 @pytest.mark.parametrize("B,H,D,S_max,L,bits,scale", [
     (2, 4, 128, 300, 300, 3, 0.0), (2, 4, 128, 300, 37, 4, 0.0), (1, 3, 64, 50, 1, 3, 0.0),
-    (3, 2, 8, 20, 19, 4, 0.5), (1, 2, 256, 130, 129, 3, 0.0), (8, 96, 128, 512, 512, 3, 0.0)])
+    (3, 2, 8, 20, 19, 4, 0.5), (1, 2, 256, 130, 129, 3, 0.0), (8, 96, 128, 512, 512, 3, 0.0),
+    (2, 3, 16, 40, 33, 3, 0.0), (2, 3, 16, 40, 40, 4, 0.0), (1, 2, 32, 70, 70, 3, 0.0), (2, 2, 8, 12, 9, 3, 0.0)])
 def test_kv_decode_attention_matches_oracle(B, H, D, S_max, L, bits, scale):
     seed = 7 * B + H + D + L
     mk = synthetic.channel_model(H * D, seed, tag=1)
