@@ -240,6 +240,17 @@ def kv_dequant(packed, D, col_cluster, s, z, bits):
     return out
 
 
+def dynamic_params(x, gamma, beta, labels, g, bits, eps=1e-5):
+    """Dynamic (per-batch) cluster ranges ([Basics] section 1.1: a static range is fixed from
+    calibration data, a dynamic one is taken from the data being quantized; [RPTQ-art] text after
+    Fig. 2: one (s, z) per cluster of channels).  The clusters (labels) stay those of the offline
+    calibration; the per-channel max / min are those of LayerNorm(x) over this batch, and every
+    cluster's (s, z) follow from them exactly as in the calibration.  Definition written out: the
+    oracle's minmax_ln, then its cluster_params."""
+    mx, mn = minmax_ln(x, gamma, beta, eps)
+    return cluster_params(mx, mn, labels, g, bits)
+
+
 def kv_append(cache, new, s_begin, col_cluster, s, z, bits):
     """Decode-time append ([RPTQ-art] results paragraph: the K/V cache is quantized per cluster;
     closing paragraph: the cache dominates memory at large batch x sequence).  A copy of the
