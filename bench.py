@@ -76,6 +76,9 @@ def stage_list(w: W.Workload):
         st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
         # the unfused pipeline the fused kernel replaces (a measurement baseline, same results)
         st += [("explicit_reorder_baseline", W.bytes_explicit_reorder(w.T, w.C, w.dtype, w.bits), 3)]
+        # what dynamic (per-batch) cluster ranges add before the same fused kernel: the batch's
+        # LayerNorm statistics and the per-cluster (s, z) of the fixed clusters
+        st += [("dynamic_ranges", W.bytes_calib(w.T, w.C, w.dtype), 3)]
     if k:
         st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
     if a:
@@ -115,6 +118,9 @@ class Step:
             self.xr_y = torch.empty((w.T, w.C), dtype=torch.float32, device=device)
             self.xr_yr = torch.empty_like(self.xr_y)
             self.xr_codes = torch.empty_like(self.codes)
+            self.dmx, self.dmn = torch.empty_like(self.mx), torch.empty_like(self.mx)
+            self.dsc = torch.empty(w.g, dtype=torch.float32, device=device)
+            self.dz = torch.empty(w.g, dtype=torch.int32, device=device)
             self.xhat = torch.empty((w.T, w.C), dtype=dt, device=device)
         if self.kvw:
             k = self.kvw
@@ -207,6 +213,10 @@ class Step:
                                                    self.km["scale"], self.km["zero"], w.bits, eps=w.eps,
                                                    y=self.xr_y, y_reordered=self.xr_yr, codes=self.xr_codes)
             mark("explicit_reorder_baseline", 1)
+            mark("dynamic_ranges", 0)
+            r.rptq_calib_minmax(self.x, self.gamma, self.beta, w.eps, ch_max=self.dmx, ch_min=self.dmn)
+            r.rptq_cluster_params(self.dmx, self.dmn, self.km["labels"], w.g, w.bits, scale=self.dsc, zero=self.dz)
+            mark("dynamic_ranges", 1)
         if k:
             mark("kv_quant", 0)
             r.rptq_kv_quant(self.k, self.v, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],

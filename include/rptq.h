@@ -181,6 +181,22 @@ int rptq_kmeans_noalloc(const float *ch_max, const float *ch_min, int C, int g, 
                         rptq_stream_t stream);
 
 /*
+ * Per-cluster scale and zero point for FIXED clusters from per-channel statistics: the parameter
+ * step of rptq_kmeans alone.  With statistics of the batch being quantized (rptq_calib_minmax on
+ * it) this gives dynamic per-batch cluster ranges ([Basics] 1.1: static ranges come from
+ * calibration data, dynamic ones from the data at hand; [RPTQ-art] text after Fig. 2: one scale
+ * and zero point per cluster of channels); the clusters, R and col_cluster stay those of the
+ * offline calibration, and the codes follow with rptq_ln_reorder_quant.
+ *   ch_max, ch_min  fp32 [C];  labels  int32 [C] (the cluster of each channel, rptq_kmeans's
+ *   labels);  scale, zero  fp32 / int32 [g] outputs, computed exactly as rptq_kmeans does:
+ *   M_k = max of members' ch_max, m_k = min of members' ch_min, s_k = (M_k - m_k) / qmax,
+ *   z_k = rint(-m_k / s_k) (fp32 IEEE, half-to-even; M_k == m_k and empty clusters as there).
+ * A label outside [0, g) is reported in the device error word and the channel is skipped.
+ */
+int rptq_cluster_params(const float *ch_max, const float *ch_min, int C, const int32_t *labels,
+                        int g, int bits, float *scale, int32_t *zero, rptq_stream_t stream);
+
+/*
  * Reorder-fused LayerNorm with per-cluster quantization: the runtime activation path.
  * [RPTQ-art] text after Fig. 3 (the LayerNorm itself emits channels in cluster order, so no
  * reordered copy of x is ever stored); text after Fig. 2 (per-cluster s, z); [Houmo-art]

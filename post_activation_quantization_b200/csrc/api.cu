@@ -239,6 +239,20 @@ int rptq_kmeans(const float *ch_max, const float *ch_min, int C, int g, int iter
     return cuda_status(launch_kmeans(a));
 }
 
+int rptq_cluster_params(const float *ch_max, const float *ch_min, int C, const int32_t *labels,
+                        int g, int bits, float *scale, int32_t *zero, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (g <= 0 || g > C || g > RPTQ_MAX_CLUSTERS) return RPTQ_ERR_INVALID_ARG;
+    if (!ch_max || !ch_min || !labels || !scale || !zero) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    return cuda_status(launch_cluster_params(ch_max, ch_min, C, labels, g, bits, scale, zero, d.err,
+                                             (cudaStream_t)stream));
+}
+
 int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const float *gamma,
                           const float *beta, float eps, const int32_t *R,
                           const int32_t *col_cluster, const float *scale, const int32_t *zero,

@@ -709,6 +709,63 @@ __global__ void __launch_bounds__(KM_THREADS, 1)
     }
 }
 
+// ------------------------------------------------------------------------------------------
+// Per-cluster (s, z) for fixed clusters from per-channel statistics: the parameter step of the
+// calibration on its own, for dynamic (per-batch) ranges.  One CTA: the members' max / min are
+// folded per cluster with order-independent shared-memory atomics (exact), then s and z follow
+// with the same fp32 IEEE operations as in the calibration above.
+__global__ void __launch_bounds__(512)
+    cluster_params_kernel(const float *__restrict__ mx, const float *__restrict__ mn, int C,
+                          const int32_t *__restrict__ labels, int g, int bits, float *__restrict__ scale,
+                          int32_t *__restrict__ zero, int *err)
+{
+    __shared__ float cmx[RPTQ_MAX_CLUSTERS], cmn[RPTQ_MAX_CLUSTERS];
+    __shared__ int cnt[RPTQ_MAX_CLUSTERS];
+    for (int k = threadIdx.x; k < g; k += blockDim.x) {
+        cmx[k] = -INFINITY;
+        cmn[k] = INFINITY;
+        cnt[k] = 0;
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < C; c += blockDim.x) {
+        const int k = labels[c];
+        if (k < 0 || k >= g) {
+            raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+            continue;
+        }
+        atomic_max_f32(cmx + k, mx[c]);
+        atomic_min_f32(cmn + k, mn[c]);
+        atomicAdd(cnt + k, 1);
+    }
+    __syncthreads();
+    const float qmax = (float)((1 << bits) - 1);
+    for (int k = threadIdx.x; k < g; k += blockDim.x) {
+        if (cnt[k] == 0) {
+            scale[k] = 1.0f;
+            zero[k] = 0;
+            continue;
+        }
+        const float M = cmx[k], m = cmn[k];
+        float s;
+        if (M == m) {
+            float r = fmaxf(fabsf(m), fabsf(M));
+            if (r == 0.0f) r = 1.0f;
+            s = __fdiv_rn(r, qmax);
+        } else {
+            s = __fdiv_rn(__fsub_rn(M, m), qmax);
+        }
+        scale[k] = s;
+        zero[k] = (int32_t)rintf(__fdiv_rn(-m, s));
+    }
+}
+
+cudaError_t launch_cluster_params(const float *mx, const float *mn, int C, const int32_t *labels, int g, int bits,
+                                  float *scale, int32_t *zero, int *err, cudaStream_t stream)
+{
+    cluster_params_kernel<<<1, 512, 0, stream>>>(mx, mn, C, labels, g, bits, scale, zero, err);
+    return cudaGetLastError();
+}
+
 bool kmeans_supported(int C, int g, int max_smem)
 {
     return C >= 1 && C <= RPTQ_MAX_CHANNELS && g >= 1 && g <= C && kmeans_smem_bytes(C, g) <= (size_t)max_smem;

@@ -174,6 +174,8 @@ cudaError_t launch_kv_calib(const KvCalibArgs &a);
 cudaError_t launch_kv_quant(const KvArgs &a);
 cudaError_t launch_dequant(const DequantArgs &a);
 cudaError_t launch_kv_append(const KvAppendArgs &a);
+cudaError_t launch_cluster_params(const float *mx, const float *mn, int C, const int32_t *labels, int g, int bits,
+                                  float *scale, int32_t *zero, int *err, cudaStream_t stream);
 cudaError_t launch_explicit_reorder(const XrArgs &a);
 cudaError_t launch_kv_attention(const KvAttnArgs &a);
 // largest number of cache positions one decode-attention call reads (its scores stay in shared

@@ -49,6 +49,7 @@ SIGNATURES = {
     "rptq_ln_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_quant": (_I, [_P, _P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
+    "rptq_cluster_params": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
     # include/rptq_baseline.h
@@ -246,6 +247,18 @@ def rptq_dequant(codes: torch.Tensor, cluster, scale, zero, bits: int, out_dtype
                             _stream(stream))
     _check(st, "rptq_dequant")
     return out
+
+
+def rptq_cluster_params(ch_max, ch_min, labels, g: int, bits: int, scale=None, zero=None, stream=None):
+    """Per-cluster (s, z) of fixed clusters from per-channel statistics (dynamic ranges)."""
+    C = ch_max.numel()
+    if scale is None:
+        scale = torch.empty(g, dtype=torch.float32, device=ch_max.device)
+        zero = torch.empty(g, dtype=torch.int32, device=ch_max.device)
+    st = lib().rptq_cluster_params(_ptr(ch_max), _ptr(ch_min), C, _ptr(labels), g, bits, _ptr(scale), _ptr(zero),
+                                   _stream(stream))
+    _check(st, "rptq_cluster_params")
+    return scale, zero
 
 
 def rptq_kv_append(k_new, v_new, cluster_k, scale_k, zero_k, cluster_v, scale_v, zero_v, bits: int,
