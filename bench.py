@@ -430,7 +430,9 @@ def run_rptq(args):
             "headline_kernel": head,
             "mtokens_per_s": round(tokens * ws * args.steps / (head_ms * 1e-3) / 1e6, 3),
             "frac_of_measured_hbm": round(value / ws / hbm, 4),
-            "step": {"what": "every stage of the path once (calibration, KMeans, quantization, dequantization)",
+            "step": {"what": "every stage of the path once: calibration, KMeans, fused quantization, the "
+                             "explicit-reorder baseline, dynamic ranges, K/V quantization, dequantization, "
+                             "one decode step (append, attention)",
                      "ms": round(ms / args.steps, 4),
                      "gbs": round(pdist.sum_over_ranks(step_bytes * args.steps, dev) / (ms * 1e-3) / 1e9, 1),
                      "frac_of_measured_hbm": round(step_bytes * args.steps / (ms * 1e-3) / 1e9 / hbm, 4),

@@ -1,4 +1,4 @@
-"""The allocation-free KMeans entry point against the regular one.
+"""The allocation-free KMeans entry point against the regular one and against the CPU oracle.
 
 rptq_kmeans_noalloc exists for callers that cannot allocate device memory while running (a
 plugin whose host application owns all GPU memory, a serving loop that forbids cudaMalloc and
@@ -96,3 +96,20 @@ def test_noalloc_refuses_invalid_sizes():
     out = _outputs(C, 8)
     assert _call_c_abi(mx, mx, C + 1, 1, 3, out) == rptq.RPTQ_ERR_INVALID_ARG   # g > C
     assert _call_c_abi(mx, mx, 8, 1, 5, out) == rptq.RPTQ_ERR_UNSUPPORTED      # bits
+
+
+def test_noalloc_matches_the_oracle():
+    """Standing alone: the entry point's outputs against the oracle's calibration chain on the
+    same statistics (labels, R, offsets, s and z exact; centroids to 1e-6)."""
+    import oracle
+    C, g, iters, bits = 4096, 32, 20, 4
+    mx, mn = _stats(C, 21)
+    hmx, hmn = mx.cpu().numpy(), mn.cpu().numpy()
+    cal = oracle.calibrate(hmx, hmn, g, iters, bits)
+    out = _outputs(C, g)
+    assert _call_c_abi(mx, mn, g, iters, bits, out) == rptq.RPTQ_OK
+    torch.cuda.synchronize()
+    for k in ("labels", "R", "col_cluster", "offsets", "scale", "zero"):
+        assert np.array_equal(out[k].cpu().numpy(), cal[k]), k
+    np.testing.assert_allclose(out["centroids"].cpu().numpy(), cal["centroids"], rtol=1e-6, atol=1e-12)
+    assert rptq.rptq_device_error() == 0
