@@ -251,6 +251,42 @@ def dynamic_params(x, gamma, beta, labels, g, bits, eps=1e-5):
     return cluster_params(mx, mn, labels, g, bits)
 
 
+def quant_weights(W, bits=4):
+    """Per-output-channel asymmetric weight quantization ([Basics] section 1.4, per-channel
+    granularity; section 1.3, s = range / (2^b - 1), z = rint(-min / s)): row n of W [N, C] gets
+    its own (s_w, z_w) from its min and max, codes q = clamp(rint(w / s_w) + z_w, 0, qmax).
+    fp32 operations as in the activation quantizer.  Returns (q uint8 [N, C], s_w fp32 [N],
+    z_w int32 [N])."""
+    W = np.asarray(W, np.float32)
+    N, C = W.shape
+    q = np.empty((N, C), np.uint8)
+    sw = np.empty(N, np.float32)
+    zw = np.empty(N, np.int32)
+    for n in range(N):
+        # one cluster spanning the whole row: its range is the row's min and max
+        s1, z1 = cluster_params(np.array([W[n].max()], np.float32), np.array([W[n].min()], np.float32),
+                                np.zeros(1, np.int32), 1, bits)
+        sw[n], zw[n] = s1[0], z1[0]
+        q[n] = quantize(W[n:n + 1], np.zeros(C, np.int32), s1, z1, bits)[0]
+    return q, sw, zw
+
+
+def reordered_linear(codes, C, col_cluster, s, z, bits, R, qw, sw, zw):
+    """The linear layer after the reorder-fused LayerNorm ([RPTQ-art], Fig. 3 caption and the text
+    after it: the next layer's weights are permuted offline by the same reorder index, so the
+    layer consumes the activations in cluster order and its output is unchanged).  codes
+    [T, C*bits/8] are the packed cluster-ordered activation codes (column j in cluster
+    col_cluster[j]); qw [N, C] the 4-bit weight codes in the ORIGINAL channel order with
+    per-row (sw, zw).  Y[t, n] = sum_j s_k (q[t, j] - z_k) * sw[n] (qw[n, R[j]] - zw[n]),
+    k = col_cluster[j], in fp64.  Returns fp64 [T, N]."""
+    q = unpack(np.asarray(codes, np.uint8).reshape(-1, C * bits // 8), C, bits).astype(np.float64)
+    cc = np.asarray(col_cluster)
+    xa = (q - np.asarray(z, np.float64)[cc]) * np.asarray(s, np.float64)[cc]          # [T, C], cluster order
+    wd = (np.asarray(qw, np.float64) - np.asarray(zw, np.float64)[:, None]) * np.asarray(sw, np.float64)[:, None]
+    wr = wd[:, np.asarray(R)]                                                          # [N, C], permuted offline
+    return xa @ wr.T
+
+
 def kv_append(cache, new, s_begin, col_cluster, s, z, bits):
     """Decode-time append ([RPTQ-art] results paragraph: the K/V cache is quantized per cluster;
     closing paragraph: the cache dominates memory at large batch x sequence).  A copy of the
