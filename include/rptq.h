@@ -281,6 +281,50 @@ int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t 
                              int g, int bits, float scale, float *out, rptq_stream_t stream);
 
 /*
+ * Offline weight preparation for the linear layer that reads the reordered activations.
+ * [RPTQ-art] Fig. 3 caption and the text after it: the weights of the layer after the reordered
+ * LayerNorm are permuted offline by the same reorder index, so that the layer consumes the
+ * activations in cluster order and computes the same output; [Basics] sections 1.3 / 1.4: the
+ * weights are 4-bit codes with one (s_w, z_w) per output row.
+ *   w_codes   uint8 [N, C/2]: 4-bit weight codes in the ORIGINAL channel order (the packed
+ *             layout above, b = 4); w_scale fp32 [N], w_zero int32 [N]: row n's (s_w, z_w).
+ *   R, col_cluster, scale, zero, g: the activation calibration (rptq_kmeans's outputs).
+ *   w_prep    fp16 [N, C] (output): the prepared operand, in cluster order, with the folded
+ *             activation scale: B[n][j] = RN16(RN32(s_k * (w[n][R[j]] - z_w[n])) / lambda[n]),
+ *             k = col_cluster[j], its columns interleaved inside each group of 8 as the GEMM
+ *             decodes them (stored column 8m + 2i holds j = 8m + i, 8m + 2i + 1 holds
+ *             j = 8m + 4 + i, i < 4).
+ *   w_bias    fp32 [N] (output): sum_j z_k B[n][j] (summed in fp64, rounded once).
+ *   w_lambda  fp32 [N] (output): the power of two that puts max_j |B[n][j]| in [2^14, 2^15)
+ *             (1 for an all-zero row).
+ * C a multiple of 64 in [64, RPTQ_MAX_CHANNELS], N >= 1, 1 <= g <= C.  An R entry outside
+ * [0, C) or a cluster id outside [0, g) sets the device error word.
+ */
+int rptq_linear_prepare(const uint8_t *w_codes, const float *w_scale, const int32_t *w_zero, int N,
+                        int C, const int32_t *R, const int32_t *col_cluster, const float *scale,
+                        const int32_t *zero, int g, void *w_prep, float *w_bias, float *w_lambda,
+                        rptq_stream_t stream);
+
+/*
+ * The reordered low-bit linear layer (W4A4 / W4A3, [RPTQ-art] results paragraph) on the tensor
+ * cores: for token t and output n,
+ *   out[t][n] = sum_j s_k (q[t][j] - z_k) * s_w[n] (w[n][R[j]] - z_w[n])
+ *             = s_w[n] lambda[n] (sum_j q[t][j] B[n][j] - w_bias[n]),
+ * with q the packed cluster-ordered activation codes (rptq_ln_reorder_quant's output).
+ *   codes     uint8 [T, C*bits/8], bits 3 or 4.
+ *   w_prep, w_bias, w_lambda: rptq_linear_prepare's outputs for this calibration; w_scale the
+ *             weights' per-row scales.
+ *   out       fp32 [T, N].
+ * The codes go to the tensor core as exact fp16 integers and the products are accumulated in
+ * fp32 (tcgen05.mma kind::f16, 128 x 256 output tiles).  C a multiple of 64 in
+ * [64, RPTQ_MAX_CHANNELS], N in [1, 2^24].  T == 0 is valid: nothing is launched.  A bounded
+ * wait that runs out sets RPTQ_DEVERR_TIMEOUT (the output is then undefined).
+ */
+int rptq_reordered_linear(const uint8_t *codes, int64_t T, int C, int bits, const void *w_prep,
+                          const float *w_bias, const float *w_lambda, const float *w_scale, int N,
+                          float *out, rptq_stream_t stream);
+
+/*
  * Dequantization, [Basics] section 1.3: value = s_k * (q - z_k), computed in fp32 (one
  * rounding) and rounded to out_dtype.
  *   layout RPTQ_LAYOUT_ROWS: codes [n0, n1*bits/8] with n0 = rows, n1 = C; cluster[j] is the

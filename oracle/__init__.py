@@ -287,6 +287,42 @@ def reordered_linear(codes, C, col_cluster, s, z, bits, R, qw, sw, zw):
     return xa @ wr.T
 
 
+def linear_fp16_operand(qw, sw, zw, R, col_cluster, s, z):
+    """The fp16 weight operand with which the library computes reordered_linear (a design reading,
+    not a step of the pages: [RPTQ-art] Fig. 3 text permutes the weights offline; folding the
+    per-cluster activation scale into them leaves only the integer codes q on the activation
+    side).  For output row n and cluster-order column j (k = col_cluster[j]):
+        b[n][j]  = RN32(s_k * (qw[n][R[j]] - zw[n]))            one fp32 product
+        lam[n]   = 2^(e - 14) with max_j |b[n][j]| in [2^e, 2^(e+1))  (1 for an all-zero row)
+        B[n][j]  = RN16(b[n][j] / lam[n])                        the division is exact
+        bz[n]    = sum_j z_k B[n][j]                             fp64, rounded to fp32 once
+    so that reordered_linear = sw[n] lam[n] (q @ B^T - bz) up to the fp16 rounding of B.
+    Returns (B fp16 [N, C] in cluster order, bz fp32 [N], lam fp32 [N])."""
+    qw = np.asarray(qw)
+    N, C = qw.shape
+    cc = np.asarray(col_cluster)
+    s32 = _f32(s)
+    B = np.empty((N, C), np.float16)
+    bz = np.empty(N, np.float32)
+    lam = np.empty(N, np.float32)
+    for n in range(N):
+        d = (qw[n, np.asarray(R)].astype(np.int64) - int(zw[n])).astype(np.float32)
+        b = (s32[cc] * d).astype(np.float32)                      # numpy fp32 multiply: RN
+        m = float(np.abs(b).max())
+        if m > 0.0:
+            e = int(np.floor(np.log2(m)))
+            if 2.0 ** e > m:                                       # guard log2's rounding
+                e -= 1
+            elif 2.0 ** (e + 1) <= m:
+                e += 1
+            lam[n] = np.float32(2.0 ** (e - 14))
+        else:
+            lam[n] = np.float32(1.0)
+        B[n] = (b.astype(np.float64) / float(lam[n])).astype(np.float16)   # RN to fp16
+        bz[n] = np.float32(np.sum(np.asarray(z, np.float64)[cc] * B[n].astype(np.float64)))
+    return B, bz, lam
+
+
 def kv_append(cache, new, s_begin, col_cluster, s, z, bits):
     """Decode-time append ([RPTQ-art] results paragraph: the K/V cache is quantized per cluster;
     closing paragraph: the cache dominates memory at large batch x sequence).  A copy of the

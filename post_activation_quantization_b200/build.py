@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "librptq.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["api.cu", "calib.cu", "kmeans.cu", "ln_quant.cu", "kv_quant.cu", "dequant.cu", "kv_attention.cu", "explicit_reorder.cu"]
+SOURCES = ["api.cu", "calib.cu", "kmeans.cu", "ln_quant.cu", "kv_quant.cu", "dequant.cu", "kv_attention.cu", "explicit_reorder.cu", "linear.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

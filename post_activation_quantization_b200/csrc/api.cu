@@ -383,6 +383,44 @@ int rptq_baseline_explicit_reorder_quant(const void *x, int dtype, int64_t T, in
     return cuda_status(launch_explicit_reorder(a));
 }
 
+int rptq_linear_prepare(const uint8_t *w_codes, const float *w_scale, const int32_t *w_zero, int N,
+                        int C, const int32_t *R, const int32_t *col_cluster, const float *scale,
+                        const int32_t *zero, int g, void *w_prep, float *w_bias, float *w_lambda,
+                        rptq_stream_t stream)
+{
+    if (C < 64 || C % 64 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (N < 1 || g < 1 || g > C) return RPTQ_ERR_INVALID_ARG;
+    if (!w_codes || !w_scale || !w_zero || !R || !col_cluster || !scale || !zero || !w_prep || !w_bias ||
+        !w_lambda)
+        return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(w_prep)) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    LinPrepArgs a{w_codes, w_scale, w_zero, R, col_cluster, scale, zero, g, C, N,
+                  static_cast<__half *>(w_prep), w_bias, w_lambda, d.err, (cudaStream_t)stream};
+    return cuda_status(launch_linear_prepare(a));
+}
+
+int rptq_reordered_linear(const uint8_t *codes, int64_t T, int C, int bits, const void *w_prep,
+                          const float *w_bias, const float *w_lambda, const float *w_scale, int N,
+                          float *out, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C < 64 || C % 64 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (T < 0 || N < 1 || N > (1 << 24)) return RPTQ_ERR_INVALID_ARG;
+    if (!w_prep || !w_bias || !w_lambda || !w_scale || !aligned16(w_prep)) return RPTQ_ERR_INVALID_ARG;
+    if (T == 0) return RPTQ_OK;
+    if (!codes || !out || !aligned16(codes) || !aligned16(out)) return RPTQ_ERR_INVALID_ARG;
+    if ((T + 127) / 128 > 0x7fffffffLL) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    LinArgs a{codes, T, C, bits, static_cast<const __half *>(w_prep), w_bias, w_lambda, w_scale, N, out,
+              d.err, (cudaStream_t)stream};
+    return cuda_status(launch_reordered_linear(a));
+}
+
 int rptq_dequant(const uint8_t *codes, int layout, int64_t n0, int n1, int64_t S, int D,
                  const int32_t *cluster, const float *scale, const int32_t *zero, int g,
                  int bits, void *out, int out_dtype, rptq_stream_t stream)

@@ -1,6 +1,7 @@
 // launch.h -- argument bundles and host launchers shared by api.cu and the kernel files.
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -133,6 +134,32 @@ struct XrArgs {
     int num_sms;
 };
 
+struct LinPrepArgs {
+    const uint8_t *qw;  // [N, C/2] 4-bit weight codes, original channel order, low nibble first
+    const float *sw;
+    const int32_t *zw;
+    const int32_t *R, *col_cluster;
+    const float *scale;
+    const int32_t *zero;
+    int g, C, N;
+    __half *B;  // [N, C] prepared fp16 weights
+    float *bz, *lam;
+    int *err;
+    cudaStream_t stream;
+};
+
+struct LinArgs {
+    const uint8_t *codes;  // [T, C*bits/8]
+    int64_t T;
+    int C, bits;
+    const __half *B;
+    const float *bz, *lam, *sw;
+    int N;
+    float *Y;  // [T, N] fp32
+    int *err;
+    cudaStream_t stream;
+};
+
 struct DequantArgs {
     const uint8_t *codes;
     int layout;
@@ -178,6 +205,8 @@ cudaError_t launch_cluster_params(const float *mx, const float *mn, int C, const
                                   float *scale, int32_t *zero, int *err, cudaStream_t stream);
 cudaError_t launch_explicit_reorder(const XrArgs &a);
 cudaError_t launch_kv_attention(const KvAttnArgs &a);
+cudaError_t launch_linear_prepare(const LinPrepArgs &a);
+cudaError_t launch_reordered_linear(const LinArgs &a);
 // largest number of cache positions one decode-attention call reads (its scores stay in shared
 // memory)
 constexpr int64_t KV_ATTN_MAX_L = 16384;

@@ -52,6 +52,8 @@ SIGNATURES = {
     "rptq_cluster_params": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
+    "rptq_linear_prepare": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
+    "rptq_reordered_linear": (_I, [_P, _I64, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
     # include/rptq_baseline.h
     "rptq_baseline_explicit_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P,
                                                   _P]),
@@ -288,6 +290,39 @@ def rptq_kv_decode_attention(q, k_cache, v_cache, L: int, cluster_k, scale_k, ze
                                         _ptr(scale_v), _ptr(zero_v), scale_k.numel(), bits, float(scale),
                                         _ptr(out), _stream(stream))
     _check(st, "rptq_kv_decode_attention")
+    return out
+
+
+def rptq_linear_prepare(w_codes, w_scale, w_zero, R, col_cluster, scale, zero, w_prep=None, w_bias=None,
+                        w_lambda=None, stream=None):
+    """Offline operand of the reordered linear layer from 4-bit weight codes w_codes [N, C/2]
+    (original channel order) and the activation calibration; returns (w_prep fp16 [N, C],
+    w_bias fp32 [N], w_lambda fp32 [N])."""
+    N = w_codes.shape[0]
+    C = R.numel()
+    dev = w_codes.device
+    if w_prep is None:
+        w_prep = torch.empty((N, C), dtype=torch.float16, device=dev)
+    if w_bias is None:
+        w_bias = torch.empty(N, dtype=torch.float32, device=dev)
+    if w_lambda is None:
+        w_lambda = torch.empty(N, dtype=torch.float32, device=dev)
+    st = lib().rptq_linear_prepare(_ptr(w_codes), _ptr(w_scale), _ptr(w_zero), N, C, _ptr(R), _ptr(col_cluster),
+                                   _ptr(scale), _ptr(zero), scale.numel(), _ptr(w_prep), _ptr(w_bias),
+                                   _ptr(w_lambda), _stream(stream))
+    _check(st, "rptq_linear_prepare")
+    return w_prep, w_bias, w_lambda
+
+
+def rptq_reordered_linear(codes, C: int, bits: int, w_prep, w_bias, w_lambda, w_scale, out=None, stream=None):
+    """out [T, N] fp32 = the linear layer applied to the packed cluster-ordered codes [T, C*bits/8]."""
+    T = codes.shape[0]
+    N = w_prep.shape[0]
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.float32, device=codes.device)
+    st = lib().rptq_reordered_linear(_ptr(codes), T, C, bits, _ptr(w_prep), _ptr(w_bias), _ptr(w_lambda),
+                                     _ptr(w_scale), N, _ptr(out), _stream(stream))
+    _check(st, "rptq_reordered_linear")
     return out
 
 

@@ -8,7 +8,8 @@ centre + hw) independently over tokens.  floor(p * C) "outlier" channels, picked
 permutation, have both centre and half-width multiplied by a factor (x100 or x200).  The
 channel draw is the "model": the calibration batch and the runtime batch of one model share
 it and differ only in their element draws.  LayerNorm gamma ~ U(0.5, 1.5) and
-beta ~ N(0, 0.1) (standard deviation 0.1).
+beta ~ N(0, 0.1) (standard deviation 0.1).  Linear-layer weights (no trained weights exist
+here) are W[n, c] ~ N(0, 1/C), the usual fan-in scaling.
 
 Every stream has its own derived seed, so any tensor can be regenerated alone.  Generation
 runs on the requested device with torch's generator for that device; CPU and CUDA streams
@@ -21,7 +22,7 @@ from dataclasses import dataclass
 import torch
 
 # sub-stream identifiers (mixed into the seed)
-_S_CHANNEL, _S_OUTLIER, _S_LN, _S_X, _S_CALIB, _S_K, _S_V = range(7)
+_S_CHANNEL, _S_OUTLIER, _S_LN, _S_X, _S_CALIB, _S_K, _S_V, _S_W = range(8)
 
 _DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
@@ -97,3 +98,10 @@ def kv_cache(B: int, H: int, S: int, D: int, model: ChannelModel, seed: int, whi
     _fill_rows(out.view(B * S, H * D), model, g, chunk_rows)
     # tokens were drawn as rows of H*D channels; lay them out as [B, H, S, D]
     return out.view(B, S, H, D).permute(0, 2, 1, 3).contiguous()
+
+
+def weights(N: int, C: int, seed: int) -> torch.Tensor:
+    """Synthetic weights [N, C] of the linear layer that reads the activations (original channel
+    order), W ~ N(0, 1/C); fp32 on CPU."""
+    g = _gen(seed, _S_W, "cpu")
+    return (torch.randn((N, C), generator=g, dtype=torch.float32) * (1.0 / C) ** 0.5).contiguous()

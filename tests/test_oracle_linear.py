@@ -63,3 +63,60 @@ def test_weight_quantizer_bound_and_ends():
     deq = (q.astype(np.float64) - zw[:, None]) * sw[:, None]
     assert (np.abs(deq - W) <= sw[:, None] / 2 * (1 + 1e-6)).all()
     assert (q[np.arange(7), W.argmin(1)] == 0).all() and (q[np.arange(7), W.argmax(1)] == 15).all()
+
+
+def _calibrated_case(C=128, T=12, N=7, g=6, bits=4, seed=5):
+    m = synthetic.channel_model(C, seed)
+    gamma, beta = synthetic.ln_params(C, seed)
+    x = oracle._f32(synthetic.activations(T, m, seed, dtype="f32"))
+    mx, mn = oracle.minmax_ln(x, gamma, beta)
+    cal = oracle.calibrate(mx, mn, g, 10, bits)
+    codes, _, _ = oracle.ln_reorder_quant(x, gamma, beta, cal["R"], cal["col_cluster"], cal["scale"], cal["zero"], bits)
+    W = np.random.default_rng(seed + 1).standard_normal((N, C)).astype(np.float32)
+    qw, sw, zw = oracle.quant_weights(W, 4)
+    return cal, codes, qw, sw, zw
+
+
+def test_fp16_operand_range_and_rounding():
+    """Each row's largest |B| lies in [2^14, 2^15) (lam a power of two), and B lam is within
+    fp16's half-ulp bound 2^-11 (relative) of the fp32 product s_k (qw - zw)."""
+    cal, _, qw, sw, zw = _calibrated_case()
+    B, bz, lam = oracle.linear_fp16_operand(qw, sw, zw, cal["R"], cal["col_cluster"], cal["scale"], cal["zero"])
+    cc = cal["col_cluster"]
+    for n in range(B.shape[0]):
+        assert np.frexp(lam[n])[0] == 0.5  # a power of two
+        top = np.abs(B[n].astype(np.float64)).max()
+        assert 2.0 ** 14 <= top < 2.0 ** 15
+        b = cal["scale"][cc].astype(np.float64) * (qw[n, cal["R"]].astype(np.float64) - zw[n])
+        err = np.abs(B[n].astype(np.float64) * lam[n] - b)
+        assert np.all(err <= 2.0 ** -11 * np.abs(b) * (1 + 2.0 ** -20) + 1e-30)
+        assert np.isclose(bz[n], np.sum(cal["zero"][cc] * B[n].astype(np.float64)), rtol=2.0 ** -23, atol=0)
+
+
+def test_fp16_operand_reproduces_the_layer():
+    """sw lam (q B^T - bz) equals the fp64 layer within the bound that B's rounding allows, and a
+    column taken in the original order instead of the cluster order breaks it."""
+    bits = 4
+    cal, codes, qw, sw, zw = _calibrated_case(bits=bits)
+    cc, R = cal["col_cluster"], cal["R"]
+    B, bz, lam = oracle.linear_fp16_operand(qw, sw, zw, R, cc, cal["scale"], cal["zero"])
+    Y = oracle.reordered_linear(codes, 128, cc, cal["scale"], cal["zero"], bits, R, qw, sw, zw)
+    q = oracle.unpack(codes, 128, bits).astype(np.float64)
+    Yb = (q @ B.astype(np.float64).T - bz.astype(np.float64)) * (sw.astype(np.float64) * lam)[None, :]
+    b = cal["scale"][cc].astype(np.float64)[None, :] * (qw[:, R].astype(np.float64) - zw[:, None])
+    A = np.abs(q - cal["zero"][cc][None, :])
+    bound = sw[None, :] * (2.0 ** -11 * (A @ np.abs(b).T)) + 2.0 ** -20 * np.abs(Y) + 1e-12
+    assert np.all(np.abs(Yb - Y) <= bound)
+    Bn, bzn, lamn = oracle.linear_fp16_operand(qw, sw, zw, np.arange(128, dtype=np.int32), cc, cal["scale"],
+                                               cal["zero"])
+    Ybad = (q @ Bn.astype(np.float64).T - bzn) * (sw.astype(np.float64) * lamn)[None, :]
+    assert not np.all(np.abs(Ybad - Y) <= bound)
+
+
+def test_fp16_operand_zero_row():
+    """A weight row whose codes all equal its zero point gives B = 0, bz = 0 and lam = 1."""
+    qw = np.full((1, 16), 5, np.uint8)
+    B, bz, lam = oracle.linear_fp16_operand(qw, np.array([0.1], np.float32), np.array([5], np.int32),
+                                            np.arange(16, dtype=np.int32), np.zeros(16, np.int32),
+                                            np.array([0.3], np.float32), np.array([2], np.int32))
+    assert not B.any() and bz[0] == 0 and lam[0] == 1
