@@ -5,6 +5,8 @@ A step is one pass of the whole path over one synthetic batch of the workload:
   1. calibration statistics of LayerNorm(x) over the calibration batch   (rptq_calib_minmax)
   2. KMeans -> reorder index R and per-cluster (s, z)                    (rptq_kmeans)
   3. reorder-fused LayerNorm + per-cluster quantization of the batch      (rptq_ln_reorder_quant)
+  3a. the explicit-reorder baseline, dynamic ranges, and the reordered linear layer on one
+      2048-token micro-batch of the codes  (rptq_baseline_..., rptq_linear_prepare, rptq_reordered_linear)
   4. K/V calibration statistics, KMeans for K and for V                   (rptq_kv_calib_minmax, rptq_kmeans)
   5. K/V cache quantization                                               (rptq_kv_quant)
   6. dequantization of the activation codes and of the K/V codes         (rptq_dequant)
@@ -57,9 +59,23 @@ def peaks():
     return HBM_FALLBACK_GBS, "fallback"
 
 
+def tensor_peak() -> float:
+    """Measured dense bf16 GEMM TFLOP/s (burst), else the pool's earlier measurement."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
 def has_act(w: W.Workload) -> bool:
     """Whether the workload carries the activation path (the K/V-only workload does not)."""
     return w.T > 0 and w.C > 0
+
+
+def stage_flops(w: W.Workload):
+    """Stages bound by the tensor cores: name -> operations per call."""
+    return {"reordered_linear": W.flops_linear(*W.linear_shape(w))} if has_act(w) else {}
 
 
 def stage_list(w: W.Workload):
@@ -79,6 +95,10 @@ def stage_list(w: W.Workload):
         # what dynamic (per-batch) cluster ranges add before the same fused kernel: the batch's
         # LayerNorm statistics and the per-cluster (s, z) of the fixed clusters
         st += [("dynamic_ranges", W.bytes_calib(w.T, w.C, w.dtype), 3)]
+        # the layer after the LayerNorm: its weights re-prepared for this calibration's R and
+        # (s, z), then one micro-batch of the codes through it (tensor cores; FLOPS below)
+        Tl, C, N = W.linear_shape(w)
+        st += [("linear_prepare", W.bytes_linear_prepare(N, C), 1), ("reordered_linear", 0, 1)]
     if k:
         st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
     if a:
@@ -122,6 +142,13 @@ class Step:
             self.dsc = torch.empty(w.g, dtype=torch.float32, device=device)
             self.dz = torch.empty(w.g, dtype=torch.int32, device=device)
             self.xhat = torch.empty((w.T, w.C), dtype=dt, device=device)
+            Tl, _, N = W.linear_shape(w)
+            self.lin_T = Tl
+            self.wq, self.wsc, self.wz = synthetic.weight_codes(N, w.C, w.seed, device=device)
+            self.wprep = torch.empty((N, w.C), dtype=torch.float16, device=device)
+            self.wbias = torch.empty(N, dtype=torch.float32, device=device)
+            self.wlam = torch.empty(N, dtype=torch.float32, device=device)
+            self.ylin = torch.empty((Tl, N), dtype=torch.float32, device=device)
         if self.kvw:
             k = self.kvw
             mk = synthetic.channel_model(k.channels, w.seed, k.outlier_frac, k.outlier_factor, tag=1)
@@ -217,6 +244,14 @@ class Step:
             r.rptq_calib_minmax(self.x, self.gamma, self.beta, w.eps, ch_max=self.dmx, ch_min=self.dmn)
             r.rptq_cluster_params(self.dmx, self.dmn, self.km["labels"], w.g, w.bits, scale=self.dsc, zero=self.dz)
             mark("dynamic_ranges", 1)
+            mark("linear_prepare", 0)
+            r.rptq_linear_prepare(self.wq, self.wz, self.km["R"], self.km["col_cluster"], self.km["scale"],
+                                  self.km["zero"], w_prep=self.wprep, w_bias=self.wbias, w_lambda=self.wlam)
+            mark("linear_prepare", 1)
+            mark("reordered_linear", 0)
+            r.rptq_reordered_linear(self.codes[:self.lin_T], w.C, w.bits, self.wprep, self.wbias, self.wlam, self.wsc,
+                                    out=self.ylin)
+            mark("reordered_linear", 1)
         if k:
             mark("kv_quant", 0)
             r.rptq_kv_quant(self.k, self.v, self.kmk["labels"], self.kmk["scale"], self.kmk["zero"],
@@ -392,6 +427,8 @@ def run_rptq(args):
     assert rptq.rptq_device_error() == 0, "device error word set during the timed steps"
 
     hbm, peak_kind = peaks()
+    tpeak = tensor_peak()
+    flops = stage_flops(w)
     kern = {}
     for n, b, launches in stages:
         per = [ev[n][i][0].elapsed_time(ev[n][i][1]) for i in range(args.steps)]
@@ -400,6 +437,11 @@ def run_rptq(args):
         if b:
             kern[n]["gbs"] = round(b / (mean_ms * 1e-3) / 1e9, 1)
             kern[n]["frac_of_measured_hbm"] = round(b / (mean_ms * 1e-3) / 1e9 / hbm, 4)
+        if n in flops:
+            # fp16 operands: the measured bf16 GEMM peak (same nominal tensor rate), burst figure
+            kern[n]["flops_per_call"] = flops[n]
+            kern[n]["tflops"] = round(flops[n] / (mean_ms * 1e-3) / 1e12, 1)
+            kern[n]["frac_of_measured_tensor_peak"] = round(flops[n] / (mean_ms * 1e-3) / 1e12 / tpeak, 4)
     # the headline: the metric's own kernel, its device time summed over the timed steps (the
     # slowest rank's), its bytes summed over ranks
     head = headline_stage(w)
@@ -431,7 +473,8 @@ def run_rptq(args):
             "mtokens_per_s": round(tokens * ws * args.steps / (head_ms * 1e-3) / 1e6, 3),
             "frac_of_measured_hbm": round(value / ws / hbm, 4),
             "step": {"what": "every stage of the path once: calibration, KMeans, fused quantization, the "
-                             "explicit-reorder baseline, dynamic ranges, K/V quantization, dequantization, "
+                             "explicit-reorder baseline, dynamic ranges, the reordered linear layer (weight "
+                             "preparation, one 2048-token micro-batch), K/V quantization, dequantization, "
                              "one decode step (append, attention)",
                      "ms": round(ms / args.steps, 4),
                      "gbs": round(pdist.sum_over_ranks(step_bytes * args.steps, dev) / (ms * 1e-3) / 1e9, 1),

@@ -287,7 +287,8 @@ int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t 
  * activations in cluster order and computes the same output; [Basics] sections 1.3 / 1.4: the
  * weights are 4-bit codes with one (s_w, z_w) per output row.
  *   w_codes   uint8 [N, C/2]: 4-bit weight codes in the ORIGINAL channel order (the packed
- *             layout above, b = 4); w_scale fp32 [N], w_zero int32 [N]: row n's (s_w, z_w).
+ *             layout above, b = 4); w_zero int32 [N]: row n's zero point z_w (its scale s_w is
+ *             applied by rptq_reordered_linear and is not needed here).
  *   R, col_cluster, scale, zero, g: the activation calibration (rptq_kmeans's outputs).
  *   w_prep    fp16 [N, C] (output): the prepared operand, in cluster order, with the folded
  *             activation scale: B[n][j] = RN16(RN32(s_k * (w[n][R[j]] - z_w[n])) / lambda[n]),
@@ -297,11 +298,12 @@ int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t 
  *   w_bias    fp32 [N] (output): sum_j z_k B[n][j] (summed in fp64, rounded once).
  *   w_lambda  fp32 [N] (output): the power of two that puts max_j |B[n][j]| in [2^14, 2^15)
  *             (1 for an all-zero row).
- * C a multiple of 64 in [64, RPTQ_MAX_CHANNELS], N >= 1, 1 <= g <= C.  An R entry outside
- * [0, C) or a cluster id outside [0, g) sets the device error word.
+ * C a multiple of 64 in [64, RPTQ_MAX_CHANNELS], N >= 1, 1 <= g <= C; w_codes and w_prep
+ * 16-byte aligned.  An R entry outside [0, C) or a cluster id outside [0, g) sets the device
+ * error word (entry 0 / cluster 0 is used instead).
  */
-int rptq_linear_prepare(const uint8_t *w_codes, const float *w_scale, const int32_t *w_zero, int N,
-                        int C, const int32_t *R, const int32_t *col_cluster, const float *scale,
+int rptq_linear_prepare(const uint8_t *w_codes, const int32_t *w_zero, int N, int C,
+                        const int32_t *R, const int32_t *col_cluster, const float *scale,
                         const int32_t *zero, int g, void *w_prep, float *w_bias, float *w_lambda,
                         rptq_stream_t stream);
 

@@ -383,22 +383,23 @@ int rptq_baseline_explicit_reorder_quant(const void *x, int dtype, int64_t T, in
     return cuda_status(launch_explicit_reorder(a));
 }
 
-int rptq_linear_prepare(const uint8_t *w_codes, const float *w_scale, const int32_t *w_zero, int N,
-                        int C, const int32_t *R, const int32_t *col_cluster, const float *scale,
+int rptq_linear_prepare(const uint8_t *w_codes, const int32_t *w_zero, int N, int C,
+                        const int32_t *R, const int32_t *col_cluster, const float *scale,
                         const int32_t *zero, int g, void *w_prep, float *w_bias, float *w_lambda,
                         rptq_stream_t stream)
 {
     if (C < 64 || C % 64 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
     if (N < 1 || g < 1 || g > C) return RPTQ_ERR_INVALID_ARG;
-    if (!w_codes || !w_scale || !w_zero || !R || !col_cluster || !scale || !zero || !w_prep || !w_bias ||
+    if (!w_codes || !w_zero || !R || !col_cluster || !scale || !zero || !w_prep || !w_bias ||
         !w_lambda)
         return RPTQ_ERR_INVALID_ARG;
-    if (!aligned16(w_prep)) return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(w_prep) || !aligned16(w_codes)) return RPTQ_ERR_INVALID_ARG;
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
-    LinPrepArgs a{w_codes, w_scale, w_zero, R, col_cluster, scale, zero, g, C, N,
-                  static_cast<__half *>(w_prep), w_bias, w_lambda, d.err, (cudaStream_t)stream};
+    if ((size_t)C * 8 + (size_t)g * 16 + (size_t)C / 2 + 32 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    LinPrepArgs a{w_codes, w_zero, R, col_cluster, scale, zero, g, C, N,
+                  static_cast<__half *>(w_prep), w_bias, w_lambda, d.err, (cudaStream_t)stream, d.num_sms};
     return cuda_status(launch_linear_prepare(a));
 }
 

@@ -136,7 +136,6 @@ struct XrArgs {
 
 struct LinPrepArgs {
     const uint8_t *qw;  // [N, C/2] 4-bit weight codes, original channel order, low nibble first
-    const float *sw;
     const int32_t *zw;
     const int32_t *R, *col_cluster;
     const float *scale;
@@ -146,6 +145,7 @@ struct LinPrepArgs {
     float *bz, *lam;
     int *err;
     cudaStream_t stream;
+    int num_sms;
 };
 
 struct LinArgs {

@@ -49,13 +49,13 @@ __device__ __forceinline__ void tc_dealloc(uint32_t taddr, uint32_t cols)
 {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
 }
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, fp16 inputs, fp32 accumulator
-__device__ __forceinline__ void tc_mma_f16(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, fp16 inputs, fp32 accumulator
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d, uint32_t a, uint64_t bdesc, uint32_t idesc, uint32_t acc)
 {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d),
+        "r"(a), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
 // arrive once on `bar` when every tcgen05.mma this thread issued so far has completed
@@ -77,6 +77,21 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&v)[32])
         : "memory");
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// 32 consecutive 32-bit columns of the calling thread's tensor-memory lane <- v (asynchronous:
+// tc_wait_st before anything that must see them)
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor of a K-major operand tile whose rows are 128 bytes (64 fp16)
 // in the 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r mod 8); groups of 8 rows
@@ -103,82 +118,153 @@ __host__ __device__ constexpr uint32_t f16_idesc(int M, int N)
 //     j = 8*(js/8) + (js even ? (js%8)/2 : 4 + (js%8)/2).
 __host__ __device__ __forceinline__ int lin_column(int js) { return (js & ~7) | ((js & 1) << 2) | ((js >> 1) & 3); }
 
-// ---- offline preparation: one CTA per output row n -----------------------------------------
-__global__ void __launch_bounds__(256)
-    linear_prepare_kernel(const uint8_t *__restrict__ qw, const float *__restrict__ sw, const int32_t *__restrict__ zw,
-                          const int32_t *__restrict__ R, const int32_t *__restrict__ col_cluster,
-                          const float *__restrict__ scale, const int32_t *__restrict__ zero, int g, int C, int N,
-                          __half *__restrict__ B, float *__restrict__ bz, float *__restrict__ lam, int *err)
+// ---- offline preparation ----------------------------------------------------------------------
+// Persistent CTAs over the output rows.  Each CTA first builds, in shared memory, the table of
+// stored column js -> (R[j] | k(j) << 16), j = lin_column(js), k = col_cluster[j] (range-checked
+// once), and the per-cluster s_k and z_k (the latter as double); then per row n: the row's packed
+// codes are staged in shared memory (16-byte loads), a first pass computes b[n][js] into shared
+// memory and max |b|, a second scales by the exact power of two 1 / lam[n], rounds pairs to fp16,
+// writes B in 16-byte stores (one group of 8 stored columns per thread and step) and sums z_k B
+// in fp64.
+constexpr int LP_THREADS = 512;
+
+__host__ __device__ inline size_t lp_smem_bytes(int C, int g)
 {
-    __shared__ float smax[8];
-    __shared__ double ssum[8];
-    const int n = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint8_t *row = qw + (int64_t)n * (C / 2);
-    const int zwn = zw[n];
-    auto value = [&](int j, int &k) -> float {  // RN(s_k (qw[n][R[j]] - z_w[n]))
-        int c = R[j];
+    return (size_t)C * 8 + (size_t)g * 16 + (((size_t)C / 2 + 15) & ~(size_t)15) + 16;
+}
+
+__global__ void __launch_bounds__(LP_THREADS)
+    linear_prepare_kernel(const uint8_t *__restrict__ qw, const int32_t *__restrict__ zw, const int32_t *__restrict__ R,
+                          const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                          const int32_t *__restrict__ zero, int g, int C, int N, __half *__restrict__ B,
+                          float *__restrict__ bz, float *__restrict__ lam, int *err)
+{
+    extern __shared__ __align__(16) uint8_t lp_smem[];
+    double *zd = reinterpret_cast<double *>(lp_smem);         // g
+    uint32_t *tab = reinterpret_cast<uint32_t *>(zd + g);     // C entries, stored order
+    float *bv = reinterpret_cast<float *>(tab + C);           // C: b of the current row
+    float *sc = bv + C;                                       // g
+    uint8_t *qrow = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sc + g) + 15) & ~(uintptr_t)15);
+    __shared__ float smax[LP_THREADS / 32];
+    __shared__ double ssum[LP_THREADS / 32];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int NW = LP_THREADS / 32;
+
+    for (int js = tid; js < C; js += LP_THREADS) {
+        const int j = lin_column(js);
+        int c = R[j], k = col_cluster[j];
         if (c < 0 || c >= C) {
             raise_error(err, RPTQ_DEVERR_REORDER);
             c = 0;
         }
-        k = col_cluster[j];
         if (k < 0 || k >= g) {
             raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
             k = 0;
         }
-        const int q = (row[c >> 1] >> ((c & 1) * 4)) & 15;
-        return scale[k] * (float)(q - zwn);
-    };
-    float m = 0.f;
-    for (int j = tid; j < C; j += 256) {
-        int k;
-        m = fmaxf(m, fabsf(value(j, k)));
+        tab[js] = (uint32_t)c | ((uint32_t)k << 16);
     }
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-    if (lane == 0) smax[warp] = m;
-    __syncthreads();
-    m = smax[0];
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, smax[w]);
-    // lam = 2^(e - 14) with m in [2^e, 2^(e+1)): the largest |B| lies in [2^14, 2^15)
-    int e = 0;
-    if (m > 0.f) frexpf(m, &e);
-    const float l = m > 0.f ? ldexpf(1.f, e - 1 - 14) : 1.f;
-    double acc = 0.0;
-    for (int js = tid; js < C; js += 256) {
-        int k;
-        const float v = value(lin_column(js), k) / l;  // a power of two: exact
-        const __half h = __float2half_rn(v);
-        B[(int64_t)n * C + js] = h;
-        acc += (double)zero[k] * (double)__half2float(h);
+    for (int k = tid; k < g; k += LP_THREADS) {
+        sc[k] = scale[k];
+        zd[k] = (double)zero[k];
     }
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if (lane == 0) ssum[warp] = acc;
-    __syncthreads();
-    if (tid == 0) {
-        double t = 0.0;
-        for (int w = 0; w < 8; ++w) t += ssum[w];
-        bz[n] = (float)t;
-        lam[n] = l;
+    const int groups = C / 8;
+    for (int n = blockIdx.x; n < N; n += gridDim.x) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(qw + (int64_t)n * (C / 2));
+        for (int i = tid; i < C / 32; i += LP_THREADS) reinterpret_cast<uint4 *>(qrow)[i] = __ldg(src + i);
+        __syncthreads();  // the row (and, the first time, the tables) are in place
+        const int zwi = zw[n];
+        // q - z_w as a float: exactly (2^23 + q) - (2^23 + z_w) while |z_w| < 2^22, else a conversion
+        const bool magic = zwi > -(1 << 22) && zwi < (1 << 22);
+        const float base = 8388608.0f + (float)zwi;
+        float m = 0.f;
+        for (int gi = tid; gi < groups; gi += LP_THREADS) {
+            const uint4 t0 = reinterpret_cast<const uint4 *>(tab)[2 * gi];
+            const uint4 t1 = reinterpret_cast<const uint4 *>(tab)[2 * gi + 1];
+            const uint32_t t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t c = t[e] & 0xFFFFu;
+                const int q = (qrow[c >> 1] >> ((c & 1) * 4)) & 15;
+                const float d = magic ? __int_as_float(0x4B000000 | q) - base : (float)(q - zwi);
+                v[e] = sc[t[e] >> 16] * d;  // b = RN(s_k (q - z_w))
+                m = fmaxf(m, fabsf(v[e]));
+            }
+            reinterpret_cast<float4 *>(bv)[2 * gi] = make_float4(v[0], v[1], v[2], v[3]);
+            reinterpret_cast<float4 *>(bv)[2 * gi + 1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+        if (lane == 0) smax[warp] = m;
+        __syncthreads();
+        m = smax[0];
+#pragma unroll
+        for (int w = 1; w < NW; ++w) m = fmaxf(m, smax[w]);
+        // lam = 2^(e - 14) with m in [2^e, 2^(e+1)): the largest |B| lies in [2^14, 2^15)
+        int e = 0;
+        if (m > 0.f) frexpf(m, &e);
+        const float l = m > 0.f ? ldexpf(1.f, e - 1 - 14) : 1.f;
+        const float rl = m > 0.f ? ldexpf(1.f, 15 - e) : 1.f;  // 1 / l, exact
+        double acc = 0.0;
+        uint4 *dst = reinterpret_cast<uint4 *>(B + (int64_t)n * C);
+        for (int gi = tid; gi < groups; gi += LP_THREADS) {
+            const uint4 t0 = reinterpret_cast<const uint4 *>(tab)[2 * gi];
+            const uint4 t1 = reinterpret_cast<const uint4 *>(tab)[2 * gi + 1];
+            const float4 v0 = reinterpret_cast<const float4 *>(bv)[2 * gi];
+            const float4 v1 = reinterpret_cast<const float4 *>(bv)[2 * gi + 1];
+            const uint32_t t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint32_t h[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                // b / l = b * (1 / l) exactly (powers of two), then one rounding to fp16
+                const __half2 hh = __floats2half2_rn(v[2 * p] * rl, v[2 * p + 1] * rl);
+                const float2 f = __half22float2(hh);
+                acc = fma(zd[t[2 * p] >> 16], (double)f.x, acc);
+                acc = fma(zd[t[2 * p + 1] >> 16], (double)f.y, acc);
+                h[p] = *reinterpret_cast<const uint32_t *>(&hh);
+            }
+            dst[gi] = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+        if (lane == 0) ssum[warp] = acc;
+        __syncthreads();
+        if (tid == 0) {
+            double tsum = 0.0;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) tsum += ssum[w];
+            bz[n] = (float)tsum;
+            lam[n] = l;
+        }
+        __syncthreads();  // qrow, bv, smax and ssum are reused by the next row
     }
 }
 
 cudaError_t launch_linear_prepare(const LinPrepArgs &a)
 {
     if (a.N == 0) return cudaSuccess;
-    linear_prepare_kernel<<<a.N, 256, 0, a.stream>>>(a.qw, a.sw, a.zw, a.R, a.col_cluster, a.scale, a.zero, a.g, a.C,
-                                                     a.N, a.B, a.bz, a.lam, a.err);
+    const size_t smem = lp_smem_bytes(a.C, a.g);
+    cudaError_t e = kernel_smem((const void *)linear_prepare_kernel, smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 1;
+    e = kernel_occupancy(&per_sm, (const void *)linear_prepare_kernel, LP_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(a.N, (int64_t)a.num_sms * std::max(1, per_sm));
+    linear_prepare_kernel<<<grid, LP_THREADS, smem, a.stream>>>(a.qw, a.zw, a.R, a.col_cluster, a.scale, a.zero, a.g,
+                                                                a.C, a.N, a.B, a.bz, a.lam, a.err);
     return cudaGetLastError();
 }
 
 // ---- the GEMM ---------------------------------------------------------------------------------
-constexpr int LIN_BM = 128, LIN_BN = 256, LIN_BK = 64, LIN_STAGES = 4;
-constexpr int LIN_PROD = 256;               // warps 0-7: A producers, then the epilogue
+constexpr int LIN_BM = 128, LIN_BN = 256, LIN_BK = 64, LIN_STAGES = 6;
+constexpr int LIN_PROD = 256;               // warps 0-7: A producers (0-3 even slabs, 4-7 odd), then the epilogue
 constexpr int LIN_THREADS = LIN_PROD + 64;  // warp 8: weight copies, warp 9: MMA issue + TMEM
-constexpr uint32_t LIN_A_BYTES = LIN_BM * LIN_BK * 2;
 constexpr uint32_t LIN_B_BYTES = LIN_BN * LIN_BK * 2;
-constexpr uint32_t LIN_TMEM_COLS = LIN_BN;  // one fp32 column per output of the tile
-constexpr size_t LIN_SMEM = 1024 + (size_t)LIN_STAGES * (LIN_A_BYTES + LIN_B_BYTES);
+constexpr uint32_t LIN_TMEM_COLS = 512;     // the accumulator (256 columns) + the A ring (6 x 32)
+constexpr uint32_t LIN_A_COL = LIN_BN;      // A slab s at columns LIN_A_COL + 32 s
+constexpr size_t LIN_SMEM = 1024 + (size_t)LIN_STAGES * LIN_B_BYTES;
 static_assert(LIN_BK * 2 == 128, "one 128-byte swizzle row per K slab");
+static_assert(LIN_STAGES % 2 == 0, "a ring slot always holds slabs of one parity");
+static_assert(LIN_A_COL + LIN_STAGES * (LIN_BK / 2) <= LIN_TMEM_COLS, "tensor memory budget");
 
 // fp16 pairs 1024 + q  ->  q (exact)
 __device__ __forceinline__ uint32_t lin_sub1024(uint32_t v)
@@ -191,32 +277,34 @@ __device__ __forceinline__ uint32_t lin_sub1024(uint32_t v)
 // little-endian word, code i in bits 4i..4i+3.  A3: 24 bits, code i in bits 3i..3i+2; codes 4-7
 // move up to bit 16 first.  A code OR-ed into the mantissa of 1024.0 (0x6400) gives 1024 + q.
 template <int BITS>
-__device__ __forceinline__ uint4 lin_decode8(uint32_t w)
+__device__ __forceinline__ void lin_decode8(uint32_t w, uint32_t *o)
 {
     if constexpr (BITS == 3) w = (w & 0xFFFu) | ((w & 0xFFF000u) << 4);
     constexpr uint32_t M = BITS == 4 ? 0x000F000Fu : 0x00070007u;
-    uint4 o;
-    o.x = lin_sub1024(((w >> 0) & M) | 0x64006400u);
-    o.y = lin_sub1024(((w >> BITS) & M) | 0x64006400u);
-    o.z = lin_sub1024(((w >> (2 * BITS)) & M) | 0x64006400u);
-    o.w = lin_sub1024(((w >> (3 * BITS)) & M) | 0x64006400u);
-    return o;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = lin_sub1024(((w >> (BITS * i)) & M) | 0x64006400u);
 }
-// Four 8-code groups of one row: 16 bytes (A4) or 12 bytes (A3) at p (4-byte aligned).
+// The 64 codes of one row and one K slab (8 groups): 32 bytes (A4) or 24 bytes (A3) at p
+// (16- resp. 8-byte aligned).  A3 group m sits in bytes 3m..3m+2; w[m] holds it in bits 0-23.
 template <int BITS>
-__device__ __forceinline__ void lin_load_groups(const uint8_t *p, uint32_t (&w)[4])
+__device__ __forceinline__ void lin_load_slab(const uint8_t *p, uint32_t (&w)[8])
 {
     if constexpr (BITS == 4) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p));
-        w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(p) + 1);
+        w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
     } else {
-        const uint32_t a = __ldg(reinterpret_cast<const uint32_t *>(p));
-        const uint32_t b = __ldg(reinterpret_cast<const uint32_t *>(p) + 1);
-        const uint32_t c = __ldg(reinterpret_cast<const uint32_t *>(p) + 2);
-        w[0] = a;                          // bytes 0-2 (the decoder drops bits 24-31)
-        w[1] = __funnelshift_r(a, b, 24);  // bytes 3-5
-        w[2] = __funnelshift_r(b, c, 16);  // bytes 6-8
-        w[3] = c >> 8;                     // bytes 9-11
+        const uint2 a = __ldg(reinterpret_cast<const uint2 *>(p));
+        const uint2 b = __ldg(reinterpret_cast<const uint2 *>(p) + 1);
+        const uint2 c = __ldg(reinterpret_cast<const uint2 *>(p) + 2);
+        const uint32_t x[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // 12 bytes = 4 groups
+            w[4 * h + 0] = x[3 * h];
+            w[4 * h + 1] = __funnelshift_r(x[3 * h], x[3 * h + 1], 24);
+            w[4 * h + 2] = __funnelshift_r(x[3 * h + 1], x[3 * h + 2], 16);
+            w[4 * h + 3] = x[3 * h + 2] >> 8;
+        }
     }
 }
 __device__ __forceinline__ void lin_tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
@@ -230,7 +318,9 @@ __device__ __forceinline__ void lin_tma_load_2d(uint32_t dst, const CUtensorMap 
 
 // Y[t][n] = f[n] (sum_j q[t][j] B[n][j] - bz[n]),  f = s_w lam.  Grid: x = token tiles of 128
 // (consecutive CTAs share one weight tile, which then comes from DRAM once), y = output tiles
-// of 256.  K = C is a multiple of 64: K / 64 slabs.
+// of 256.  K = C is a multiple of 64: K / 64 slabs.  The decoded codes go straight from the
+// producers' registers into tensor memory (tcgen05.st) and the MMA reads A from there, so shared
+// memory carries only the weight slabs.
 template <int BITS>
 __global__ void __launch_bounds__(LIN_THREADS, 1)
     reordered_linear_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ codes, int64_t T,
@@ -247,14 +337,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     const int64_t m0 = (int64_t)blockIdx.x * LIN_BM;
     const int n0 = blockIdx.y * LIN_BN;
     const int KT = K / LIN_BK;
-    const uint32_t sbase = (smem_u32(lin_smem_raw) + 1023u) & ~1023u;  // swizzled tiles: 1024-aligned
-    const uint32_t sA = sbase, sB = sbase + LIN_STAGES * LIN_A_BYTES;
+    const uint32_t sB = (smem_u32(lin_smem_raw) + 1023u) & ~1023u;  // swizzled tiles: 1024-aligned
     const uint32_t full_a = smem_u32(&bars[0]), full_b = smem_u32(&bars[LIN_STAGES]);
     const uint32_t empty = smem_u32(&bars[2 * LIN_STAGES]), done = smem_u32(&bars[3 * LIN_STAGES]);
 
     if (tid == 0) {
         for (int s = 0; s < LIN_STAGES; ++s) {
-            mbar_init(full_a + 8 * s, LIN_PROD);
+            mbar_init(full_a + 8 * s, LIN_PROD / 2);  // the 4 warps of one slab parity
             mbar_init(full_b + 8 * s, 1);
             mbar_init(empty + 8 * s, 1);
         }
@@ -274,49 +363,52 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     const uint32_t tmem = tmem_slot;
 
     if (warp < 8) {
-        // ---- A producers: thread = (row r, half h of the slab's 64 codes = 4 groups of 8) ----
-        const int r = tid >> 1, h = tid & 1;
+        // ---- A producers: warp w owns TMEM lanes 32 (w % 4) .. +31 (the tile's rows) and the
+        //      slabs of parity w / 4; a thread decodes its row's 64 codes into 32 columns ----
+        const int qd = warp & 3, par = warp >> 2;
+        const int r = 32 * qd + lane;
         const bool row_ok = m0 + r < T;
         const int64_t pitch = (int64_t)K * BITS / 8;
-        const uint8_t *src = codes + (row_ok ? m0 + r : 0) * pitch + h * (4 * BITS);
-        uint32_t wa[4] = {0, 0, 0, 0}, wb[4] = {0, 0, 0, 0};
-        if (row_ok) lin_load_groups<BITS>(src, wa);
-        if (row_ok && KT > 1) lin_load_groups<BITS>(src + 8 * BITS, wb);
+        const uint8_t *src = codes + (row_ok ? m0 + r : 0) * pitch;
+        const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + LIN_A_COL;
+        uint32_t wa[8], wb[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wa[i] = wb[i] = 0;
+        if (row_ok && par < KT) lin_load_slab<BITS>(src + (int64_t)par * (8 * BITS), wa);
+        if (row_ok && par + 2 < KT) lin_load_slab<BITS>(src + (int64_t)(par + 2) * (8 * BITS), wb);
         bool ok = true;
-        for (int kt = 0; kt < KT; ++kt) {
-            uint32_t wc[4] = {0, 0, 0, 0};
-            if (row_ok && kt + 2 < KT) lin_load_groups<BITS>(src + (int64_t)(kt + 2) * (8 * BITS), wc);
+        for (int kt = par; kt < KT; kt += 2) {
+            uint32_t wc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wc[i] = 0;
+            if (row_ok && kt + 4 < KT) lin_load_slab<BITS>(src + (int64_t)(kt + 4) * (8 * BITS), wc);
             const int s = kt % LIN_STAGES, u = kt / LIN_STAGES;
             if (!mbar_wait_bounded(empty + 8 * s, (u & 1) ^ 1, err)) {
                 ok = false;
                 *(volatile int *)&s_abort = 1;
                 break;
             }
-            const uint32_t dst = sA + s * LIN_A_BYTES + r * 128;
+            tc_fence_after();  // the slot's previous MMAs are complete
+            uint32_t d[32];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 v = lin_decode8<BITS>(wa[i]);
-                const uint32_t c = (uint32_t)(4 * h + i) ^ (uint32_t)(r & 7);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (c << 4)), "r"(v.x), "r"(v.y),
-                             "r"(v.z), "r"(v.w)
-                             : "memory");
-            }
-            fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+            for (int gi = 0; gi < 8; ++gi) lin_decode8<BITS>(wa[gi], d + 4 * gi);
+            tc_st32(ta + 32 * s, d);
+            tc_wait_st();
+            tc_fence_before();
             lin_arrive(full_a + 8 * s);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) wa[i] = wb[i], wb[i] = wc[i];
+            for (int i = 0; i < 8; ++i) wa[i] = wb[i], wb[i] = wc[i];
         }
         // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, columns 128 (w / 4) .. +127 ----
         if (ok) ok = mbar_wait_bounded(done, 0, err);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective: the whole warp or none
         tc_fence_after();
         if (ok) {
-            const int q = warp & 3;
-            const int64_t row = m0 + 32 * q + lane;
+            const int64_t row = m0 + r;
             for (int i = 0; i < 4; ++i) {
-                const int col0 = (warp >> 2) * 128 + 32 * i;
+                const int col0 = par * 128 + 32 * i;
                 uint32_t v[32];
-                tc_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)col0, v);
+                tc_ld32(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)col0, v);
                 if (row >= T || n0 + col0 >= N) continue;
                 float *yrow = Y + row * (int64_t)N + n0 + col0;
                 if (vec_store && n0 + col0 + 32 <= N) {
@@ -359,7 +451,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 mbar_wait_bounded(empty + 8 * (kt % LIN_STAGES), (kt / LIN_STAGES) & 1, err);
         }
     } else {
-        // ---- MMA issue: four K = 16 steps per slab; the descriptor start advances 32 bytes ----
+        // ---- MMA issue: four K = 16 steps per slab (8 TMEM columns of A, 32 bytes of B each) ----
         if (lane == 0) {
             constexpr uint32_t idesc = f16_idesc(LIN_BM, LIN_BN);
             for (int kt = 0; kt < KT; ++kt) {
@@ -369,11 +461,12 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint64_t ad = sw128_desc(sA + s * LIN_A_BYTES), bd = sw128_desc(sB + s * LIN_B_BYTES);
+                const uint64_t bd = sw128_desc(sB + s * LIN_B_BYTES);
+                const uint32_t at = tmem + LIN_A_COL + 32 * s;
 #pragma unroll
                 for (int kk = 0; kk < LIN_BK / 16; ++kk)
-                    tc_mma_f16(tmem, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (kt | kk) != 0);
-                tc_commit(empty + 8 * s);  // the slab may be refilled once these MMAs are done
+                    tc_mma_f16_ts(tmem, at + 8 * kk, bd + (uint64_t)(2 * kk), idesc, (kt | kk) != 0);
+                tc_commit(empty + 8 * s);  // the slot may be refilled once these MMAs are done
             }
             tc_commit(done);
             // the accumulator is released below: wait for every issued MMA first

@@ -52,7 +52,7 @@ SIGNATURES = {
     "rptq_cluster_params": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
-    "rptq_linear_prepare": (_I, [_P, _P, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
+    "rptq_linear_prepare": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "rptq_reordered_linear": (_I, [_P, _I64, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
     # include/rptq_baseline.h
     "rptq_baseline_explicit_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P,
@@ -293,8 +293,8 @@ def rptq_kv_decode_attention(q, k_cache, v_cache, L: int, cluster_k, scale_k, ze
     return out
 
 
-def rptq_linear_prepare(w_codes, w_scale, w_zero, R, col_cluster, scale, zero, w_prep=None, w_bias=None,
-                        w_lambda=None, stream=None):
+def rptq_linear_prepare(w_codes, w_zero, R, col_cluster, scale, zero, w_prep=None, w_bias=None, w_lambda=None,
+                        stream=None):
     """Offline operand of the reordered linear layer from 4-bit weight codes w_codes [N, C/2]
     (original channel order) and the activation calibration; returns (w_prep fp16 [N, C],
     w_bias fp32 [N], w_lambda fp32 [N])."""
@@ -307,7 +307,7 @@ def rptq_linear_prepare(w_codes, w_scale, w_zero, R, col_cluster, scale, zero, w
         w_bias = torch.empty(N, dtype=torch.float32, device=dev)
     if w_lambda is None:
         w_lambda = torch.empty(N, dtype=torch.float32, device=dev)
-    st = lib().rptq_linear_prepare(_ptr(w_codes), _ptr(w_scale), _ptr(w_zero), N, C, _ptr(R), _ptr(col_cluster),
+    st = lib().rptq_linear_prepare(_ptr(w_codes), _ptr(w_zero), N, C, _ptr(R), _ptr(col_cluster),
                                    _ptr(scale), _ptr(zero), scale.numel(), _ptr(w_prep), _ptr(w_bias),
                                    _ptr(w_lambda), _stream(stream))
     _check(st, "rptq_linear_prepare")

@@ -22,7 +22,7 @@ from dataclasses import dataclass
 import torch
 
 # sub-stream identifiers (mixed into the seed)
-_S_CHANNEL, _S_OUTLIER, _S_LN, _S_X, _S_CALIB, _S_K, _S_V, _S_W = range(8)
+_S_CHANNEL, _S_OUTLIER, _S_LN, _S_X, _S_CALIB, _S_K, _S_V, _S_W, _S_WQ = range(9)
 
 _DTYPES = {"f32": torch.float32, "f16": torch.float16, "bf16": torch.bfloat16}
 
@@ -105,3 +105,14 @@ def weights(N: int, C: int, seed: int) -> torch.Tensor:
     order), W ~ N(0, 1/C); fp32 on CPU."""
     g = _gen(seed, _S_W, "cpu")
     return (torch.randn((N, C), generator=g, dtype=torch.float32) * (1.0 / C) ** 0.5).contiguous()
+
+
+def weight_codes(N: int, C: int, seed: int, device="cpu"):
+    """Synthetic 4-bit weight codes of the linear layer for the benchmark, already packed
+    (uniform random bytes: every nibble uniform on 0..15, low nibble = even channel), with per-row
+    scales s_w ~ U(0.5, 1.5) / (15 sqrt(C)) and zero points z_w ~ U{0..15}."""
+    g = _gen(seed, _S_WQ, "cpu")
+    packed = torch.randint(0, 256, (N, C // 2), generator=g, dtype=torch.uint8)
+    sw = ((torch.rand(N, generator=g, dtype=torch.float64) + 0.5) / (15.0 * C ** 0.5)).float()
+    zw = torch.randint(0, 16, (N,), generator=g, dtype=torch.int32)
+    return packed.to(device), sw.to(device), zw.to(device)

@@ -123,3 +123,24 @@ def bytes_explicit_reorder(T: int, C: int, dtype: str, bits: int) -> int:
     reordered copy, read that and write the packed codes."""
     n = T * C
     return n * ESIZE[dtype] + 4 * n * 4 + n * bits // 8
+
+
+# ---- the reordered linear layer after the LayerNorm (a tensor-core contraction, not HBM-bound)
+LINEAR_TOKENS = 2048  # one 2048-token micro-batch of the step's activation codes
+
+
+def linear_shape(w: "Workload"):
+    """(tokens, C, N) of the layer the step runs on the activation codes: the first
+    min(T, 2048) tokens through the fused Q/K/V projection of the model (N = 3 C)."""
+    return min(w.T, LINEAR_TOKENS), w.C, 3 * w.C
+
+
+def flops_linear(T: int, C: int, N: int) -> int:
+    """Multiply-adds of the layer, counted as 2 operations each."""
+    return 2 * T * C * N
+
+
+def bytes_linear_prepare(N: int, C: int) -> int:
+    """Offline operand preparation: read the 4-bit weight codes, write the fp16 operand and the
+    per-row bias and scale."""
+    return N * C // 2 + N * C * 2 + 2 * N * 4

@@ -49,8 +49,8 @@ def test_stage_accounting_per_workload():
     from post_activation_quantization_b200 import workloads as W
     st = bench.stage_list(W.WORKLOADS["opt175b-12288"])
     assert [s[0] for s in st] == ["calib_ln", "kv_calib", "kmeans", "ln_reorder_quant", "explicit_reorder_baseline",
-                                  "dynamic_ranges", "kv_quant", "dequant_act", "dequant_kv", "kv_append",
-                                  "kv_decode_attention"]
+                                  "dynamic_ranges", "linear_prepare", "reordered_linear", "kv_quant", "dequant_act",
+                                  "dequant_kv", "kv_append", "kv_decode_attention"]
     b = dict((n, v) for n, v, _ in st)
     T, C, Tc, kv = 32768, 12288, 262144, 8 * 96 * 2048 * 128
     assert b["calib_ln"] == Tc * C * 2
@@ -63,14 +63,20 @@ def test_stage_accounting_per_workload():
     assert b["kv_decode_attention"] == 2 * kv * 3 // 8 + 2 * 8 * 96 * 128 * 4
     assert b["explicit_reorder_baseline"] == T * C * 2 + 4 * T * C * 4 + T * C * 3 // 8
     assert b["dynamic_ranges"] == T * C * 2
-    assert sum(l for _, _, l in st) == 25  # 2 + 4 + 6 + 1 + 3 + 3 + 1 + 1 + 2 + 1 + 1
+    # the Q/K/V projection (N = 3C) on a 2048-token micro-batch: its operand preparation reads
+    # the 4-bit codes and writes fp16 plus two floats per row; the GEMM is counted in FLOPs
+    N = 3 * C
+    assert b["linear_prepare"] == N * C // 2 + N * C * 2 + 8 * N and b["reordered_linear"] == 0
+    assert bench.stage_flops(W.WORKLOADS["opt175b-12288"]) == {"reordered_linear": 2 * 2048 * C * N}
+    assert sum(l for _, _, l in st) == 27  # 2 + 4 + 6 + 1 + 3 + 3 + 1 + 1 + 1 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["kv-4096"])
     assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "dequant_kv", "kv_append", "kv_decode_attention"]
     assert sum(l for _, _, l in st) == 4 + 4 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["tiny-768"])
     assert [s[0] for s in st] == ["calib_ln", "kmeans", "ln_reorder_quant", "explicit_reorder_baseline",
-                                  "dynamic_ranges", "dequant_act"]
-    assert sum(l for _, _, l in st) == 2 + 2 + 1 + 3 + 3 + 1
+                                  "dynamic_ranges", "linear_prepare", "reordered_linear", "dequant_act"]
+    assert sum(l for _, _, l in st) == 2 + 2 + 1 + 3 + 3 + 1 + 1 + 1
+    assert bench.stage_flops(W.WORKLOADS["tiny-768"]) == {"reordered_linear": 2 * 512 * 768 * 2304}
 
 
 def test_gpus_n_starts_n_ranks():

@@ -65,7 +65,7 @@ def _run(cal, codes, qw, sw, zw, C, bits):
     p = dev_params(cal)
     wq = torch.from_numpy(oracle.pack(qw, 4)).to(DEV)
     sw_d, zw_d = torch.from_numpy(sw).to(DEV), torch.from_numpy(zw).to(DEV)
-    w_prep, w_bias, w_lam = rptq.rptq_linear_prepare(wq, sw_d, zw_d, p["R"], p["col_cluster"], p["scale"], p["zero"])
+    w_prep, w_bias, w_lam = rptq.rptq_linear_prepare(wq, zw_d, p["R"], p["col_cluster"], p["scale"], p["zero"])
     Y = rptq.rptq_reordered_linear(torch.from_numpy(codes).to(DEV), C, bits, w_prep, w_bias, w_lam, sw_d)
     torch.cuda.synchronize()
     return to_np(Y), to_np(w_prep), to_np(w_bias), to_np(w_lam)
@@ -114,7 +114,7 @@ def _check(Y, wp, wb, wl, cal, codes, qw, sw, zw, C, bits, what, rows=None, cols
     (1, 64, 1, 2, 3),          # one token, one output
     (1000, 768, 1000, 8, 4),   # the tiny layer's width, several tiles each way
     (257, 768, 520, 8, 3),
-    (300, 1280, 384, 16, 4),   # K = 20 slabs: the four-stage ring wraps five times
+    (300, 1280, 384, 16, 4),   # K = 20 slabs: the six-slot ring wraps three times
 ])
 def test_reordered_linear_matches_the_oracle(T, C, N, g, bits):
     seed = 3 * T + C + N
@@ -147,13 +147,36 @@ def test_full_shape_sampled(bits):
     assert np.isfinite(Y).all()
 
 
+def test_bench_shape_sampled():
+    """The OPT-175B-shaped layer the bench step runs: 2048 tokens x 12288 channels of A3 codes
+    into the 36864-wide Q/K/V projection, with the bench's synthetic 4-bit weight codes; 64 x 64
+    sampled outputs (the last token and output included)."""
+    T, C, N, g, bits = 2048, 12288, 36864, 64, 3
+    cal, codes, _, _, _ = _case(T, C, 8, g, bits, 31)
+    wq, sw_t, zw_t = synthetic.weight_codes(N, C, 31)
+    p = dev_params(cal)
+    sw_d, zw_d = sw_t.to(DEV), zw_t.to(DEV)
+    w_prep, w_bias, w_lam = rptq.rptq_linear_prepare(wq.to(DEV), zw_d, p["R"], p["col_cluster"], p["scale"], p["zero"])
+    Y = rptq.rptq_reordered_linear(torch.from_numpy(codes).to(DEV), C, bits, w_prep, w_bias, w_lam, sw_d)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    rows = np.unique(np.r_[rng.choice(T, 63, replace=False), T - 1])
+    cols = np.unique(np.r_[rng.choice(N, 63, replace=False), N - 1])
+    ci = torch.from_numpy(cols).to(DEV)
+    # the sampled outputs' columns of Y and rows of the operand, gathered on the device
+    Ys, wps, wbs, wls = to_np(Y[:, ci]), to_np(w_prep[ci]), to_np(w_bias[ci]), to_np(w_lam[ci])
+    qws = oracle.unpack(wq.numpy()[cols], C, 4)
+    _check(Ys, wps, wbs, wls, cal, codes, qws, sw_t.numpy()[cols], zw_t.numpy()[cols], C, bits,
+           "linear bench shape A3 (sampled)", rows)
+
+
 def test_no_tokens_and_refused_shapes():
     C, N, g = 128, 64, 4
     cal, codes, qw, sw, zw = _case(4, C, N, g, 4, 5)
     p = dev_params(cal)
     wq = torch.from_numpy(oracle.pack(qw, 4)).to(DEV)
     sw_d, zw_d = torch.from_numpy(sw).to(DEV), torch.from_numpy(zw).to(DEV)
-    w_prep, w_bias, w_lam = rptq.rptq_linear_prepare(wq, sw_d, zw_d, p["R"], p["col_cluster"], p["scale"], p["zero"])
+    w_prep, w_bias, w_lam = rptq.rptq_linear_prepare(wq, zw_d, p["R"], p["col_cluster"], p["scale"], p["zero"])
     empty = torch.empty((0, C // 2), dtype=torch.uint8, device=DEV)
     out = rptq.rptq_reordered_linear(empty, C, 4, w_prep, w_bias, w_lam, sw_d)
     assert out.shape == (0, N)
@@ -173,6 +196,5 @@ def test_out_of_range_reorder_entry_sets_the_error_word():
     R_bad = p["R"].clone()
     R_bad[3] = C + 5
     wq = torch.from_numpy(oracle.pack(qw, 4)).to(DEV)
-    rptq.rptq_linear_prepare(wq, torch.from_numpy(sw).to(DEV), torch.from_numpy(zw).to(DEV), R_bad,
-                             p["col_cluster"], p["scale"], p["zero"])
+    rptq.rptq_linear_prepare(wq, torch.from_numpy(zw).to(DEV), R_bad, p["col_cluster"], p["scale"], p["zero"])
     assert rptq.rptq_device_error() & 2
