@@ -4,7 +4,9 @@
 A step is one pass of the whole path over one synthetic batch of the workload:
   1. calibration statistics of LayerNorm(x) over the calibration batch   (rptq_calib_minmax)
   2. KMeans -> reorder index R and per-cluster (s, z)                    (rptq_kmeans)
-  3. reorder-fused LayerNorm + per-cluster quantization of the batch      (rptq_ln_reorder_quant)
+  3. the LayerNorm rewrite of this calibration, then the reorder-fused LayerNorm + per-cluster
+     quantization of the batch       (rptq_ln_quant_plan, rptq_ln_reorder_quant_planned; the
+     unplanned rptq_ln_reorder_quant is timed beside it)
   3a. the explicit-reorder baseline, dynamic ranges, and the reordered linear layer on one
       2048-token micro-batch of the codes  (rptq_baseline_..., rptq_linear_prepare, rptq_reordered_linear)
   4. K/V calibration statistics, KMeans for K and for V                   (rptq_kv_calib_minmax, rptq_kmeans)
@@ -89,7 +91,12 @@ def stage_list(w: W.Workload):
         st += [("kv_calib", 2 * W.bytes_calib(k.B * k.S, k.channels, k.dtype), 4)]
     st += [("kmeans", 0, 2 * ((1 if a else 0) + (2 if k else 0)))]
     if a:
-        st += [("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
+        # the offline LayerNorm rewrite of this calibration (per-channel offsets and
+        # coefficients), then the fused kernel reading it; the same kernel building those tables
+        # in every CTA is timed beside it
+        st += [("ln_quant_plan", W.bytes_ln_quant_plan(w.C), 1),
+               ("ln_reorder_quant", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1),
+               ("ln_reorder_quant_unplanned", W.bytes_ln_quant(w.T, w.C, w.dtype, w.bits), 1)]
         # the unfused pipeline the fused kernel replaces (a measurement baseline, same results)
         st += [("explicit_reorder_baseline", W.bytes_explicit_reorder(w.T, w.C, w.dtype, w.bits), 3)]
         # what dynamic (per-batch) cluster ranges add before the same fused kernel: the batch's
@@ -135,6 +142,7 @@ class Step:
             self.km = self._km_out(w.C, w.g)
             self.ws = torch.empty(rptq.rptq_kmeans_workspace_size(w.C, w.g), dtype=torch.uint8, device=device)
             self.codes = torch.empty((w.T, w.C * w.bits // 8), dtype=torch.uint8, device=device)
+            self.plan = torch.empty(rptq.rptq_ln_quant_plan_bytes(w.C), dtype=torch.uint8, device=device)
             self.xr_y = torch.empty((w.T, w.C), dtype=torch.float32, device=device)
             self.xr_yr = torch.empty_like(self.xr_y)
             self.xr_codes = torch.empty_like(self.codes)
@@ -231,10 +239,17 @@ class Step:
                 main.wait_stream(s)
         mark("kmeans", 1)
         if self.act:
+            mark("ln_quant_plan", 0)
+            r.rptq_ln_quant_plan(self.gamma, self.beta, self.km["R"], self.km["col_cluster"], self.km["scale"],
+                                 self.km["zero"], w.bits, plan=self.plan)
+            mark("ln_quant_plan", 1)
             mark("ln_reorder_quant", 0)
-            r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
-                                    self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.codes)
+            r.rptq_ln_reorder_quant_planned(self.x, self.plan, w.bits, eps=w.eps, codes=self.codes)
             mark("ln_reorder_quant", 1)
+            mark("ln_reorder_quant_unplanned", 0)
+            r.rptq_ln_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
+                                    self.km["scale"], self.km["zero"], w.bits, eps=w.eps, codes=self.xr_codes)
+            mark("ln_reorder_quant_unplanned", 1)
             mark("explicit_reorder_baseline", 0)
             r.rptq_baseline_explicit_reorder_quant(self.x, self.gamma, self.beta, self.km["R"], self.km["col_cluster"],
                                                    self.km["scale"], self.km["zero"], w.bits, eps=w.eps,
@@ -472,7 +487,8 @@ def run_rptq(args):
             "headline_kernel": head,
             "mtokens_per_s": round(tokens * ws * args.steps / (head_ms * 1e-3) / 1e6, 3),
             "frac_of_measured_hbm": round(value / ws / hbm, 4),
-            "step": {"what": "every stage of the path once: calibration, KMeans, fused quantization, the "
+            "step": {"what": "every stage of the path once: calibration, KMeans, the LayerNorm plan, fused quantization "
+                             "(planned, and unplanned for comparison), the "
                              "explicit-reorder baseline, dynamic ranges, the reordered linear layer (weight "
                              "preparation, one 2048-token micro-batch), K/V quantization, dequantization, "
                              "one decode step (append, attention)",
@@ -537,8 +553,7 @@ def run_e2e(step: Step, args, dev, ws):
         ins, outs = [step.x], [step.codes]
 
         def call():
-            r.rptq_ln_reorder_quant(step.x, step.gamma, step.beta, step.km["R"], step.km["col_cluster"],
-                                    step.km["scale"], step.km["zero"], w.bits, eps=w.eps, codes=step.codes)
+            r.rptq_ln_reorder_quant_planned(step.x, step.plan, w.bits, eps=w.eps, codes=step.codes)
     else:
         k = step.kvw
         ins, outs = [step.k, step.v], [step.kq, step.vq]

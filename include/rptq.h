@@ -224,6 +224,36 @@ int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const floa
                           int g, int bits, uint8_t *codes, void *ln_out, rptq_stream_t stream);
 
 /*
+ * The offline LayerNorm rewrite as data: [RPTQ-art] text after Fig. 3 (the LayerNorm is changed
+ * once, offline, so that it emits the reordered, quantized activations) folded with the text
+ * after Fig. 2 (one (s, z) per cluster).  For every channel c, with j its stored column
+ * (R[j] = c) and k = col_cluster[j], the plan holds the code-buffer offset of j and the affine
+ * coefficients A_c = gamma_c / (s_k qmax), B_c = beta_c / (s_k qmax) + z_k / qmax (fp64,
+ * rounded to fp32 once) with which rptq_ln_reorder_quant computes the codes; with the plan the
+ * fused kernel does not rebuild these tables in every CTA.
+ *   plan  device buffer of rptq_ln_quant_plan_bytes(C) bytes, 16-byte aligned, written here
+ *         (layout: uint32 offset[C], float A[C], float B[C]; to be read only by
+ *         rptq_ln_reorder_quant_planned).
+ * Arguments as in rptq_ln_reorder_quant.  An R entry outside [0, C) or a cluster id outside
+ * [0, g) sets the device error word (the channel keeps offset 0, A = B = 0, resp. uses
+ * cluster 0).
+ */
+size_t rptq_ln_quant_plan_bytes(int C);
+int rptq_ln_quant_plan(const float *gamma, const float *beta, const int32_t *R,
+                       const int32_t *col_cluster, const float *scale, const int32_t *zero, int C,
+                       int g, int bits, void *plan, rptq_stream_t stream);
+
+/*
+ * rptq_ln_reorder_quant (codes only) from a plan: the same codes, bit for bit, as
+ * rptq_ln_reorder_quant with the arguments the plan was made from.  `bits` must be the plan's.
+ * Shapes: those for which rptq_ln_reorder_quant uses its direct kernel -- C a multiple of 32 with
+ * a thread split of the row (every OPT hidden size 768 .. 12288 qualifies); others return
+ * RPTQ_ERR_UNSUPPORTED.  T == 0 is valid: nothing is launched.
+ */
+int rptq_ln_reorder_quant_planned(const void *x, int dtype, int64_t T, int C, float eps,
+                                  const void *plan, int bits, uint8_t *codes, rptq_stream_t stream);
+
+/*
  * K/V cache quantization with per-cluster parameters ([RPTQ-art] results paragraph:
  * W4A4KV / W4A3KV / W3A3KV quantize the key and value caches alone).
  * k, v: [B, H, S, D] of `dtype` (either may be NULL, not both); channel c = h*D + d.

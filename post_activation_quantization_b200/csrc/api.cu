@@ -277,6 +277,42 @@ int rptq_ln_reorder_quant(const void *x, int dtype, int64_t T, int C, const floa
     return cuda_status(launch_ln_quant(a, 0));
 }
 
+size_t rptq_ln_quant_plan_bytes(int C) { return C > 0 ? (size_t)C * 12 : 0; }
+
+int rptq_ln_quant_plan(const float *gamma, const float *beta, const int32_t *R, const int32_t *col_cluster,
+                       const float *scale, const int32_t *zero, int C, int g, int bits, void *plan,
+                       rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (g <= 0 || g > C) return RPTQ_ERR_INVALID_ARG;
+    if (!gamma || !beta || !R || !col_cluster || !scale || !zero || !plan || !aligned16(plan))
+        return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    return cuda_status(launch_ln_quant_plan(gamma, beta, R, col_cluster, scale, zero, C, g, bits, plan, d.err,
+                                            (cudaStream_t)stream));
+}
+
+int rptq_ln_reorder_quant_planned(const void *x, int dtype, int64_t T, int C, float eps, const void *plan,
+                                  int bits, uint8_t *codes, rptq_stream_t stream)
+{
+    if (!dtype_ok(dtype)) return RPTQ_ERR_UNSUPPORTED;
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (T < 0 || !(eps >= 0.0f) || !plan || !aligned16(plan)) return RPTQ_ERR_INVALID_ARG;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if (!ln_quant_plan_supported(C, esize(dtype), d.max_smem)) return RPTQ_ERR_UNSUPPORTED;
+    if (T == 0) return RPTQ_OK;
+    if (!x || !codes || !aligned16(x) || !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
+    LnQuantArgs a{x, dtype, T, C, nullptr, nullptr, eps, nullptr, nullptr, nullptr, nullptr, 0, bits, codes,
+                  nullptr, d.err, (cudaStream_t)stream, d.num_sms, d.max_smem, plan};
+    return cuda_status(launch_ln_quant(a, 0));
+}
+
 int rptq_kv_quant(const void *k, const void *v, int dtype, int B, int H, int64_t S, int D,
                   const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,
                   const int32_t *cluster_v, const float *scale_v, const int32_t *zero_v, int g,

@@ -31,6 +31,7 @@ struct LnQuantArgs {
     cudaStream_t stream;
     int num_sms;
     int max_smem;
+    const void *plan;  // rptq_ln_quant_plan's output, or NULL (tables built from R, s, z, gamma, beta)
 };
 
 struct CalibArgs {
@@ -195,6 +196,10 @@ struct KmArgs {
 
 // force_simple = 1 routes codes-only calls to the general kernel (used by tests of that path)
 cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple);
+cudaError_t launch_ln_quant_plan(const float *gamma, const float *beta, const int32_t *R, const int32_t *col_cluster,
+                                 const float *scale, const int32_t *zero, int C, int g, int bits, void *plan,
+                                 int *err, cudaStream_t stream);
+bool ln_quant_plan_supported(int C, int esize, int max_smem);
 bool ln_quant_fast_plan(int C, int esize, int max_smem, bool allow_direct, int *CPT, int *NT, int *NS, int *alias);
 cudaError_t launch_calib(const CalibArgs &a);
 cudaError_t launch_kv_calib(const KvCalibArgs &a);

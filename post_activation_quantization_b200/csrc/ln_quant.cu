@@ -172,6 +172,74 @@ __device__ __forceinline__ void quant_tables_direct(const int32_t *R, const int3
     }
 }
 
+// The same per-thread state from a plan written by ln_quant_plan_kernel (one entry per channel:
+// code-buffer offset, A, B; computed once per calibration, which is the offline LayerNorm
+// rewrite): each thread reads only its own channels' entries, coalesced 16-byte loads, and
+// keeps its offsets in its own slots of the shared position table.  An offset is clamped into the
+// code buffer and 4-byte aligned, so even a damaged plan cannot store outside it.
+template <typename T, int CPT>
+__device__ __forceinline__ void load_plan(const void *plan, int C, int NCH, int NT, uint32_t *postab, uint32_t pbase,
+                                          float (&pA)[CPT][Elem<T>::VEC], float (&pB)[CPT][Elem<T>::VEC])
+{
+    constexpr int VEC = Elem<T>::VEC, V4 = VEC / 4;
+    const uint4 *P = static_cast<const uint4 *>(plan);
+    const float4 *PA = reinterpret_cast<const float4 *>(static_cast<const uint32_t *>(plan) + C);
+    const float4 *PB = PA + C / 4;
+    const uint32_t lim = 4u * (uint32_t)C - 4u;
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int kc = 0; kc < CPT; ++kc) {
+        const int ch = tid + kc * NT;
+#pragma unroll
+        for (int q = 0; q < V4; ++q) {
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+            if (ch < NCH) {
+                uint4 pp = __ldg(P + ch * V4 + q);
+                pp.x = pbase + (min(pp.x, lim) & ~3u);
+                pp.y = pbase + (min(pp.y, lim) & ~3u);
+                pp.z = pbase + (min(pp.z, lim) & ~3u);
+                pp.w = pbase + (min(pp.w, lim) & ~3u);
+                reinterpret_cast<uint4 *>(postab)[ch * V4 + q] = pp;
+                a = __ldg(PA + ch * V4 + q);
+                b = __ldg(PB + ch * V4 + q);
+            }
+            pA[kc][4 * q + 0] = a.x, pA[kc][4 * q + 1] = a.y, pA[kc][4 * q + 2] = a.z, pA[kc][4 * q + 3] = a.w;
+            pB[kc][4 * q + 0] = b.x, pB[kc][4 * q + 1] = b.y, pB[kc][4 * q + 2] = b.z, pB[kc][4 * q + 3] = b.w;
+        }
+    }
+}
+
+// The plan: for every stored column j, channel c = R[j] of cluster k = col_cluster[j] gets
+// offset codebuf_offset(j), A = gamma_c / (s_k qmax) and B = beta_c / (s_k qmax) + z_k / qmax,
+// with the fp64 arithmetic of quant_tables_direct (so both paths give the same coefficients).
+// The plan is zeroed first; an R entry outside [0, C) is skipped, a cluster id outside [0, g)
+// uses cluster 0; both set the error word.
+template <int BITS>
+__global__ void __launch_bounds__(256)
+    ln_quant_plan_kernel(const float *__restrict__ gamma, const float *__restrict__ beta, const int32_t *__restrict__ R,
+                         const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
+                         const int32_t *__restrict__ zero, int C, int g, uint32_t *__restrict__ pos,
+                         float *__restrict__ A, float *__restrict__ B, int *err)
+{
+    constexpr double QMAX = (double)((1 << BITS) - 1);
+    for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < C; j += gridDim.x * blockDim.x) {
+        const int c = R[j];
+        int k = col_cluster[j];
+        if (k < 0 || k >= g) {
+            raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+            k = 0;
+        }
+        if (c < 0 || c >= C) {
+            raise_error(err, RPTQ_DEVERR_REORDER);
+            continue;
+        }
+        const double inv = 1.0 / ((double)scale[k] * QMAX);
+        pos[c] = codebuf_offset((uint32_t)j);
+        A[c] = (float)((double)gamma[c] * inv);
+        B[c] = (float)fma((double)beta[c], inv, (double)zero[k] / QMAX);
+    }
+}
+
 // Codes of the quad's four tokens for every channel of the thread -> one word per channel at
 // its stored position in the code buffer.  The normalised value of x is fmaf(x - sub[r], rstd[r],
 // nmr[r]) (sub = 0 except for rows with a large offset, see quad_stats); x - sub is formed by the
@@ -391,12 +459,15 @@ __host__ __device__ inline size_t direct_db_off(int C, int g) { return (direct_s
 // count (CC / VEC / CPT, the exact split) and every loop bound, row pitch and load offset are
 // constants, which removes most of the per-quad address, bound and branch instructions; the
 // launcher instantiates it for the common hidden sizes.
-template <typename T, int BITS, int CPT, int MAXT, bool DB, int CC = 0>
+// PLAN: the per-channel offsets and coefficients come from a plan (load_plan) instead of being
+// built by every CTA from R, col_cluster, s, z, gamma and beta (quant_tables_direct).
+template <typename T, int BITS, int CPT, int MAXT, bool DB, bool PLAN, int CC = 0>
 __global__ void __launch_bounds__(MAXT, 1)
     ln_quant_direct_kernel(const T *__restrict__ x, int64_t T_, int C_, const float *__restrict__ gamma,
                            const float *__restrict__ beta, float eps, const int32_t *__restrict__ R,
                            const int32_t *__restrict__ col_cluster, const float *__restrict__ scale,
-                           const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes, int *err)
+                           const int32_t *__restrict__ zero, int g, uint8_t *__restrict__ codes,
+                           const void *__restrict__ plan, int *err)
 {
     constexpr int VEC = Elem<T>::VEC;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -415,8 +486,11 @@ __global__ void __launch_bounds__(MAXT, 1)
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x);
     prefetch_quad_l2(x, T_, rowbytes, blockIdx.x + G);
     float pA[CPT][VEC], pB[CPT][VEC];
-    quant_tables_direct<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, ctab, ctl,
-                                      smem_u32(codebuf), pA, pB, err);
+    if constexpr (PLAN)
+        load_plan<T, CPT>(plan, C, NCH, NT, postab, smem_u32(codebuf), pA, pB);
+    else
+        quant_tables_direct<T, BITS, CPT>(R, col_cluster, scale, zero, gamma, beta, g, C, postab, ctab, ctl,
+                                          smem_u32(codebuf), pA, pB, err);
     uint4 xr[4][CPT];
     load_quad_direct<T, CPT>(x, T_, C, blockIdx.x, exact, xr, NT);  // the L2 prefetch above is in flight
 
@@ -541,41 +615,56 @@ __global__ void __launch_bounds__(256)
 // Host launchers
 // ------------------------------------------------------------------------------------------
 
+// The direct kernel for (C, thread split, DB, PLAN); the hidden sizes of OPT-6.7B, -66B and
+// -175B with 16-bit inputs are compiled for their exact thread split (the plan below picks
+// 512 x 1, 384 x 3 and 384 x 4 chunks).
+template <typename T, int BITS, int CPT, int MAXT, bool PLAN>
+static const void *direct_kernel_for(int C, int NT, bool db)
+{
+    const void *kern = db ? (const void *)ln_quant_direct_kernel<T, BITS, CPT, MAXT, true, PLAN>
+                          : (const void *)ln_quant_direct_kernel<T, BITS, CPT, MAXT, false, PLAN>;
+    if constexpr (sizeof(T) == 2 && CPT == 1 && MAXT == 512) {
+        if (C == 4096 && NT == 4096 / 8)
+            kern = db ? (const void *)ln_quant_direct_kernel<T, BITS, 1, 512, true, PLAN, 4096>
+                      : (const void *)ln_quant_direct_kernel<T, BITS, 1, 512, false, PLAN, 4096>;
+    }
+    if constexpr (sizeof(T) == 2 && CPT == 3 && MAXT == 384) {
+        if (C == 9216 && NT == 9216 / 8 / 3)
+            kern = db ? (const void *)ln_quant_direct_kernel<T, BITS, 3, 384, true, PLAN, 9216>
+                      : (const void *)ln_quant_direct_kernel<T, BITS, 3, 384, false, PLAN, 9216>;
+    }
+    if constexpr (sizeof(T) == 2 && CPT == 4 && MAXT == 384) {
+        if (C == 12288 && NT == 12288 / 8 / 4)
+            kern = db ? (const void *)ln_quant_direct_kernel<T, BITS, 4, 384, true, PLAN, 12288>
+                      : (const void *)ln_quant_direct_kernel<T, BITS, 4, 384, false, PLAN, 12288>;
+    }
+    return kern;
+}
+
 template <typename T, int BITS, int CPT, int MAXT>
 static cudaError_t launch_direct_t(const LnQuantArgs &a, int NT)
 {
     // two code buffers (one barrier per quad) whenever they fit: with the thread split fixed at
     // compile time, bf16 A3 measured 0.685 -> 0.706 of the HBM copy rate at C = 12288 (one
     // buffer was faster there with a runtime split) and 0.59 -> 0.62 at C = 9216
-    const size_t db_smem = direct_db_off(a.C, a.g) + (size_t)4 * a.C;
+    const int g = a.plan ? 0 : a.g;  // a planned launch keeps no cluster table in shared memory
+    const size_t db_smem = direct_db_off(a.C, g) + (size_t)4 * a.C;
     const bool db = db_smem <= (size_t)a.max_smem;
-    const size_t smem = db ? db_smem : direct_smem_bytes(a.C, a.g);
-    auto kern = db ? ln_quant_direct_kernel<T, BITS, CPT, MAXT, true> : ln_quant_direct_kernel<T, BITS, CPT, MAXT, false>;
-    // the hidden sizes of OPT-6.7B, -66B and -175B with 16-bit inputs, compiled for their exact
-    // thread split (the plan below picks 512 x 1, 384 x 3 and 384 x 4 chunks)
-    if constexpr (sizeof(T) == 2 && CPT == 1 && MAXT == 512) {
-        if (a.C == 4096 && NT == 4096 / 8)
-            kern = db ? ln_quant_direct_kernel<T, BITS, 1, 512, true, 4096> : ln_quant_direct_kernel<T, BITS, 1, 512, false, 4096>;
-    }
-    if constexpr (sizeof(T) == 2 && CPT == 3 && MAXT == 384) {
-        if (a.C == 9216 && NT == 9216 / 8 / 3)
-            kern = db ? ln_quant_direct_kernel<T, BITS, 3, 384, true, 9216> : ln_quant_direct_kernel<T, BITS, 3, 384, false, 9216>;
-    }
-    if constexpr (sizeof(T) == 2 && CPT == 4 && MAXT == 384) {
-        if (a.C == 12288 && NT == 12288 / 8 / 4)
-            kern = db ? ln_quant_direct_kernel<T, BITS, 4, 384, true, 12288> : ln_quant_direct_kernel<T, BITS, 4, 384, false, 12288>;
-    }
-    cudaError_t e = kernel_smem((const void *)kern, smem);
+    const size_t smem = db ? db_smem : direct_smem_bytes(a.C, g);
+    const void *kern = a.plan ? direct_kernel_for<T, BITS, CPT, MAXT, true>(a.C, NT, db)
+                              : direct_kernel_for<T, BITS, CPT, MAXT, false>(a.C, NT, db);
+    cudaError_t e = kernel_smem(kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = kernel_occupancy(&per_sm, (const void *)kern, NT, smem);
+    e = kernel_occupancy(&per_sm, kern, NT, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const int64_t quads = (a.T + 3) / 4;
     const int64_t grid = std::min<int64_t>(quads, (int64_t)per_sm * a.num_sms);
-    kern<<<(unsigned)grid, NT, smem, a.stream>>>((const T *)a.x, a.T, a.C, a.gamma, a.beta, a.eps, a.R,
-                                                 a.col_cluster, a.scale, a.zero, a.g, a.codes, a.err);
-    return cudaGetLastError();
+    void *args[] = {(void *)&a.x,     (void *)&a.T,     (void *)&a.C,     (void *)&a.gamma, (void *)&a.beta,
+                    (void *)&a.eps,   (void *)&a.R,     (void *)&a.col_cluster, (void *)&a.scale,
+                    (void *)&a.zero,  (void *)&a.g,     (void *)&a.codes, (void *)&a.plan,  (void *)&a.err};
+    return cudaLaunchKernel(kern, dim3((unsigned)grid), dim3(NT), args, smem, a.stream);
 }
 
 template <typename T, int BITS, int CPT>
@@ -705,6 +794,29 @@ static cudaError_t launch_simple_t(const LnQuantArgs &a)
     return cudaGetLastError();
 }
 
+cudaError_t launch_ln_quant_plan(const float *gamma, const float *beta, const int32_t *R, const int32_t *col_cluster,
+                                 const float *scale, const int32_t *zero, int C, int g, int bits, void *plan,
+                                 int *err, cudaStream_t stream)
+{
+    cudaError_t e = cudaMemsetAsync(plan, 0, (size_t)C * 12, stream);
+    if (e != cudaSuccess) return e;
+    uint32_t *pos = static_cast<uint32_t *>(plan);
+    float *A = reinterpret_cast<float *>(pos + C), *B = A + C;
+    const unsigned grid = (unsigned)((C + 255) / 256);
+    if (bits == 4)
+        ln_quant_plan_kernel<4><<<grid, 256, 0, stream>>>(gamma, beta, R, col_cluster, scale, zero, C, g, pos, A, B, err);
+    else
+        ln_quant_plan_kernel<3><<<grid, 256, 0, stream>>>(gamma, beta, R, col_cluster, scale, zero, C, g, pos, A, B, err);
+    return cudaGetLastError();
+}
+
+// Whether (C, dtype) runs on the direct kernel, the only one that takes a plan.
+bool ln_quant_plan_supported(int C, int esize, int max_smem)
+{
+    int CPT = 0, NT = 0, NS = 0, alias = 0;
+    return ln_quant_fast_plan(C, esize, max_smem, true, &CPT, &NT, &NS, &alias) && alias == 2;
+}
+
 cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple)
 {
     if (a.T == 0) return cudaSuccess;
@@ -713,7 +825,8 @@ cudaError_t launch_ln_quant(const LnQuantArgs &a, int force_simple)
     const bool vec_tables = (uintptr_t)a.R % 16 == 0 && (uintptr_t)a.col_cluster % 16 == 0 &&
                             (uintptr_t)a.gamma % 16 == 0 && (uintptr_t)a.beta % 16 == 0;
     const bool fast = !force_simple && a.ln_out == nullptr && a.codes != nullptr &&
-                      ln_quant_fast_plan(a.C, esize, a.max_smem, vec_tables, &CPT, &NT, &NS, &alias);
+                      ln_quant_fast_plan(a.C, esize, a.max_smem, vec_tables || a.plan, &CPT, &NT, &NS, &alias);
+    if (a.plan && !(fast && alias == 2)) return cudaErrorInvalidValue;  // checked by the caller
     if (fast) {
         switch (a.dtype) {
         case RPTQ_F32: return launch_fast_d<float>(a, CPT, NT, NS, alias);

@@ -52,6 +52,9 @@ SIGNATURES = {
     "rptq_cluster_params": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_decode_attention": (_I, [_P, _I, _I, _I, _P, _P, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _F, _P, _P]),
+    "rptq_ln_quant_plan_bytes": (ctypes.c_size_t, [_I]),
+    "rptq_ln_quant_plan": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
+    "rptq_ln_reorder_quant_planned": (_I, [_P, _I, _I64, _I, _F, _P, _I, _P, _P]),
     "rptq_linear_prepare": (_I, [_P, _P, _I, _I, _P, _P, _P, _P, _I, _P, _P, _P, _P]),
     "rptq_reordered_linear": (_I, [_P, _I64, _I, _I, _P, _P, _P, _P, _I, _P, _P]),
     # include/rptq_baseline.h
@@ -291,6 +294,34 @@ def rptq_kv_decode_attention(q, k_cache, v_cache, L: int, cluster_k, scale_k, ze
                                         _ptr(out), _stream(stream))
     _check(st, "rptq_kv_decode_attention")
     return out
+
+
+def rptq_ln_quant_plan_bytes(C: int) -> int:
+    """Bytes of the LayerNorm plan for C channels."""
+    return int(lib().rptq_ln_quant_plan_bytes(C))
+
+
+def rptq_ln_quant_plan(gamma, beta, R, col_cluster, scale, zero, bits: int, plan=None, stream=None):
+    """The per-channel plan (code-buffer offsets and LayerNorm-quantization coefficients) of one
+    calibration; returns the uint8 plan buffer."""
+    C = R.numel()
+    if plan is None:
+        plan = torch.empty(rptq_ln_quant_plan_bytes(C), dtype=torch.uint8, device=R.device)
+    st = lib().rptq_ln_quant_plan(_ptr(gamma), _ptr(beta), _ptr(R), _ptr(col_cluster), _ptr(scale), _ptr(zero), C,
+                                  scale.numel(), bits, _ptr(plan), _stream(stream))
+    _check(st, "rptq_ln_quant_plan")
+    return plan
+
+
+def rptq_ln_reorder_quant_planned(x: torch.Tensor, plan, bits: int, eps: float = 1e-5, codes=None, stream=None):
+    """Packed cluster-ordered codes of x [T, C] from a plan (rptq_ln_quant_plan)."""
+    T, C = x.shape
+    if codes is None:
+        codes = torch.empty((T, C * bits // 8), dtype=torch.uint8, device=x.device)
+    st = lib().rptq_ln_reorder_quant_planned(_ptr(x), _DT[x.dtype], T, C, eps, _ptr(plan), bits, _ptr(codes),
+                                             _stream(stream))
+    _check(st, "rptq_ln_reorder_quant_planned")
+    return codes
 
 
 def rptq_linear_prepare(w_codes, w_zero, R, col_cluster, scale, zero, w_prep=None, w_bias=None, w_lambda=None,

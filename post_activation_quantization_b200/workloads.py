@@ -93,6 +93,12 @@ def bytes_ln_quant(T: int, C: int, dtype: str, bits: int, ln_out: bool = False) 
     return b
 
 
+def bytes_ln_quant_plan(C: int) -> int:
+    """The LayerNorm plan of one calibration: read gamma, beta, R, col_cluster (4 bytes each per
+    channel), write the offset and two coefficients per channel."""
+    return 16 * C + 12 * C
+
+
 def bytes_kv_quant(n_elems: int, dtype: str, bits: int, tensors: int = 2) -> int:
     """K and V quant: read each element, write its packed code."""
     return tensors * (n_elems * ESIZE[dtype] + n_elems * bits // 8)
