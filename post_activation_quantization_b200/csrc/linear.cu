@@ -168,9 +168,17 @@ __global__ void __launch_bounds__(LP_THREADS)
         zd[k] = (double)zero[k];
     }
     const int groups = C / 8;
+    // a row's packed codes are C / 32 16-byte pieces, at most one per thread; the next row's piece
+    // is loaded into a register while this row is processed
+    static_assert(RPTQ_MAX_CHANNELS / 32 <= LP_THREADS, "one 16-byte piece of a row per thread");
+    const int nv = C / 32;
+    uint4 pre = make_uint4(0u, 0u, 0u, 0u);
+    if (blockIdx.x < N && tid < nv)
+        pre = __ldg(reinterpret_cast<const uint4 *>(qw + (int64_t)blockIdx.x * (C / 2)) + tid);
     for (int n = blockIdx.x; n < N; n += gridDim.x) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(qw + (int64_t)n * (C / 2));
-        for (int i = tid; i < C / 32; i += LP_THREADS) reinterpret_cast<uint4 *>(qrow)[i] = __ldg(src + i);
+        if (tid < nv) reinterpret_cast<uint4 *>(qrow)[tid] = pre;
+        if (n + (int)gridDim.x < N && tid < nv)
+            pre = __ldg(reinterpret_cast<const uint4 *>(qw + (int64_t)(n + gridDim.x) * (C / 2)) + tid);
         __syncthreads();  // the row (and, the first time, the tables) are in place
         const int zwi = zw[n];
         // q - z_w as a float: exactly (2^23 + q) - (2^23 + z_w) while |z_w| < 2^22, else a conversion
