@@ -407,14 +407,14 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) wa[i] = wb[i], wb[i] = wc[i];
         }
-        // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, columns 128 (w / 4) .. +127 ----
+        // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, the (w / 4)-th half of the columns ----
         if (ok) ok = mbar_wait_bounded(done, 0, err);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective: the whole warp or none
         tc_fence_after();
         if (ok) {
             const int64_t row = m0 + r;
-            for (int i = 0; i < 4; ++i) {
-                const int col0 = par * 128 + 32 * i;
+            for (int i = 0; i < LIN_BN / 64; ++i) {
+                const int col0 = par * (LIN_BN / 2) + 32 * i;
                 uint32_t v[32];
                 tc_ld32(tmem + ((uint32_t)(32 * qd) << 16) + (uint32_t)col0, v);
                 if (row >= T || n0 + col0 >= N) continue;
