@@ -59,6 +59,10 @@ def test_fused_quant_full_size_sampled_rows(name):
     ref, _, _ = oracle.ln_reorder_quant(xs, gamma, beta, cal["R"], cal["col_cluster"], cal["scale"],
                                         cal["zero"], w.bits, eps=w.eps)
     compare_codes(to_np(codes[ri]), ref, w.C, w.bits, name)
+    # the planned launch the bench reports, on the same batch: every byte equal
+    plan = rptq.rptq_ln_quant_plan(gamma.to(DEV), beta.to(DEV), p["R"], p["col_cluster"], p["scale"], p["zero"],
+                                   w.bits)
+    assert torch.equal(rptq.rptq_ln_reorder_quant_planned(x, plan, w.bits, eps=w.eps), codes), name
 
 
 @pytest.mark.parametrize("name", [n for n in ACT if WORKLOADS[n].T_cal])

@@ -147,11 +147,12 @@ def test_full_shape_sampled(bits):
     assert np.isfinite(Y).all()
 
 
-def test_bench_shape_sampled():
-    """The OPT-175B-shaped layer the bench step runs: 2048 tokens x 12288 channels of A3 codes
-    into the 36864-wide Q/K/V projection, with the bench's synthetic 4-bit weight codes; 64 x 64
-    sampled outputs (the last token and output included)."""
-    T, C, N, g, bits = 2048, 12288, 36864, 64, 3
+@pytest.mark.parametrize("C,g", [(12288, 64), (9216, 64)])
+def test_bench_shape_sampled(C, g):
+    """The layers the bench step runs for the OPT-175B- and OPT-66B-shaped workloads: 2048 tokens
+    of A3 codes into the 3C-wide Q/K/V projection, with the bench's synthetic 4-bit weight codes;
+    64 x 64 sampled outputs (the last token and output included)."""
+    T, N, bits = 2048, 3 * C, 3
     cal, codes, _, _, _ = _case(T, C, 8, g, bits, 31)
     wq, sw_t, zw_t = synthetic.weight_codes(N, C, 31)
     p = dev_params(cal)
@@ -167,7 +168,7 @@ def test_bench_shape_sampled():
     Ys, wps, wbs, wls = to_np(Y[:, ci]), to_np(w_prep[ci]), to_np(w_bias[ci]), to_np(w_lam[ci])
     qws = oracle.unpack(wq.numpy()[cols], C, 4)
     _check(Ys, wps, wbs, wls, cal, codes, qws, sw_t.numpy()[cols], zw_t.numpy()[cols], C, bits,
-           "linear bench shape A3 (sampled)", rows)
+           f"linear bench shape C={C} A3 (sampled)", rows)
 
 
 def test_no_tokens_and_refused_shapes():
