@@ -349,7 +349,7 @@ int rptq_linear_prepare(const uint8_t *w_codes, const int32_t *w_zero, int N, in
  *   out       fp32 [T, N].
  * The codes go to the tensor core as exact fp16 integers and the products are accumulated in
  * fp32 (tcgen05.mma kind::f16, 128 x 256 output tiles).  C a multiple of 64 in
- * [64, RPTQ_MAX_CHANNELS], N in [1, 2^24].  T == 0 is valid: nothing is launched.  A bounded
+ * [64, RPTQ_MAX_CHANNELS], N in [1, 65535 * 256].  T == 0 is valid: nothing is launched.  A bounded
  * wait that runs out sets RPTQ_DEVERR_TIMEOUT (the output is then undefined).
  */
 int rptq_reordered_linear(const uint8_t *codes, int64_t T, int C, int bits, const void *w_prep,

@@ -302,12 +302,13 @@ int rptq_ln_reorder_quant_planned(const void *x, int dtype, int64_t T, int C, fl
     if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
     if (C <= 0 || C % 8 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
     if (T < 0 || !(eps >= 0.0f) || !plan || !aligned16(plan)) return RPTQ_ERR_INVALID_ARG;
+    if (C % 32 != 0) return RPTQ_ERR_UNSUPPORTED;  // no direct kernel, so no planned launch
+    if (T == 0) return RPTQ_OK;
+    if (!x || !codes || !aligned16(x) || !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
     if (!ln_quant_plan_supported(C, esize(dtype), d.max_smem)) return RPTQ_ERR_UNSUPPORTED;
-    if (T == 0) return RPTQ_OK;
-    if (!x || !codes || !aligned16(x) || !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
     LnQuantArgs a{x, dtype, T, C, nullptr, nullptr, eps, nullptr, nullptr, nullptr, nullptr, 0, bits, codes,
                   nullptr, d.err, (cudaStream_t)stream, d.num_sms, d.max_smem, plan};
     return cuda_status(launch_ln_quant(a, 0));
@@ -445,7 +446,7 @@ int rptq_reordered_linear(const uint8_t *codes, int64_t T, int C, int bits, cons
 {
     if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
     if (C < 64 || C % 64 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
-    if (T < 0 || N < 1 || N > (1 << 24)) return RPTQ_ERR_INVALID_ARG;
+    if (T < 0 || N < 1 || N > 65535 * 256) return RPTQ_ERR_INVALID_ARG;  // output tiles of 256 columns
     if (!w_prep || !w_bias || !w_lambda || !w_scale || !aligned16(w_prep)) return RPTQ_ERR_INVALID_ARG;
     if (T == 0) return RPTQ_OK;
     if (!codes || !out || !aligned16(codes) || !aligned16(out)) return RPTQ_ERR_INVALID_ARG;

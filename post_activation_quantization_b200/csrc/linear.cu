@@ -493,16 +493,16 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda).
 static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static bool looked = false;
-    if (!looked) {
+    // looked up once per process (a function-local static is initialised exactly once, also when
+    // several host threads call at the same time)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        looked = true;
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    }();
     return fn;
 }
 

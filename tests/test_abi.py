@@ -85,6 +85,15 @@ def test_host_validation_rejects_before_any_launch(rlib):
                               fake, fake, None) == -1
     # dequant: bad layout
     assert rlib.rptq_dequant(fake, 5, 4, 64, 0, 0, fake, fake, fake, 8, 3, fake, 0, None) == -1
+    # LayerNorm plan: bad bits, no plan buffer; planned launch: C not a multiple of 32
+    assert rlib.rptq_ln_quant_plan(fake, fake, fake, fake, fake, fake, 64, 8, 5, fake, None) == -2
+    assert rlib.rptq_ln_quant_plan(fake, fake, fake, fake, fake, fake, 64, 8, 3, None, None) == -1
+    assert rlib.rptq_ln_reorder_quant_planned(fake, 2, 4, 40, 1e-5, fake, 3, fake, None) == -2
+    # linear layer: C not a multiple of 64, no rows of weights, bad bits, too many outputs
+    assert rlib.rptq_linear_prepare(fake, fake, 8, 96, fake, fake, fake, fake, 4, fake, fake, fake, None) == -2
+    assert rlib.rptq_linear_prepare(fake, fake, 0, 128, fake, fake, fake, fake, 4, fake, fake, fake, None) == -1
+    assert rlib.rptq_reordered_linear(fake, 4, 128, 5, fake, fake, fake, fake, 8, fake, None) == -2
+    assert rlib.rptq_reordered_linear(fake, 4, 128, 3, fake, fake, fake, fake, 65535 * 256 + 1, fake, None) == -1
     assert rlib.rptq_device_error(None, None) == -1
 
 
@@ -104,6 +113,9 @@ def test_empty_problems_succeed_on_the_host(rlib):
     # n0 = 0 rows; S = 0 positions of a BHSD cache
     assert rlib.rptq_dequant(None, 0, 0, 64, 0, 0, fake, fake, fake, 8, 3, None, 0, None) == 0
     assert rlib.rptq_dequant(None, 1, 2, 3, 0, 64, fake, fake, fake, 8, 3, None, 0, None) == 0
+    # T = 0 tokens through the planned launch and the linear layer
+    assert rlib.rptq_ln_reorder_quant_planned(None, 2, 0, 64, 1e-5, fake, 3, None, None) == 0
+    assert rlib.rptq_reordered_linear(None, 0, 128, 3, fake, fake, fake, fake, 8, None, None) == 0
     # ... but an empty problem with an invalid shape is still refused
     assert rlib.rptq_ln_reorder_quant(None, 2, 0, 60, fake, fake, 1e-5, fake, fake, fake, fake, 8, 3,
                                       None, None, None) == -2
