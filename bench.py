@@ -663,37 +663,72 @@ def workload_config(w):
     return c
 
 
+E2E_CHUNKS = 8
+
+
 def run_e2e(step: Step, args, dev, ws):
     """The headline call through the public API with host buffers: every step copies its input
     from pinned host memory, runs the call, and reads its codes back, all inside the timing
-    (the calibration results of the timed steps are the call's tables)."""
+    (the calibration results of the timed steps are the call's tables).  The batch goes in
+    E2E_CHUNKS chunks (token rows, or whole batch entries of the K/V cache) over three streams --
+    upload, the call on the chunk, readback -- so the upload of one chunk overlaps the readback of
+    the one before (the host link is full duplex); every byte still crosses the link once per
+    step."""
     r, w = step.r, step.w
+    main = torch.cuda.current_stream(dev)
     if step.act:
         ins, outs = [step.x], [step.codes]
-
-        def call():
-            r.rptq_ln_reorder_quant_planned(step.x, step.plan, w.bits, eps=w.eps, codes=step.codes)
+        T = w.T
+        nch = max(1, min(E2E_CHUNKS, T // 4))
+        bounds = [(T * i // nch) // 4 * 4 for i in range(nch)] + [T]
     else:
         k = step.kvw
         ins, outs = [step.k, step.v], [step.kq, step.vq]
-
-        def call():
-            r.rptq_kv_quant(step.k, step.v, step.kmk["labels"], step.kmk["scale"], step.kmk["zero"],
-                            step.kmv["labels"], step.kmv["scale"], step.kmv["zero"], k.bits,
-                            k_codes=step.kq, v_codes=step.vq)
+        nch = max(1, min(E2E_CHUNKS, k.B))  # chunks of whole batch entries
+        bounds = [k.B * i // nch for i in range(nch)] + [k.B]
     h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
     for h, t in zip(h_in, ins):
         h.copy_(t)
     h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     bi = sum(t.numel() * t.element_size() for t in ins)
     bo = sum(t.numel() * t.element_size() for t in outs)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(nch)]
+    ev_k = [torch.cuda.Event() for _ in range(nch)]
+    ev_out = [torch.cuda.Event() for _ in range(nch)]
+    for e in ev_in + ev_k + ev_out:  # every event recorded once, so the first waits are valid
+        e.record(main)
+
+    def call(t0, t1):
+        if step.act:
+            r.rptq_ln_reorder_quant_planned(step.x[t0:t1], step.plan, w.bits, eps=w.eps, codes=step.codes[t0:t1])
+        else:
+            r.rptq_kv_quant(step.k[t0:t1], step.v[t0:t1], step.kmk["labels"], step.kmk["scale"], step.kmk["zero"],
+                            step.kmv["labels"], step.kmv["scale"], step.kmv["zero"], k.bits,
+                            k_codes=step.kq[t0:t1], v_codes=step.vq[t0:t1])
 
     def one():
-        for h, t in zip(h_in, ins):
-            t.copy_(h, non_blocking=True)
-        call()
-        for h, t in zip(h_out, outs):
-            h.copy_(t, non_blocking=True)
+        for c in range(nch):
+            t0, t1 = bounds[c], bounds[c + 1]
+            if t1 == t0:
+                continue
+            # upload: the chunk's rows are free once the previous step's call on them is done
+            s_in.wait_event(ev_k[c])
+            with torch.cuda.stream(s_in):
+                for h, t in zip(h_in, ins):
+                    t[t0:t1].copy_(h[t0:t1], non_blocking=True)
+            ev_in[c].record(s_in)
+            # the call: after the upload, and after the previous readback of the chunk's codes
+            main.wait_event(ev_in[c])
+            main.wait_event(ev_out[c])
+            call(t0, t1)
+            ev_k[c].record(main)
+            # readback
+            s_out.wait_event(ev_k[c])
+            with torch.cuda.stream(s_out):
+                for h, t in zip(h_out, outs):
+                    h[t0:t1].copy_(t[t0:t1], non_blocking=True)
+            ev_out[c].record(s_out)
 
     one()
     torch.cuda.synchronize()
@@ -701,16 +736,22 @@ def run_e2e(step: Step, args, dev, ws):
     if ws > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    a.record()
+    a.record(main)
+    s_in.wait_stream(main)
+    s_out.wait_stream(main)
     for _ in range(args.e2e_steps):
         one()
-    b.record()
+    main.wait_stream(s_in)
+    main.wait_stream(s_out)
+    b.record(main)
     torch.cuda.synchronize()
     ms = pdist.max_over_ranks(a.elapsed_time(b), dev)
     nbytes = stage_bytes(w, headline_stage(w))
     total = pdist.sum_over_ranks(nbytes * args.e2e_steps, dev)
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "steps": args.e2e_steps,
-            "what": f"{headline_stage(w)} through the C ABI with host buffers",
+            "what": (f"{headline_stage(w)} through the C ABI with host buffers"
+                     + (f", {nch} chunks ({'tokens' if step.act else 'batch entries'}) pipelined over upload / call / "
+                        "readback streams" if nch > 1 else "")),
             "ms_per_step": round(ms / args.e2e_steps, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
 
