@@ -434,7 +434,7 @@ int rptq_linear_prepare(const uint8_t *w_codes, const int32_t *w_zero, int N, in
     DevInfo d;
     int st = dev_info(&d);
     if (st) return st;
-    if ((size_t)C * 8 + (size_t)g * 16 + (size_t)C / 2 + 32 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
+    if ((size_t)C * 4 + (size_t)g * 12 + (size_t)4 * (C / 2 + 16) + 16 > (size_t)d.max_smem) return RPTQ_ERR_UNSUPPORTED;
     LinPrepArgs a{w_codes, w_zero, R, col_cluster, scale, zero, g, C, N,
                   static_cast<__half *>(w_prep), w_bias, w_lambda, d.err, (cudaStream_t)stream, d.num_sms};
     return cuda_status(launch_linear_prepare(a));

@@ -119,18 +119,20 @@ __host__ __device__ constexpr uint32_t f16_idesc(int M, int N)
 __host__ __device__ __forceinline__ int lin_column(int js) { return (js & ~7) | ((js & 1) << 2) | ((js >> 1) & 3); }
 
 // ---- offline preparation ----------------------------------------------------------------------
-// Persistent CTAs over the output rows.  Each CTA first builds, in shared memory, the table of
-// stored column js -> (R[j] | k(j) << 16), j = lin_column(js), k = col_cluster[j] (range-checked
-// once), and the per-cluster s_k and z_k (the latter as double); then per row n: the row's packed
-// codes are staged in shared memory (16-byte loads), a first pass computes b[n][js] into shared
-// memory and max |b|, a second scales by the exact power of two 1 / lam[n], rounds pairs to fp16,
-// writes B in 16-byte stores (one group of 8 stored columns per thread and step) and sums z_k B
-// in fp64.
-constexpr int LP_THREADS = 512;
+// Persistent CTAs, LP_ROWS output rows per iteration, one group of LP_GROUP threads per row.  Each
+// CTA first builds, in shared memory, the table of stored column js -> (R[j] | k(j) << 16),
+// j = lin_column(js), k = col_cluster[j] (range-checked once), and the per-cluster s_k and z_k (the
+// latter as double).  Per iteration: the rows' packed codes are staged in shared memory (the next
+// iteration's are loaded into registers meanwhile); a first pass finds max_j |b[n][j]| of each row
+// and its lam[n]; a second recomputes b, scales it by the exact power of two 1 / lam[n], rounds
+// pairs to fp16, writes B in 16-byte stores (one group of 8 stored columns per thread and step)
+// and sums z_k B in fp64.  Three CTA barriers serve LP_ROWS rows.
+constexpr int LP_THREADS = 512, LP_ROWS = 4, LP_GROUP = LP_THREADS / LP_ROWS;
+constexpr int LP_PIECES = (RPTQ_MAX_CHANNELS / 32 + LP_GROUP - 1) / LP_GROUP;  // 16-byte pieces per thread and row
 
 __host__ __device__ inline size_t lp_smem_bytes(int C, int g)
 {
-    return (size_t)C * 8 + (size_t)g * 16 + (((size_t)C / 2 + 15) & ~(size_t)15) + 16;
+    return (size_t)g * 8 + (size_t)C * 4 + (size_t)g * 4 + (size_t)LP_ROWS * (((size_t)C / 2 + 15) & ~(size_t)15) + 16;
 }
 
 __global__ void __launch_bounds__(LP_THREADS)
@@ -140,15 +142,16 @@ __global__ void __launch_bounds__(LP_THREADS)
                           float *__restrict__ bz, float *__restrict__ lam, int *err)
 {
     extern __shared__ __align__(16) uint8_t lp_smem[];
-    double *zd = reinterpret_cast<double *>(lp_smem);         // g
-    uint32_t *tab = reinterpret_cast<uint32_t *>(zd + g);     // C entries, stored order
-    float *bv = reinterpret_cast<float *>(tab + C);           // C: b of the current row
-    float *sc = bv + C;                                       // g
-    uint8_t *qrow = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sc + g) + 15) & ~(uintptr_t)15);
-    __shared__ float smax[LP_THREADS / 32];
-    __shared__ double ssum[LP_THREADS / 32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    constexpr int NW = LP_THREADS / 32;
+    double *zd = reinterpret_cast<double *>(lp_smem);      // g
+    uint32_t *tab = reinterpret_cast<uint32_t *>(zd + g);  // C entries, stored order
+    float *sc = reinterpret_cast<float *>(tab + C);        // g
+    const size_t rowb = ((size_t)C / 2 + 15) & ~(size_t)15;
+    uint8_t *qrows = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(sc + g) + 15) & ~(uintptr_t)15);
+    __shared__ float smax[LP_ROWS][LP_GROUP / 32];
+    __shared__ double ssum[LP_ROWS][LP_GROUP / 32];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int rg = tid / LP_GROUP, t = tid % LP_GROUP, gw = t >> 5;  // row group, thread and warp in it
+    constexpr int NW = LP_GROUP / 32;
 
     for (int js = tid; js < C; js += LP_THREADS) {
         const int j = lin_column(js);
@@ -167,83 +170,89 @@ __global__ void __launch_bounds__(LP_THREADS)
         sc[k] = scale[k];
         zd[k] = (double)zero[k];
     }
-    const int groups = C / 8;
-    // a row's packed codes are C / 32 16-byte pieces, at most one per thread; the next row's piece
-    // is loaded into a register while this row is processed
-    static_assert(RPTQ_MAX_CHANNELS / 32 <= LP_THREADS, "one 16-byte piece of a row per thread");
-    const int nv = C / 32;
-    uint4 pre = make_uint4(0u, 0u, 0u, 0u);
-    if (blockIdx.x < N && tid < nv)
-        pre = __ldg(reinterpret_cast<const uint4 *>(qw + (int64_t)blockIdx.x * (C / 2)) + tid);
-    for (int n = blockIdx.x; n < N; n += gridDim.x) {
-        if (tid < nv) reinterpret_cast<uint4 *>(qrow)[tid] = pre;
-        if (n + (int)gridDim.x < N && tid < nv)
-            pre = __ldg(reinterpret_cast<const uint4 *>(qw + (int64_t)(n + gridDim.x) * (C / 2)) + tid);
-        __syncthreads();  // the row (and, the first time, the tables) are in place
-        const int zwi = zw[n];
+    const int groups = C / 8, nv = C / 32;
+    uint8_t *qrow = qrows + (size_t)rg * rowb;
+    const int64_t stride = (int64_t)gridDim.x * LP_ROWS;
+    // the codes of row n0 + rg: LP_PIECES 16-byte pieces per thread (zero past the row)
+    uint4 pre[LP_PIECES];
+    auto fetch = [&](int64_t n0) {
+        const int64_t n = n0 + rg;
+#pragma unroll
+        for (int i = 0; i < LP_PIECES; ++i) {
+            const int v = t + i * LP_GROUP;
+            pre[i] = (n < N && v < nv) ? __ldg(reinterpret_cast<const uint4 *>(qw + n * (C / 2)) + v)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    fetch((int64_t)blockIdx.x * LP_ROWS);
+    for (int64_t n0 = (int64_t)blockIdx.x * LP_ROWS; n0 < N; n0 += stride) {
+#pragma unroll
+        for (int i = 0; i < LP_PIECES; ++i) {
+            const int v = t + i * LP_GROUP;
+            if (v < nv) reinterpret_cast<uint4 *>(qrow)[v] = pre[i];
+        }
+        fetch(n0 + stride);  // the next iteration's rows, while this one is processed
+        __syncthreads();     // the rows (and, the first time, the tables) are in place
+        const int64_t n = n0 + rg;
+        const bool live = n < N;
+        const int zwi = live ? zw[n] : 0;
         // q - z_w as a float: exactly (2^23 + q) - (2^23 + z_w) while |z_w| < 2^22, else a conversion
         const bool magic = zwi > -(1 << 22) && zwi < (1 << 22);
         const float base = 8388608.0f + (float)zwi;
+        // b = RN(s_k (q - z_w)) of the stored column whose table entry is e
+        auto bval = [&](uint32_t e) -> float {
+            const uint32_t c = e & 0xFFFFu;
+            const int q = (qrow[c >> 1] >> ((c & 1) * 4)) & 15;
+            const float d = magic ? __int_as_float(0x4B000000 | q) - base : (float)(q - zwi);
+            return sc[e >> 16] * d;
+        };
         float m = 0.f;
-        for (int gi = tid; gi < groups; gi += LP_THREADS) {
+        for (int gi = t; gi < groups; gi += LP_GROUP) {
             const uint4 t0 = reinterpret_cast<const uint4 *>(tab)[2 * gi];
             const uint4 t1 = reinterpret_cast<const uint4 *>(tab)[2 * gi + 1];
-            const uint32_t t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t c = t[e] & 0xFFFFu;
-                const int q = (qrow[c >> 1] >> ((c & 1) * 4)) & 15;
-                const float d = magic ? __int_as_float(0x4B000000 | q) - base : (float)(q - zwi);
-                v[e] = sc[t[e] >> 16] * d;  // b = RN(s_k (q - z_w))
-                m = fmaxf(m, fabsf(v[e]));
-            }
-            reinterpret_cast<float4 *>(bv)[2 * gi] = make_float4(v[0], v[1], v[2], v[3]);
-            reinterpret_cast<float4 *>(bv)[2 * gi + 1] = make_float4(v[4], v[5], v[6], v[7]);
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bval(t0.x)), fabsf(bval(t0.y))), fmaxf(fabsf(bval(t0.z)), fabsf(bval(t0.w)))));
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(bval(t1.x)), fabsf(bval(t1.y))), fmaxf(fabsf(bval(t1.z)), fabsf(bval(t1.w)))));
         }
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-        if (lane == 0) smax[warp] = m;
+        if (lane == 0) smax[rg][gw] = m;
         __syncthreads();
-        m = smax[0];
+        m = smax[rg][0];
 #pragma unroll
-        for (int w = 1; w < NW; ++w) m = fmaxf(m, smax[w]);
+        for (int w = 1; w < NW; ++w) m = fmaxf(m, smax[rg][w]);
         // lam = 2^(e - 14) with m in [2^e, 2^(e+1)): the largest |B| lies in [2^14, 2^15)
-        int e = 0;
-        if (m > 0.f) frexpf(m, &e);
-        const float l = m > 0.f ? ldexpf(1.f, e - 1 - 14) : 1.f;
-        const float rl = m > 0.f ? ldexpf(1.f, 15 - e) : 1.f;  // 1 / l, exact
+        int ex = 0;
+        if (m > 0.f) frexpf(m, &ex);
+        const float l = m > 0.f ? ldexpf(1.f, ex - 1 - 14) : 1.f;
+        const float rl = m > 0.f ? ldexpf(1.f, 15 - ex) : 1.f;  // 1 / l, exact
         double acc = 0.0;
-        uint4 *dst = reinterpret_cast<uint4 *>(B + (int64_t)n * C);
-        for (int gi = tid; gi < groups; gi += LP_THREADS) {
+        uint4 *dst = reinterpret_cast<uint4 *>(B + (live ? n : 0) * (int64_t)C);
+        for (int gi = t; gi < groups && live; gi += LP_GROUP) {
             const uint4 t0 = reinterpret_cast<const uint4 *>(tab)[2 * gi];
             const uint4 t1 = reinterpret_cast<const uint4 *>(tab)[2 * gi + 1];
-            const float4 v0 = reinterpret_cast<const float4 *>(bv)[2 * gi];
-            const float4 v1 = reinterpret_cast<const float4 *>(bv)[2 * gi + 1];
-            const uint32_t t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-            const float v[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            const uint32_t te[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
             uint32_t h[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
                 // b / l = b * (1 / l) exactly (powers of two), then one rounding to fp16
-                const __half2 hh = __floats2half2_rn(v[2 * p] * rl, v[2 * p + 1] * rl);
+                const __half2 hh = __floats2half2_rn(bval(te[2 * p]) * rl, bval(te[2 * p + 1]) * rl);
                 const float2 f = __half22float2(hh);
-                acc = fma(zd[t[2 * p] >> 16], (double)f.x, acc);
-                acc = fma(zd[t[2 * p + 1] >> 16], (double)f.y, acc);
+                acc = fma(zd[te[2 * p] >> 16], (double)f.x, acc);
+                acc = fma(zd[te[2 * p + 1] >> 16], (double)f.y, acc);
                 h[p] = *reinterpret_cast<const uint32_t *>(&hh);
             }
             dst[gi] = make_uint4(h[0], h[1], h[2], h[3]);
         }
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-        if (lane == 0) ssum[warp] = acc;
+        if (lane == 0) ssum[rg][gw] = acc;
         __syncthreads();
-        if (tid == 0) {
+        if (t == 0 && live) {
             double tsum = 0.0;
 #pragma unroll
-            for (int w = 0; w < NW; ++w) tsum += ssum[w];
+            for (int w = 0; w < NW; ++w) tsum += ssum[rg][w];
             bz[n] = (float)tsum;
             lam[n] = l;
         }
-        __syncthreads();  // qrow, bv, smax and ssum are reused by the next row
+        __syncthreads();  // qrows, smax and ssum are reused by the next rows
     }
 }
 
@@ -256,7 +265,8 @@ cudaError_t launch_linear_prepare(const LinPrepArgs &a)
     int per_sm = 1;
     e = kernel_occupancy(&per_sm, (const void *)linear_prepare_kernel, LP_THREADS, smem);
     if (e != cudaSuccess) return e;
-    const int grid = (int)std::min<int64_t>(a.N, (int64_t)a.num_sms * std::max(1, per_sm));
+    const int64_t units = (a.N + LP_ROWS - 1) / LP_ROWS;
+    const int grid = (int)std::min<int64_t>(units, (int64_t)a.num_sms * std::max(1, per_sm));
     linear_prepare_kernel<<<grid, LP_THREADS, smem, a.stream>>>(a.qw, a.zw, a.R, a.col_cluster, a.scale, a.zero, a.g,
                                                                 a.C, a.N, a.B, a.bz, a.lam, a.err);
     return cudaGetLastError();
