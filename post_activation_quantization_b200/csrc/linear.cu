@@ -14,14 +14,16 @@
 // so that Y[t][n] = s_w[n] lam[n] (sum_j q[t][j] B[n][j] - bz[n]).  The code q itself (0..15) is
 // the A operand, exact in fp16, decoded from the packed activation codes inside the kernel.
 //
-// GEMM (rptq_reordered_linear): one CTA per 128 x 256 output tile, fp32 accumulator in tensor
-// memory (256 of the SM's 512 columns).  Eight producer warps decode a 64-column slab of codes
-// into fp16 and copy the matching B slab, both into shared memory in the 128-byte-swizzled
-// K-major layout the tensor core reads; one thread of a ninth warp issues four
-// tcgen05.mma.kind::f16 (K = 16 each) per slab and commits them to the slab's "empty" barrier;
-// four slabs are in flight.  After the last slab the producers read the accumulator back with
-// tcgen05.ld and write Y.  Every wait is bounded; a wait that runs out sets the device error
-// word, and the CTA still waits (bounded) for its issued MMAs and frees its tensor memory.
+// GEMM (rptq_reordered_linear): one CTA per 128 x 256 output tile, all 512 tensor-memory columns:
+// the fp32 accumulator (256) and a ring of six A slabs (32 columns of fp16 pairs each).  Eight
+// producer warps (0-3 the even K slabs, 4-7 the odd ones) decode a 64-column slab of their rows'
+// codes into fp16 in registers and write it to its ring slot with tcgen05.st; warp 8 copies the
+// matching 256 x 64 B slab with TMA into a six-slot shared-memory ring (128-byte swizzle, the
+// K-major layout the tensor core reads); one thread of warp 9 issues four tcgen05.mma.kind::f16
+// (K = 16 each, A from tensor memory) per slab and commits them to the slot's "empty" barrier.
+// After the last slab the producer warps read the accumulator back with tcgen05.ld and write Y.
+// Every wait is bounded; a wait that runs out sets the device error word, and the CTA still
+// waits (bounded) for its issued copies and MMAs and frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
