@@ -21,13 +21,17 @@
 // matching 256 x 64 B slab with TMA into a six-slot shared-memory ring (128-byte swizzle, the
 // K-major layout the tensor core reads); one thread of warp 9 issues four tcgen05.mma.kind::f16
 // (K = 16 each, A from tensor memory) per slab and commits them to the slot's "empty" barrier.
-// After the last slab the producer warps read the accumulator back with tcgen05.ld and write Y.
+// The codes reach the producers through a three-unit shared-memory ring that warp 8 fills by TMA
+// (two K slabs x 128 rows per box) where the row pitch allows it, else by the producers' own
+// loads.  After the last slab the producer warps read the accumulator back with tcgen05.ld and
+// write Y.
 // Every wait is bounded; a wait that runs out sets the device error word, and the CTA still
 // waits (bounded) for its issued copies and MMAs and frees its tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "launch.h"
@@ -282,6 +286,10 @@ constexpr uint32_t LIN_B_BYTES = LIN_BN * LIN_BK * 2;
 constexpr uint32_t LIN_TMEM_COLS = 512;     // the accumulator (256 columns) + the A ring (6 x 32)
 constexpr uint32_t LIN_A_COL = LIN_BN;      // A slab s at columns LIN_A_COL + 32 s
 constexpr size_t LIN_SMEM = 1024 + (size_t)LIN_STAGES * LIN_B_BYTES;
+// codes staged by TMA: a ring of units of two K slabs (128 rows x 16 BITS bytes, at most 64)
+constexpr int LIN_C_UNITS = 3;
+constexpr uint32_t LIN_C_BYTES = LIN_BM * 64;
+constexpr size_t LIN_SMEM_CTMA = LIN_SMEM + (size_t)LIN_C_UNITS * LIN_C_BYTES;
 static_assert(LIN_BK * 2 == 128, "one 128-byte swizzle row per K slab");
 static_assert(LIN_STAGES % 2 == 0, "a ring slot always holds slabs of one parity");
 static_assert(LIN_A_COL + LIN_STAGES * (LIN_BK / 2) <= LIN_TMEM_COLS, "tensor memory budget");
@@ -306,6 +314,35 @@ __device__ __forceinline__ void lin_decode8(uint32_t w, uint32_t *o)
 }
 // The 64 codes of one row and one K slab (8 groups): 32 bytes (A4) or 24 bytes (A3) at p
 // (16- resp. 8-byte aligned).  A3 group m sits in bytes 3m..3m+2; w[m] holds it in bits 0-23.
+// A3: the 24 bytes x[0..5] of one slab -> w[m] = group m in bits 0-23
+__device__ __forceinline__ void lin_unpack_a3(const uint32_t (&x)[6], uint32_t (&w)[8])
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // 12 bytes = 4 groups
+        w[4 * h + 0] = x[3 * h];
+        w[4 * h + 1] = __funnelshift_r(x[3 * h], x[3 * h + 1], 24);
+        w[4 * h + 2] = __funnelshift_r(x[3 * h + 1], x[3 * h + 2], 16);
+        w[4 * h + 3] = x[3 * h + 2] >> 8;
+    }
+}
+// the same 32 (A4) or 24 (A3) bytes from shared memory (16- resp. 8-byte aligned)
+template <int BITS>
+__device__ __forceinline__ void lin_load_slab_smem(uint32_t saddr, uint32_t (&w)[8])
+{
+    if constexpr (BITS == 4) {
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(saddr) : "memory");
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7]) : "r"(saddr + 16) : "memory");
+    } else {
+        uint32_t x[6];
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(x[2 * i]), "=r"(x[2 * i + 1]) : "r"(saddr + 8 * i)
+                         : "memory");
+        lin_unpack_a3(x, w);
+    }
+}
 template <int BITS>
 __device__ __forceinline__ void lin_load_slab(const uint8_t *p, uint32_t (&w)[8])
 {
@@ -318,13 +355,7 @@ __device__ __forceinline__ void lin_load_slab(const uint8_t *p, uint32_t (&w)[8]
         const uint2 b = __ldg(reinterpret_cast<const uint2 *>(p) + 1);
         const uint2 c = __ldg(reinterpret_cast<const uint2 *>(p) + 2);
         const uint32_t x[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {  // 12 bytes = 4 groups
-            w[4 * h + 0] = x[3 * h];
-            w[4 * h + 1] = __funnelshift_r(x[3 * h], x[3 * h + 1], 24);
-            w[4 * h + 2] = __funnelshift_r(x[3 * h + 1], x[3 * h + 2], 16);
-            w[4 * h + 3] = x[3 * h + 2] >> 8;
-        }
+        lin_unpack_a3(x, w);
     }
 }
 __device__ __forceinline__ void lin_tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar)
@@ -340,15 +371,18 @@ __device__ __forceinline__ void lin_tma_load_2d(uint32_t dst, const CUtensorMap 
 // (consecutive CTAs share one weight tile, which then comes from DRAM once), y = output tiles
 // of 256.  K = C is a multiple of 64: K / 64 slabs.  The decoded codes go straight from the
 // producers' registers into tensor memory (tcgen05.st) and the MMA reads A from there, so shared
-// memory carries only the weight slabs.
-template <int BITS>
+// memory carries only the weight slabs.  With CTMA the producers read their codes from a ring of
+// units (two K slabs x 128 rows) that warp 8 fills by TMA ahead of the weight slabs (cmap: the
+// codes [T, K BITS / 8] as bytes), instead of loading them from global memory themselves.
+template <int BITS, bool CTMA>
 __global__ void __launch_bounds__(LIN_THREADS, 1)
-    reordered_linear_kernel(const __grid_constant__ CUtensorMap wmap, const uint8_t *__restrict__ codes, int64_t T,
-                            int K, int N, const float *__restrict__ bz, const float *__restrict__ lam,
+    reordered_linear_kernel(const __grid_constant__ CUtensorMap wmap, const __grid_constant__ CUtensorMap cmap,
+                            const uint8_t *__restrict__ codes, int64_t T, int K, int N,
+                            const float *__restrict__ bz, const float *__restrict__ lam,
                             const float *__restrict__ sw, float *__restrict__ Y, int vec_store, int *err)
 {
     extern __shared__ uint8_t lin_smem_raw[];
-    __shared__ __align__(8) uint64_t bars[3 * LIN_STAGES + 1];
+    __shared__ __align__(8) uint64_t bars[3 * LIN_STAGES + 1 + 2 * LIN_C_UNITS];
     __shared__ uint32_t tmem_slot;
     __shared__ int s_abort;  // set by any role whose bounded wait ran out
     __shared__ float s_bz[LIN_BN], s_f[LIN_BN];
@@ -360,6 +394,9 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     const uint32_t sB = (smem_u32(lin_smem_raw) + 1023u) & ~1023u;  // swizzled tiles: 1024-aligned
     const uint32_t full_a = smem_u32(&bars[0]), full_b = smem_u32(&bars[LIN_STAGES]);
     const uint32_t empty = smem_u32(&bars[2 * LIN_STAGES]), done = smem_u32(&bars[3 * LIN_STAGES]);
+    const uint32_t full_c = done + 8, empty_c = full_c + 8 * LIN_C_UNITS;  // the code ring (CTMA)
+    const uint32_t sC = sB + LIN_STAGES * LIN_B_BYTES;
+    constexpr uint32_t UB = 16 * BITS;  // bytes of one row in a code unit
 
     if (tid == 0) {
         for (int s = 0; s < LIN_STAGES; ++s) {
@@ -368,6 +405,10 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
             mbar_init(empty + 8 * s, 1);
         }
         mbar_init(done, 1);
+        for (int c = 0; c < LIN_C_UNITS; ++c) {
+            mbar_init(full_c + 8 * c, 1);
+            mbar_init(empty_c + 8 * c, LIN_PROD / 32);  // one lane of each producer warp
+        }
         fence_mbar_init();
         s_abort = 0;
     }
@@ -391,34 +432,51 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         const int64_t pitch = (int64_t)K * BITS / 8;
         const uint8_t *src = codes + (row_ok ? m0 + r : 0) * pitch;
         const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + LIN_A_COL;
-        uint32_t wa[8], wb[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) wa[i] = wb[i] = 0;
-        if (row_ok && par < KT) lin_load_slab<BITS>(src + (int64_t)par * (8 * BITS), wa);
-        if (row_ok && par + 2 < KT) lin_load_slab<BITS>(src + (int64_t)(par + 2) * (8 * BITS), wb);
-        bool ok = true;
-        for (int kt = par; kt < KT; kt += 2) {
-            uint32_t wc[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) wc[i] = 0;
-            if (row_ok && kt + 4 < KT) lin_load_slab<BITS>(src + (int64_t)(kt + 4) * (8 * BITS), wc);
+        // slab kt: wait for its A slot (the whole warp agrees: tcgen05.st is warp-collective),
+        // decode, store into tensor memory, signal the MMA
+        auto put = [&](int kt, const uint32_t (&w)[8]) -> bool {
             const int s = kt % LIN_STAGES, u = kt / LIN_STAGES;
-            if (!mbar_wait_bounded(empty + 8 * s, (u & 1) ^ 1, err)) {
-                ok = false;
-                *(volatile int *)&s_abort = 1;
-                break;
-            }
+            if (!__all_sync(FULL, mbar_wait_bounded(empty + 8 * s, (u & 1) ^ 1, err))) return false;
             tc_fence_after();  // the slot's previous MMAs are complete
             uint32_t d[32];
 #pragma unroll
-            for (int gi = 0; gi < 8; ++gi) lin_decode8<BITS>(wa[gi], d + 4 * gi);
+            for (int gi = 0; gi < 8; ++gi) lin_decode8<BITS>(w[gi], d + 4 * gi);
             tc_st32(ta + 32 * s, d);
             tc_wait_st();
             tc_fence_before();
             lin_arrive(full_a + 8 * s);
+            return true;
+        };
+        bool ok = true;
+        if constexpr (CTMA) {
+            // codes from the ring: unit kt / 2, this slab's half of the row
+            for (int kt = par; kt < KT && ok; kt += 2) {
+                const int u = kt >> 1, cu = u % LIN_C_UNITS;
+                if (!(ok = __all_sync(FULL, mbar_wait_bounded(full_c + 8 * cu, (uint32_t)(u / LIN_C_UNITS) & 1, err))))
+                    break;
+                uint32_t w[8];
+                lin_load_slab_smem<BITS>(sC + cu * LIN_C_BYTES + r * UB + (kt & 1) * (UB / 2), w);
+                __syncwarp();  // every lane has read the unit before it is released
+                if (lane == 0) lin_arrive(empty_c + 8 * cu);
+                ok = put(kt, w);
+            }
+        } else {
+            uint32_t wa[8], wb[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) wa[i] = wb[i], wb[i] = wc[i];
+            for (int i = 0; i < 8; ++i) wa[i] = wb[i] = 0;
+            if (row_ok && par < KT) lin_load_slab<BITS>(src + (int64_t)par * (8 * BITS), wa);
+            if (row_ok && par + 2 < KT) lin_load_slab<BITS>(src + (int64_t)(par + 2) * (8 * BITS), wb);
+            for (int kt = par; kt < KT && ok; kt += 2) {
+                uint32_t wc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wc[i] = 0;
+                if (row_ok && kt + 4 < KT) lin_load_slab<BITS>(src + (int64_t)(kt + 4) * (8 * BITS), wc);
+                ok = put(kt, wa);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wa[i] = wb[i], wb[i] = wc[i];
+            }
         }
+        if (!ok) *(volatile int *)&s_abort = 1;
         // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, the (w / 4)-th half of the columns ----
         if (ok) ok = mbar_wait_bounded(done, 0, err);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective: the whole warp or none
@@ -451,19 +509,34 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     } else if (warp == 8) {
         // ---- weight slabs: one 256 x 64 fp16 box per slab, 128-byte swizzle, through TMA ----
         if (lane == 0) {
+            // code units (CTMA) go two units ahead of the weight slabs
+            const int units = (KT + 1) >> 1;
+            int cissued = 0;
+            auto issue_unit = [&](int u) -> bool {
+                const int cu = u % LIN_C_UNITS;
+                if (!mbar_wait_bounded(empty_c + 8 * cu, ((uint32_t)(u / LIN_C_UNITS) & 1) ^ 1, err)) return false;
+                mbar_expect_tx(full_c + 8 * cu, LIN_BM * UB);
+                lin_tma_load_2d(sC + cu * LIN_C_BYTES, &cmap, u * (int)UB, (int)m0, full_c + 8 * cu);
+                cissued = u + 1;
+                return true;
+            };
+            bool ok = true;
+            if constexpr (CTMA)
+                for (int u = 0; u < 2 && u < units && ok; ++u) ok = issue_unit(u);
             int issued = 0;
-            for (int kt = 0; kt < KT; ++kt) {
+            for (int kt = 0; kt < KT && ok; ++kt) {
+                if (CTMA && (kt & 1) == 0 && kt / 2 + 2 < units && !(ok = issue_unit(kt / 2 + 2))) break;
                 const int s = kt % LIN_STAGES, u = kt / LIN_STAGES;
-                if (!mbar_wait_bounded(empty + 8 * s, (u & 1) ^ 1, err)) {
-                    *(volatile int *)&s_abort = 1;
-                    break;
-                }
+                if (!(ok = mbar_wait_bounded(empty + 8 * s, (u & 1) ^ 1, err))) break;
                 mbar_expect_tx(full_b + 8 * s, LIN_B_BYTES);
                 lin_tma_load_2d(sB + s * LIN_B_BYTES, &wmap, kt * LIN_BK, n0, full_b + 8 * s);
                 issued = kt + 1;
             }
+            if (!ok) *(volatile int *)&s_abort = 1;
             // Nothing asynchronous may still write this CTA's shared memory when it exits: the
             // copies (their barrier phases), then the MMA commits to the last slabs' barriers.
+            for (int u = cissued > LIN_C_UNITS ? cissued - LIN_C_UNITS : 0; u < cissued; ++u)
+                mbar_wait_bounded(full_c + 8 * (u % LIN_C_UNITS), (uint32_t)(u / LIN_C_UNITS) & 1, err);
             const int first = issued > LIN_STAGES ? issued - LIN_STAGES : 0;
             for (int kt = first; kt < issued; ++kt)
                 mbar_wait_bounded(full_b + 8 * (kt % LIN_STAGES), (kt / LIN_STAGES) & 1, err);
@@ -534,14 +607,33 @@ cudaError_t launch_reordered_linear(const LinArgs &a)
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
-    const void *kern = a.bits == 4 ? (const void *)reordered_linear_kernel<4> : (const void *)reordered_linear_kernel<3>;
-    cudaError_t e = kernel_smem(kern, LIN_SMEM);
+    // the codes [T, K bits / 8] as bytes, boxes of 128 rows x one unit (two K slabs), rows past T
+    // read as zeros: where TMA can address them (row pitch a multiple of 16 bytes, row index
+    // within int32), otherwise the producers load their codes themselves
+    const int64_t pitch = (int64_t)a.C * a.bits / 8;
+    CUtensorMap cmap;
+    memset(&cmap, 0, sizeof(cmap));
+    bool ctma = pitch % 16 == 0 && a.T <= 0x7fffffffLL;
+    if (ctma) {
+        const cuuint64_t cdims[2] = {(cuuint64_t)pitch, (cuuint64_t)a.T};
+        const cuuint64_t cstrides[1] = {(cuuint64_t)pitch};
+        const cuuint32_t cbox[2] = {(cuuint32_t)(16 * a.bits), (cuuint32_t)LIN_BM};
+        ctma = encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(a.codes), cdims, cstrides, cbox,
+                      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    }
+    const void *kern = a.bits == 4 ? (ctma ? (const void *)reordered_linear_kernel<4, true>
+                                           : (const void *)reordered_linear_kernel<4, false>)
+                                   : (ctma ? (const void *)reordered_linear_kernel<3, true>
+                                           : (const void *)reordered_linear_kernel<3, false>);
+    const size_t smem = ctma ? LIN_SMEM_CTMA : LIN_SMEM;
+    cudaError_t e = kernel_smem(kern, smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)((a.T + LIN_BM - 1) / LIN_BM), (unsigned)((a.N + LIN_BN - 1) / LIN_BN));
     const int vec = (a.N % 4 == 0 && (reinterpret_cast<uintptr_t>(a.Y) & 15) == 0) ? 1 : 0;
-    void *args[] = {(void *)&map, (void *)&a.codes, (void *)&a.T,   (void *)&a.C, (void *)&a.N, (void *)&a.bz,
-                    (void *)&a.lam, (void *)&a.sw,  (void *)&a.Y, (void *)&vec, (void *)&a.err};
-    return cudaLaunchKernel(kern, grid, dim3(LIN_THREADS), args, LIN_SMEM, a.stream);
+    void *args[] = {(void *)&map,  (void *)&cmap, (void *)&a.codes, (void *)&a.T, (void *)&a.C, (void *)&a.N,
+                    (void *)&a.bz, (void *)&a.lam, (void *)&a.sw,   (void *)&a.Y, (void *)&vec, (void *)&a.err};
+    return cudaLaunchKernel(kern, grid, dim3(LIN_THREADS), args, smem, a.stream);
 }
 
 }  // namespace rptq
