@@ -280,8 +280,12 @@ cudaError_t launch_linear_prepare(const LinPrepArgs &a)
 
 // ---- the GEMM ---------------------------------------------------------------------------------
 constexpr int LIN_BM = 128, LIN_BN = 256, LIN_BK = 64, LIN_STAGES = 6;
-constexpr int LIN_PROD = 256;               // warps 0-7: A producers (0-3 even slabs, 4-7 odd), then the epilogue
-constexpr int LIN_THREADS = LIN_PROD + 64;  // warp 8: weight copies, warp 9: MMA issue + TMEM
+// A producers: LIN_GROUPS groups of 4 warps, group i taking the K slabs kt = i (mod LIN_GROUPS);
+// warps 0-7 then run the epilogue
+constexpr int LIN_GROUPS = 2;
+constexpr int LIN_PROD = 128 * LIN_GROUPS;
+constexpr int LIN_TMA_WARP = LIN_PROD / 32, LIN_MMA_WARP = LIN_TMA_WARP + 1;  // weight / code copies; MMA + TMEM
+constexpr int LIN_THREADS = LIN_PROD + 64;
 constexpr uint32_t LIN_B_BYTES = LIN_BN * LIN_BK * 2;
 constexpr uint32_t LIN_TMEM_COLS = 512;     // the accumulator (256 columns) + the A ring (6 x 32)
 constexpr uint32_t LIN_A_COL = LIN_BN;      // A slab s at columns LIN_A_COL + 32 s
@@ -291,7 +295,7 @@ constexpr int LIN_C_UNITS = 3;
 constexpr uint32_t LIN_C_BYTES = LIN_BM * 64;
 constexpr size_t LIN_SMEM_CTMA = LIN_SMEM + (size_t)LIN_C_UNITS * LIN_C_BYTES;
 static_assert(LIN_BK * 2 == 128, "one 128-byte swizzle row per K slab");
-static_assert(LIN_STAGES % 2 == 0, "a ring slot always holds slabs of one parity");
+static_assert(LIN_STAGES % LIN_GROUPS == 0, "a ring slot always holds slabs of one producer group");
 static_assert(LIN_A_COL + LIN_STAGES * (LIN_BK / 2) <= LIN_TMEM_COLS, "tensor memory budget");
 
 // fp16 pairs 1024 + q  ->  q (exact)
@@ -400,14 +404,14 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 
     if (tid == 0) {
         for (int s = 0; s < LIN_STAGES; ++s) {
-            mbar_init(full_a + 8 * s, LIN_PROD / 2);  // the 4 warps of one slab parity
+            mbar_init(full_a + 8 * s, LIN_PROD / LIN_GROUPS);  // the 4 warps of one producer group
             mbar_init(full_b + 8 * s, 1);
             mbar_init(empty + 8 * s, 1);
         }
         mbar_init(done, 1);
         for (int c = 0; c < LIN_C_UNITS; ++c) {
             mbar_init(full_c + 8 * c, 1);
-            mbar_init(empty_c + 8 * c, LIN_PROD / 32);  // one lane of each producer warp
+            mbar_init(empty_c + 8 * c, 8);  // one lane of each warp of the two groups reading the unit
         }
         fence_mbar_init();
         s_abort = 0;
@@ -417,13 +421,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         s_bz[tid] = n < N ? bz[n] : 0.f;
         s_f[tid] = n < N ? sw[n] * lam[n] : 0.f;  // lam is a power of two
     }
-    if (warp == 9) tc_alloc(smem_u32(&tmem_slot), LIN_TMEM_COLS);
+    if (warp == LIN_MMA_WARP) tc_alloc(smem_u32(&tmem_slot), LIN_TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_slot;
 
-    if (warp < 8) {
+    if (warp < LIN_PROD / 32) {
         // ---- A producers: warp w owns TMEM lanes 32 (w % 4) .. +31 (the tile's rows) and the
         //      slabs of parity w / 4; a thread decodes its row's 64 codes into 32 columns ----
         const int qd = warp & 3, par = warp >> 2;
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
         bool ok = true;
         if constexpr (CTMA) {
             // codes from the ring: unit kt / 2, this slab's half of the row
-            for (int kt = par; kt < KT && ok; kt += 2) {
+            for (int kt = par; kt < KT && ok; kt += LIN_GROUPS) {
                 const int u = kt >> 1, cu = u % LIN_C_UNITS;
                 if (!(ok = __all_sync(FULL, mbar_wait_bounded(full_c + 8 * cu, (uint32_t)(u / LIN_C_UNITS) & 1, err))))
                     break;
@@ -465,19 +469,23 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) wa[i] = wb[i] = 0;
             if (row_ok && par < KT) lin_load_slab<BITS>(src + (int64_t)par * (8 * BITS), wa);
-            if (row_ok && par + 2 < KT) lin_load_slab<BITS>(src + (int64_t)(par + 2) * (8 * BITS), wb);
-            for (int kt = par; kt < KT && ok; kt += 2) {
+            if (row_ok && par + LIN_GROUPS < KT)
+                lin_load_slab<BITS>(src + (int64_t)(par + LIN_GROUPS) * (8 * BITS), wb);
+            for (int kt = par; kt < KT && ok; kt += LIN_GROUPS) {
                 uint32_t wc[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) wc[i] = 0;
-                if (row_ok && kt + 4 < KT) lin_load_slab<BITS>(src + (int64_t)(kt + 4) * (8 * BITS), wc);
+                if (row_ok && kt + 2 * LIN_GROUPS < KT)
+                    lin_load_slab<BITS>(src + (int64_t)(kt + 2 * LIN_GROUPS) * (8 * BITS), wc);
                 ok = put(kt, wa);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) wa[i] = wb[i], wb[i] = wc[i];
             }
         }
         if (!ok) *(volatile int *)&s_abort = 1;
-        // ---- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31, the (w / 4)-th half of the columns ----
+        // ---- epilogue (warps 0-7): warp w reads TMEM lanes 32 (w % 4) .. +31, the (w / 4)-th half of
+        //      the columns ----
+        if (warp >= 8) ok = false;
         if (ok) ok = mbar_wait_bounded(done, 0, err);
         ok = __all_sync(FULL, ok);  // tcgen05.ld is warp-collective: the whole warp or none
         tc_fence_after();
@@ -506,7 +514,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                 }
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == LIN_TMA_WARP) {
         // ---- weight slabs: one 256 x 64 fp16 box per slab, 128-byte swizzle, through TMA ----
         if (lane == 0) {
             // code units (CTMA) go two units ahead of the weight slabs
@@ -569,7 +577,7 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == LIN_MMA_WARP) {
         tc_fence_after();
         tc_dealloc(tmem, LIN_TMEM_COLS);
     }
