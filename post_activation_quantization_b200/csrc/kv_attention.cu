@@ -23,12 +23,14 @@
 // the sum of the exponentials; pass 2 accumulates per lane over its share of the positions,
 // then across the row slots of a warp and the warps.  At entry one bulk L2 prefetch per cache
 // pulls the CTA's K and V rows (contiguous) towards the SM.
-// Measured at batch 8 x 96 heads x 2048 positions, D = 128, 3-bit (152 MB of codes): 0.151 ms.
-// ncu: about 6 instructions per code (unpacking a 3-bit field costs a shift and a mask-or, the
-// math two packed operations per pair), 42 % issue-active: the kernel is bound by instruction
-// issue, not by HBM (12 % of its bandwidth).  Splitting the positions of a (b, h) over a
-// thread-block cluster (combining max, sum and partial outputs through distributed shared
-// memory) measured slower: 2 CTAs 0.174 ms, 4 CTAs 0.244 ms.
+// Measured at batch 8 x 96 heads x 2048 positions, D = 128, 3-bit (152 MB of codes): 0.142 ms
+// with KVA_UNROLL = 8 rows in flight per warp (0.148 ms with 4; 16 needs 180 registers and runs
+// at 0.226 ms).  ncu: about 6 instructions per code, 42 % issue-active: neither issue nor HBM
+// (12 % of its bandwidth) is the bound; fewer instructions per code (codes masked in place at
+// their bit position) and four independent accumulators in pass 1 measured no faster, more
+// loads in flight did.  Splitting the positions of a (b, h) over a thread-block cluster
+// (combining max, sum and partial outputs through distributed shared memory) measured slower:
+// 2 CTAs 0.174 ms, 4 CTAs 0.244 ms.
 #include <algorithm>
 
 #include "common.cuh"
@@ -37,7 +39,7 @@
 namespace rptq {
 
 constexpr int KVA_THREADS = 256;
-constexpr int KVA_UNROLL = 4;
+constexpr int KVA_UNROLL = 8;  // row steps per warp iteration, their loads issued first
 constexpr uint32_t KVA_MAGIC = 0x4B000000u;  // the float 2^23
 
 // The codes of channels CPL*cc .. CPL*cc + CPL - 1 of a packed row, as the little-endian bit
