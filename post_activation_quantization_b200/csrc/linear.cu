@@ -460,9 +460,13 @@ __global__ void __launch_bounds__(LIN_THREADS, 1)
                     break;
                 uint32_t w[8];
                 lin_load_slab_smem<BITS>(sC + cu * LIN_C_BYTES + r * UB + (kt & 1) * (UB / 2), w);
-                __syncwarp();  // every lane has read the unit before it is released
-                if (lane == 0) lin_arrive(empty_c + 8 * cu);
                 ok = put(kt, w);
+                // the unit is released only after the decode in put() has consumed the loaded
+                // words: a shared-memory load still in flight at the release could read bytes
+                // of the next unit, which the TMA may already be writing (measured: an earlier
+                // release made the A4 results differ from run to run)
+                __syncwarp();
+                if (lane == 0) lin_arrive(empty_c + 8 * cu);
             }
         } else {
             uint32_t wa[8], wb[8];

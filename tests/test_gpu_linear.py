@@ -171,6 +171,26 @@ def test_bench_shape_sampled(C, g):
            f"linear bench shape C={C} A3 (sampled)", rows)
 
 
+@pytest.mark.parametrize("C,bits", [(4096, 4), (4096, 3), (768, 4), (1280, 3)])
+def test_repeated_launches_are_bit_identical(C, bits):
+    """The GEMM has a fixed accumulation order, so every launch on the same inputs must give the
+    same bits: a race between the rings (a slot refilled while it is still read) shows up here as
+    launches that differ, even where each result stays within the parity bounds.  2048 tokens into
+    3C outputs (the bench's layer shape at C = 4096), 40 launches against the first."""
+    T, N = 2048, 3 * C
+    g = torch.Generator().manual_seed(C + bits)
+    codes = torch.randint(0, 256, (T, C * bits // 8), dtype=torch.uint8, generator=g).to(DEV)
+    w_prep = (torch.randn(N, C, generator=g) * 1000).half().to(DEV)
+    bz, lam, sw = torch.randn(N, generator=g).to(DEV), torch.ones(N).to(DEV), torch.rand(N, generator=g).to(DEV)
+    ref = rptq.rptq_reordered_linear(codes, C, bits, w_prep, bz, lam, sw)
+    out = torch.empty_like(ref)
+    differing = 0
+    for _ in range(40):
+        rptq.rptq_reordered_linear(codes, C, bits, w_prep, bz, lam, sw, out=out)
+        differing += int(not torch.equal(out, ref))
+    assert differing == 0, f"{differing} of 40 launches differ from the first"
+
+
 def test_no_tokens_and_refused_shapes():
     C, N, g = 128, 64, 4
     cal, codes, qw, sw, zw = _case(4, C, N, g, 4, 5)
