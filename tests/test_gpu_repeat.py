@@ -1,0 +1,99 @@
+"""Repeated launches on the same inputs give the same bits.
+
+Every kernel of the path has a fixed order of operations, so a launch repeated on unchanged inputs
+must reproduce its outputs exactly.  A race between a shared-memory ring's refill and the reads of
+the slot it overwrites (or any other ordering bug) shows up here as launches that differ, even where
+each result on its own stays within the parity bounds.  Sizes are large enough for the streaming
+kernels to run their rings many times around: the OPT-175B width at 8192 tokens, a K/V cache of
+8 x 96 x 512 x 128, each entry point launched 30 times against its first result."""
+import pytest
+import torch
+
+from post_activation_quantization_b200 import rptq, synthetic
+from tests.gpu_common import DEV, dev_params, model_inputs, oracle_calibration
+
+pytestmark = pytest.mark.gpu
+REPEATS = 30
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from post_activation_quantization_b200 import build
+    build.build()
+    rptq.lib()
+    yield
+    assert rptq.rptq_device_error() == 0
+
+
+def _same_every_time(run):
+    """run() -> tuple of tensors; the number of launches whose outputs differ from the first."""
+    ref = [t.clone() for t in run()]
+    differing = 0
+    for _ in range(REPEATS):
+        got = run()
+        differing += int(any(not torch.equal(a, b) for a, b in zip(got, ref)))
+    torch.cuda.synchronize()
+    return differing
+
+
+@pytest.fixture(scope="module")
+def act():
+    """OPT-175B width, 8192 tokens, bf16, with the oracle's calibration of a 64-token batch."""
+    C, g, bits = 12288, 64, 3
+    m, gamma, beta = model_inputs(C, 41)
+    xc = synthetic.activations(64, m, 41, dtype="bf16", calibration=True)
+    cal = oracle_calibration(xc, gamma, beta, g, 10, bits)
+    x = synthetic.activations(8192, m, 41, dtype="bf16").to(DEV)
+    return dict(C=C, g=g, bits=bits, x=x, gamma=gamma.to(DEV), beta=beta.to(DEV), p=dev_params(cal), cal=cal)
+
+
+def test_fused_quantizer_repeats(act):
+    a, p = act, act["p"]
+    codes = torch.empty((a["x"].shape[0], a["C"] * a["bits"] // 8), dtype=torch.uint8, device=DEV)
+    plan = rptq.rptq_ln_quant_plan(a["gamma"], a["beta"], p["R"], p["col_cluster"], p["scale"], p["zero"], a["bits"])
+    assert _same_every_time(lambda: (rptq.rptq_ln_reorder_quant_planned(a["x"], plan, a["bits"], codes=codes),)) == 0
+    assert _same_every_time(lambda: rptq.rptq_ln_reorder_quant(
+        a["x"], a["gamma"], a["beta"], p["R"], p["col_cluster"], p["scale"], p["zero"], a["bits"], codes=codes)[:1]) == 0
+
+
+def test_calibration_and_dequant_repeats(act):
+    a, p = act, act["p"]
+    assert _same_every_time(lambda: rptq.rptq_calib_minmax(a["x"], a["gamma"], a["beta"], 1e-5)) == 0
+    assert _same_every_time(lambda: rptq.rptq_calib_minmax(a["x"])) == 0
+    codes, _ = rptq.rptq_ln_reorder_quant(a["x"], a["gamma"], a["beta"], p["R"], p["col_cluster"], p["scale"],
+                                          p["zero"], a["bits"])
+    out = torch.empty((a["x"].shape[0], a["C"]), dtype=torch.bfloat16, device=DEV)
+    assert _same_every_time(lambda: (rptq.rptq_dequant(codes, p["col_cluster"], p["scale"], p["zero"], a["bits"],
+                                                       C=a["C"], out=out),)) == 0
+
+
+def test_kmeans_repeats(act):
+    a = act
+    mx = torch.from_numpy(a["cal"]["ch_max"]).to(DEV)
+    mn = torch.from_numpy(a["cal"]["ch_min"]).to(DEV)
+    assert _same_every_time(lambda: tuple(rptq.rptq_kmeans(mx, mn, a["g"], 50, a["bits"]).values())) == 0
+
+
+def test_kv_repeats():
+    B, H, S, D, g, bits = 8, 96, 512, 128, 64, 3
+    mk = synthetic.channel_model(H * D, 43, tag=1)
+    mv = synthetic.channel_model(H * D, 43, tag=2)
+    k = synthetic.kv_cache(B, H, S, D, mk, 43, "k", "bf16").to(DEV)
+    v = synthetic.kv_cache(B, H, S, D, mv, 43, "v", "bf16").to(DEV)
+    assert _same_every_time(lambda: rptq.rptq_kv_calib_minmax(k)) == 0
+    kmx, kmn = rptq.rptq_kv_calib_minmax(k)
+    vmx, vmn = rptq.rptq_kv_calib_minmax(v)
+    ck = rptq.rptq_kmeans(kmx, kmn, g, 10, bits)
+    cv = rptq.rptq_kmeans(vmx, vmn, g, 10, bits)
+    kq = torch.empty((B, H, S, D * bits // 8), dtype=torch.uint8, device=DEV)
+    vq = torch.empty_like(kq)
+    args = (ck["labels"], ck["scale"], ck["zero"], cv["labels"], cv["scale"], cv["zero"], bits)
+    assert _same_every_time(lambda: rptq.rptq_kv_quant(k, v, *args, k_codes=kq, v_codes=vq)) == 0
+    out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=DEV)
+    assert _same_every_time(lambda: (rptq.rptq_dequant(kq, ck["labels"], ck["scale"], ck["zero"], bits,
+                                                       layout=rptq.RPTQ_LAYOUT_BHSD, out=out),)) == 0
+    q = torch.randn(B, H, D, generator=torch.Generator().manual_seed(43)).to(DEV)
+    att = torch.empty((B, H, D), dtype=torch.float32, device=DEV)
+    assert _same_every_time(lambda: (rptq.rptq_kv_decode_attention(q, kq, vq, S, *args, out=att),)) == 0
