@@ -711,10 +711,13 @@ __global__ void __launch_bounds__(KM_THREADS, 1)
 
 // ------------------------------------------------------------------------------------------
 // Per-cluster (s, z) for fixed clusters from per-channel statistics: the parameter step of the
-// calibration on its own, for dynamic (per-batch) ranges.  One CTA: the members' max / min are
-// folded per cluster with order-independent shared-memory atomics (exact), then s and z follow
-// with the same fp32 IEEE operations as in the calibration above.
-__global__ void __launch_bounds__(512)
+// calibration on its own, for dynamic (per-batch) ranges.  One CTA of CP_THREADS: the members'
+// max / min are folded per cluster with order-independent shared-memory atomics (exact), then s
+// and z follow with the same fp32 IEEE operations as in the calibration above.  A thread loads
+// the (label, max, min) of CP_UNROLL channels before folding any, so the loads of a whole pass
+// over the channels are in flight together instead of one round trip per CP_THREADS channels.
+constexpr int CP_THREADS = 1024, CP_UNROLL = 4;
+__global__ void __launch_bounds__(CP_THREADS)
     cluster_params_kernel(const float *__restrict__ mx, const float *__restrict__ mn, int C,
                           const int32_t *__restrict__ labels, int g, int bits, float *__restrict__ scale,
                           int32_t *__restrict__ zero, int *err)
@@ -727,15 +730,28 @@ __global__ void __launch_bounds__(512)
         cnt[k] = 0;
     }
     __syncthreads();
-    for (int c = threadIdx.x; c < C; c += blockDim.x) {
-        const int k = labels[c];
-        if (k < 0 || k >= g) {
-            raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
-            continue;
+    for (int c0 = threadIdx.x; c0 < C; c0 += CP_THREADS * CP_UNROLL) {
+        int kk[CP_UNROLL];
+        float vx[CP_UNROLL], vn[CP_UNROLL];
+#pragma unroll
+        for (int u = 0; u < CP_UNROLL; ++u) {
+            const int c = c0 + u * CP_THREADS;
+            kk[u] = c < C ? __ldg(labels + c) : -1;
+            vx[u] = c < C ? __ldg(mx + c) : 0.f;
+            vn[u] = c < C ? __ldg(mn + c) : 0.f;
         }
-        atomic_max_f32(cmx + k, mx[c]);
-        atomic_min_f32(cmn + k, mn[c]);
-        atomicAdd(cnt + k, 1);
+#pragma unroll
+        for (int u = 0; u < CP_UNROLL; ++u) {
+            if (c0 + u * CP_THREADS >= C) continue;
+            const int k = kk[u];
+            if (k < 0 || k >= g) {
+                raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+                continue;
+            }
+            atomic_max_f32(cmx + k, vx[u]);
+            atomic_min_f32(cmn + k, vn[u]);
+            atomicAdd(cnt + k, 1);
+        }
     }
     __syncthreads();
     const float qmax = (float)((1 << bits) - 1);
@@ -762,7 +778,7 @@ __global__ void __launch_bounds__(512)
 cudaError_t launch_cluster_params(const float *mx, const float *mn, int C, const int32_t *labels, int g, int bits,
                                   float *scale, int32_t *zero, int *err, cudaStream_t stream)
 {
-    cluster_params_kernel<<<1, 512, 0, stream>>>(mx, mn, C, labels, g, bits, scale, zero, err);
+    cluster_params_kernel<<<1, CP_THREADS, 0, stream>>>(mx, mn, C, labels, g, bits, scale, zero, err);
     return cudaGetLastError();
 }
 
