@@ -231,6 +231,22 @@ def kv_quant(kv, col_cluster, s, z, bits):
     return out
 
 
+def kv_quant_cluster_ordered(kv, R, col_cluster, s, z, bits):
+    """The K/V cache stored in cluster order ([RPTQ-art] text after Fig. 2: the channels of one
+    cluster placed side by side, each cluster with its own s and z; results paragraph: the K/V
+    cache quantized per cluster) -- the layout variant of the cache, beside kv_quant's kept
+    [B, H, S, D] layout.  For every token (b, s) the C = H*D channels (channel c = h*D + d) are
+    gathered through the reorder index (stored column j holds channel R[j]), quantized with the
+    cluster of the stored column (col_cluster[j]) and packed as one row: codes [B, S, C*bits/8],
+    the layout of the activation codes.  Definition written out: transpose to token rows, gather,
+    then the oracle's quantize and pack."""
+    kv = _f32(kv)
+    B, H, S, D = kv.shape
+    rows = np.ascontiguousarray(kv.transpose(0, 2, 1, 3).reshape(B * S, H * D))
+    q = quantize(rows[:, np.asarray(R, dtype=np.int64)], col_cluster, s, z, bits)
+    return pack(q, bits).reshape(B, S, H * D * bits // 8)
+
+
 def kv_dequant(packed, D, col_cluster, s, z, bits):
     packed = np.ascontiguousarray(packed, dtype=np.uint8)
     B, H, S, _ = packed.shape
