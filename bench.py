@@ -108,6 +108,9 @@ def stage_list(w: W.Workload):
         st += [("linear_prepare", W.bytes_linear_prepare(N, C), 1), ("reordered_linear", 0, 1)]
     if k:
         st += [("kv_quant", W.bytes_kv_quant(k.elems, k.dtype, k.bits), 1)]
+        # the layout variant: the K cache quantized into token rows in cluster order (a comparison
+        # beside the kept layout's K/V quantizer: one tensor, the same codes)
+        st += [("kv_quant_cluster_ordered", W.bytes_kv_quant(k.elems, k.dtype, k.bits, tensors=1), 1)]
     if a:
         st += [("dequant_act", W.bytes_dequant(n, w.dtype, w.bits), 1)]
     if k:
@@ -172,6 +175,7 @@ class Step:
             shape = (k.B, k.H, k.S, k.D * k.bits // 8)
             self.kq = torch.empty(shape, dtype=torch.uint8, device=device)
             self.vq = torch.empty(shape, dtype=torch.uint8, device=device)
+            self.kq_co = torch.empty((k.B, k.S, k.H * k.D * k.bits // 8), dtype=torch.uint8, device=device)
             kvdt = synthetic.torch_dtype(k.dtype)
             self.khat = torch.empty((k.B, k.H, k.S, k.D), dtype=kvdt, device=device)
             self.vhat = torch.empty_like(self.khat)
@@ -287,6 +291,10 @@ class Step:
                             self.kmv["labels"], self.kmv["scale"], self.kmv["zero"], k.bits,
                             k_codes=self.kq, v_codes=self.vq)
             mark("kv_quant", 1)
+            mark("kv_quant_cluster_ordered", 0)
+            r.rptq_kv_quant_cluster_ordered(self.k, self.kmk["R"], self.kmk["col_cluster"], self.kmk["scale"],
+                                            self.kmk["zero"], k.bits, codes=self.kq_co)
+            mark("kv_quant_cluster_ordered", 1)
         if self.act:
             mark("dequant_act", 0)
             r.rptq_dequant(self.codes, self.km["col_cluster"], self.km["scale"], self.km["zero"], w.bits,
@@ -397,7 +405,7 @@ def _traffic(kernel: str):
 
 
 # ------------------------------------------------------------------------------------------
-COMPARISON_STAGES = ("explicit_reorder_baseline", "ln_reorder_quant_unplanned")
+COMPARISON_STAGES = ("explicit_reorder_baseline", "ln_reorder_quant_unplanned", "kv_quant_cluster_ordered")
 GRAPH_SLOTS = 8
 B2B_LAUNCHES = 20
 

@@ -291,6 +291,30 @@ int rptq_kv_append(const void *k_new, const void *v_new, int dtype, int B, int H
                    uint8_t *k_cache, uint8_t *v_cache, rptq_stream_t stream);
 
 /*
+ * The K or V cache stored in cluster order: the layout variant of the cache beside
+ * rptq_kv_quant's kept [B, H, S, D] layout ([RPTQ-art] text after Fig. 2: the channels of one
+ * cluster placed side by side, one s and z per cluster; results paragraph: the K/V cache
+ * quantized per cluster).  For every token (b, s) the C = H*D channels (c = h*D + d) are
+ * gathered through the reorder index and quantized per cluster:
+ *   codes[b][s] = pack over j of clamp(rint(kv[b, h, s, d] / s_k) + z_k, 0, qmax),
+ *                 c = R[j] = h*D + d, k = col_cluster[j],
+ * the same codes as rptq_kv_quant channel for channel (the same quotient, rounding and clamp),
+ * in the row layout of the activation codes, so rptq_dequant's rows layout reads them back with
+ * col_cluster.
+ *   kv     [B, H, S, D] of `dtype` (RPTQ_F32 / RPTQ_F16 / RPTQ_BF16), 16-byte aligned.
+ *   R, col_cluster  int32 [C] (rptq_kmeans's outputs for this cache); scale fp32 [g], zero int32 [g].
+ *   codes  uint8 [B, S, C*bits/8] output, 16-byte aligned.
+ * D a multiple of 8, C a multiple of 32 and at most RPTQ_MAX_CHANNELS (RPTQ_ERR_UNSUPPORTED
+ * otherwise); B == 0 or S == 0 is valid: nothing is launched.  An R entry outside [0, C) or a
+ * cluster id outside [0, g) is reported in the device error word (the codes are then undefined,
+ * every store stays inside `codes`).
+ */
+int rptq_kv_quant_cluster_ordered(const void *kv, int dtype, int B, int H, int64_t S, int D,
+                                  const int32_t *R, const int32_t *col_cluster, const float *scale,
+                                  const int32_t *zero, int g, int bits, uint8_t *codes,
+                                  rptq_stream_t stream);
+
+/*
  * One decode step of attention over the packed caches, dequantizing every code in registers
  * as it is read (value = s_k * (q - z_k) in fp32, the value rptq_dequant writes): the consumer
  * of the quantized K/V cache ([RPTQ-art] results and closing memory paragraphs).  For every

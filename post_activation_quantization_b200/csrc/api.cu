@@ -367,6 +367,28 @@ int rptq_kv_append(const void *k_new, const void *v_new, int dtype, int B, int H
     return cuda_status(launch_kv_append(a));
 }
 
+int rptq_kv_quant_cluster_ordered(const void *kv, int dtype, int B, int H, int64_t S, int D, const int32_t *R,
+                                  const int32_t *col_cluster, const float *scale, const int32_t *zero, int g,
+                                  int bits, uint8_t *codes, rptq_stream_t stream)
+{
+    if (bits != 3 && bits != 4) return RPTQ_ERR_UNSUPPORTED;
+    if (dtype != RPTQ_F32 && dtype != RPTQ_F16 && dtype != RPTQ_BF16) return RPTQ_ERR_UNSUPPORTED;
+    if (B < 0 || H <= 0 || S < 0 || D <= 0 || g <= 0 || g > RPTQ_MAX_CLUSTERS) return RPTQ_ERR_INVALID_ARG;
+    const int64_t C = (int64_t)H * D;
+    if (D % 8 != 0 || C % 32 != 0 || C > RPTQ_MAX_CHANNELS) return RPTQ_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return RPTQ_OK;
+    if (!kv || !R || !col_cluster || !scale || !zero || !codes) return RPTQ_ERR_INVALID_ARG;
+    if (!aligned16(kv) || !aligned16(codes)) return RPTQ_ERR_INVALID_ARG;
+    if ((int64_t)B * ((S + 3) / 4) > ((int64_t)1 << 40)) return RPTQ_ERR_UNSUPPORTED;
+    DevInfo d;
+    int st = dev_info(&d);
+    if (st) return st;
+    if (!kv_quant_reordered_supported(H, D, g, d.max_smem)) return RPTQ_ERR_UNSUPPORTED;
+    KvReorderedArgs a{kv, dtype, B, H, S, D, R, col_cluster, scale, zero, g, bits, codes, d.err,
+                      (cudaStream_t)stream, d.num_sms};
+    return cuda_status(launch_kv_quant_reordered(a));
+}
+
 int rptq_kv_decode_attention(const float *q, int B, int H, int D, const uint8_t *k_cache,
                              const uint8_t *v_cache, int64_t S_max, int64_t L,
                              const int32_t *cluster_k, const float *scale_k, const int32_t *zero_k,

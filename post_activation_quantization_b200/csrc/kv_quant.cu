@@ -532,3 +532,196 @@ extern "C" int rptq_testing_kv_quotient(const float *x, int64_t n, float s, floa
     if (cudaGetLastError() != cudaSuccess) return RPTQ_ERR_CUDA;
     return RPTQ_OK;
 }
+
+// ==========================================================================================
+// The K/V cache in cluster order (rptq_kv_quant_cluster_ordered): the layout variant of the cache
+// that stores every token's C = H*D channels (c = h*D + d) in cluster order, as the activation
+// codes are stored -- RPTQ article, text after Fig. 2 (the channels of one cluster placed side
+// by side, one (s, z) per cluster) and results paragraph (the K/V cache quantized per cluster).
+// Output rows [B, S, C*bits/8]; stored column j holds channel R[j] with cluster col_cluster[j].
+// The codes are those of the kept layout (the same quotient, rounding and clamp as kv_quant_row
+// above), channel for channel.
+//
+// Persistent CTAs.  Each CTA first builds, in shared memory, the word offset of every channel's
+// stored column and the channel's cluster (entries of R outside [0, C) are reported and leave
+// the offset at 0, so every store stays inside the code buffer), and the per-cluster quotient
+// coefficients.  Per quad of 4 tokens of one b: a thread takes groups of 8 channels of one head
+// (16-byte loads, 4 rows apart by D), forms the 4 tokens' codes of each channel into one word and
+// stores it at the channel's stored column; after a barrier, threads pack 32 stored columns x 4
+// tokens each (the same 8 x 4 packers as the fused activation kernel) and write whole words.
+namespace rptq {
+namespace {
+constexpr int KVO_THREADS = 256;
+struct KvoCluster {
+    float ns, r, s;    // -s 2^24, RN(1/s) 2^-24, s
+    int32_t lo, hi, z;  // clamp of the rounded bit pattern: MAGIC_BITS - z .. + qmax
+    int32_t fast, pad;
+};
+__host__ __device__ inline size_t kvo_smem_bytes(int C, int g)
+{
+    return ((size_t)C * 6 + 15) / 16 * 16 + (size_t)g * sizeof(KvoCluster) + (size_t)C * 4;
+}
+}  // namespace
+
+template <int BITS>
+__device__ __forceinline__ uint32_t kvo_code(float x, const KvoCluster &k)
+{
+    constexpr int QMAX = (1 << BITS) - 1;
+    if (k.fast) {
+        const float q0 = x * k.r;
+        const float qq = __fmaf_rn(__fmaf_rn(q0, k.ns, x), k.r, q0);  // RN(x / (s 2^24))
+        const float b = __fmaf_rn(qq, KV_QSCALE, MAGIC_RINT);           // 1.5*2^23 + rint(x / s)
+        const int32_t l = min(max((int32_t)__float_as_uint(b), k.lo), k.hi);
+        return (uint32_t)(l - k.lo);
+    }
+    return kv_code_ieee<QMAX>(x, k.s, k.z);
+}
+
+template <typename T, int BITS>
+__global__ void __launch_bounds__(KVO_THREADS)
+    kv_quant_reordered_kernel(const T *__restrict__ kv, int H, int64_t S, int D, int64_t units,
+                              const int32_t *__restrict__ R, const int32_t *__restrict__ col_cluster,
+                              const float *__restrict__ scale, const int32_t *__restrict__ zero, int g,
+                              uint8_t *__restrict__ codes, int *err)
+{
+    constexpr int VEC = Elem<T>::VEC;  // elements per 16 bytes
+    constexpr uint32_t MAGIC_BITS = 0x4B400000u;
+    constexpr int QMAX = (1 << BITS) - 1;
+    extern __shared__ __align__(16) uint8_t kvo_smem[];
+    const int C = H * D, tid = threadIdx.x;
+    uint32_t *posw = reinterpret_cast<uint32_t *>(kvo_smem);  // [C] word index of channel c's stored column
+    uint16_t *kcl = reinterpret_cast<uint16_t *>(posw + C);    // [C] cluster of channel c
+    KvoCluster *cl = reinterpret_cast<KvoCluster *>(kvo_smem + ((size_t)C * 6 + 15) / 16 * 16);  // [g]
+    uint32_t *cbuf = reinterpret_cast<uint32_t *>(cl + g);     // [C] 4 tokens' codes per stored column
+
+    for (int c = tid; c < C; c += KVO_THREADS) {
+        posw[c] = 0;
+        kcl[c] = 0;
+    }
+    for (int k = tid; k < g; k += KVO_THREADS) {
+        const float sv = scale[k];
+        const int z = zero[k];
+        KvoCluster e;
+        e.ns = -(sv * KV_QSCALE);
+        e.r = __frcp_rn(sv) * KV_QSCALE_INV;
+        e.s = sv;
+        e.z = z;
+        e.lo = (int32_t)(MAGIC_BITS - (uint32_t)z);
+        e.hi = (int32_t)(MAGIC_BITS + (uint32_t)QMAX - (uint32_t)z);
+        e.fast = (z > -(1 << 21)) && (z < (1 << 21)) && kv_fast_scale(sv);
+        e.pad = 0;
+        cl[k] = e;
+    }
+    __syncthreads();
+    for (int j = tid; j < C; j += KVO_THREADS) {
+        const int c = R[j];
+        int k = col_cluster[j];
+        if (k < 0 || k >= g) {
+            raise_error(err, RPTQ_DEVERR_CLUSTER_ID);
+            k = 0;
+        }
+        if (c < 0 || c >= C) {
+            raise_error(err, RPTQ_DEVERR_REORDER);
+            continue;
+        }
+        posw[c] = (uint32_t)j;
+        kcl[c] = (uint16_t)k;
+    }
+    __syncthreads();
+
+    const int64_t NQ = (S + 3) / 4, pitch = (int64_t)C * BITS / 8;
+    const int NG8 = C / 8, NU = C / 32;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int64_t b = u / NQ, s0 = (u - b * NQ) * 4;
+        const int nt = (int)min((int64_t)4, S - s0);
+        for (int i = tid; i < NG8; i += KVO_THREADS) {
+            const int c0 = 8 * i, h = c0 / D, d0 = c0 - h * D;
+            const T *row = kv + ((b * H + h) * S + s0) * D + d0;
+            uint4 xv[4][8 / VEC];
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int v = 0; v < 8 / VEC; ++v)
+                    xv[t][v] = t < nt ? __ldg(reinterpret_cast<const uint4 *>(row + (int64_t)t * D) + v)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const KvoCluster k0 = cl[kcl[c0 + e]], k1 = cl[kcl[c0 + e + 1]];
+                uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    const f32x2 x2 = pair_of<T>(xv[t][e / VEC], (e % VEC) / 2);
+                    w0 |= kvo_code<BITS>(lo2(x2), k0) << (8 * t);
+                    w1 |= kvo_code<BITS>(hi2(x2), k1) << (8 * t);
+                }
+                cbuf[posw[c0 + e]] = w0;
+                cbuf[posw[c0 + e + 1]] = w1;
+            }
+        }
+        __syncthreads();
+        for (int pu = tid; pu < NU; pu += KVO_THREADS) {
+            uint32_t o[4][4];  // [group m of 8 stored columns][token]
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                uint32_t w[8];
+                const uint4 a = *reinterpret_cast<const uint4 *>(cbuf + 32 * pu + 8 * m);
+                const uint4 c4 = *reinterpret_cast<const uint4 *>(cbuf + 32 * pu + 8 * m + 4);
+                w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = c4.x, w[5] = c4.y, w[6] = c4.z, w[7] = c4.w;
+                if constexpr (BITS == 4)
+                    pack8x4_a4(w, o[m]);
+                else
+                    pack8x4_a3(w, o[m]);
+            }
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                if (t >= nt) continue;
+                uint8_t *dst = codes + (b * S + s0 + t) * pitch + (int64_t)pu * (4 * BITS);
+                if constexpr (BITS == 4) {
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(o[0][t], o[1][t], o[2][t], o[3][t]);
+                } else {  // four 24-bit groups -> three words
+                    uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
+                    d32[0] = o[0][t] | (o[1][t] << 24);
+                    d32[1] = (o[1][t] >> 8) | (o[2][t] << 16);
+                    d32[2] = (o[2][t] >> 16) | (o[3][t] << 8);
+                }
+            }
+        }
+        __syncthreads();  // the code buffer is refilled by the next quad
+    }
+}
+
+bool kv_quant_reordered_supported(int H, int D, int g, int max_smem)
+{
+    const int64_t C = (int64_t)H * D;
+    return D >= 8 && D % 8 == 0 && C % 32 == 0 && C <= RPTQ_MAX_CHANNELS && g >= 1 &&
+           g <= RPTQ_MAX_CLUSTERS && kvo_smem_bytes((int)C, g) <= (size_t)max_smem;
+}
+
+cudaError_t launch_kv_quant_reordered(const KvReorderedArgs &a)
+{
+    const int64_t units = (int64_t)a.B * ((a.S + 3) / 4);
+    if (units == 0) return cudaSuccess;
+    const int C = a.H * a.D;
+    const size_t smem = kvo_smem_bytes(C, a.g);
+    const void *kern = nullptr;
+    if (a.dtype == 0)
+        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<float, 4> : (const void *)kv_quant_reordered_kernel<float, 3>;
+    else if (a.dtype == 1)
+        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<__half, 4> : (const void *)kv_quant_reordered_kernel<__half, 3>;
+    else
+        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<__nv_bfloat16, 4>
+                           : (const void *)kv_quant_reordered_kernel<__nv_bfloat16, 3>;
+    cudaError_t e = kernel_smem(kern, smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 1;
+    e = kernel_occupancy(&per_sm, kern, KVO_THREADS, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(units, (int64_t)a.num_sms * std::max(1, per_sm));
+    int H = a.H, D = a.D, g = a.g;
+    int64_t S = a.S, U = units;
+    void *args[] = {(void *)&a.kv, (void *)&H, (void *)&S, (void *)&D, (void *)&U, (void *)&a.R,
+                    (void *)&a.col_cluster, (void *)&a.scale, (void *)&a.zero, (void *)&g, (void *)&a.codes, (void *)&a.err};
+    return cudaLaunchKernel(kern, dim3((unsigned)grid), dim3(KVO_THREADS), args, smem, a.stream);
+}
+
+}  // namespace rptq

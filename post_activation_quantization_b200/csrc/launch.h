@@ -98,6 +98,22 @@ struct KvAppendArgs {
     int num_sms;
 };
 
+// rptq_kv_quant_cluster_ordered: K or V [B, H, S, D] -> codes [B, S, C*bits/8] in cluster order
+struct KvReorderedArgs {
+    const void *kv;
+    int dtype, B, H;
+    int64_t S;
+    int D;
+    const int32_t *R, *col_cluster;
+    const float *scale;
+    const int32_t *zero;
+    int g, bits;
+    uint8_t *codes;
+    int *err;
+    cudaStream_t stream;
+    int num_sms;
+};
+
 struct KvAttnArgs {
     const float *q;
     int B, H, D;
@@ -210,6 +226,9 @@ cudaError_t launch_cluster_params(const float *mx, const float *mn, int C, const
                                   float *scale, int32_t *zero, int *err, cudaStream_t stream);
 cudaError_t launch_explicit_reorder(const XrArgs &a);
 cudaError_t launch_kv_attention(const KvAttnArgs &a);
+cudaError_t launch_kv_quant_reordered(const KvReorderedArgs &a);
+// (H, D, g) that the cluster-ordered K/V kernel takes, with its tables within max_smem
+bool kv_quant_reordered_supported(int H, int D, int g, int max_smem);
 cudaError_t launch_linear_prepare(const LinPrepArgs &a);
 cudaError_t launch_reordered_linear(const LinArgs &a);
 // largest number of cache positions one decode-attention call reads (its scores stay in shared

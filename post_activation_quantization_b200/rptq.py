@@ -48,6 +48,7 @@ SIGNATURES = {
     "rptq_kmeans_noalloc": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P]),
     "rptq_ln_reorder_quant": (_I, [_P, _I, _I64, _I, _P, _P, _F, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_quant": (_I, [_P, _P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
+    "rptq_kv_quant_cluster_ordered": (_I, [_P, _I, _I, _I, _I64, _I, _P, _P, _P, _P, _I, _I, _P, _P]),
     "rptq_dequant": (_I, [_P, _I, _I64, _I, _I64, _I, _P, _P, _P, _I, _I, _P, _I, _P]),
     "rptq_cluster_params": (_I, [_P, _P, _I, _P, _I, _I, _P, _P, _P]),
     "rptq_kv_append": (_I, [_P, _P, _I, _I, _I, _I64, _I, _I64, _I64, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P]),
@@ -230,6 +231,19 @@ def rptq_kv_quant(k, v, cluster_k, scale_k, zero_k, cluster_v, scale_v, zero_v, 
                              _ptr(zero_v), g, bits, _ptr(k_codes), _ptr(v_codes), _stream(stream))
     _check(st, "rptq_kv_quant")
     return k_codes, v_codes
+
+
+def rptq_kv_quant_cluster_ordered(kv, R, col_cluster, scale, zero, bits: int, codes=None, stream=None):
+    """K or V [B, H, S, D] quantized per cluster and stored in cluster order: codes [B, S, C*bits/8]
+    (C = H*D; stored column j holds channel R[j])."""
+    B, H, S, D = kv.shape
+    if codes is None:
+        codes = torch.empty((B, S, H * D * bits // 8), dtype=torch.uint8, device=kv.device)
+    st = lib().rptq_kv_quant_cluster_ordered(_ptr(kv), _DT[kv.dtype], B, H, S, D, _ptr(R), _ptr(col_cluster),
+                                             _ptr(scale), _ptr(zero), scale.numel(), bits, _ptr(codes),
+                                             _stream(stream))
+    _check(st, "rptq_kv_quant_cluster_ordered")
+    return codes
 
 
 def rptq_dequant(codes: torch.Tensor, cluster, scale, zero, bits: int, out_dtype=torch.float32,

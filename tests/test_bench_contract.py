@@ -50,8 +50,8 @@ def test_stage_accounting_per_workload():
     st = bench.stage_list(W.WORKLOADS["opt175b-12288"])
     assert [s[0] for s in st] == ["calib_ln", "kv_calib", "kmeans", "ln_quant_plan", "ln_reorder_quant",
                                   "ln_reorder_quant_unplanned", "explicit_reorder_baseline", "dynamic_ranges",
-                                  "linear_prepare", "reordered_linear", "kv_quant", "dequant_act", "dequant_kv",
-                                  "kv_append", "kv_decode_attention"]
+                                  "linear_prepare", "reordered_linear", "kv_quant", "kv_quant_cluster_ordered",
+                                  "dequant_act", "dequant_kv", "kv_append", "kv_decode_attention"]
     b = dict((n, v) for n, v, _ in st)
     T, C, Tc, kv = 32768, 12288, 262144, 8 * 96 * 2048 * 128
     assert b["calib_ln"] == Tc * C * 2
@@ -59,6 +59,7 @@ def test_stage_accounting_per_workload():
     assert b["ln_reorder_quant"] == b["ln_reorder_quant_unplanned"] == T * C * 2 + T * C * 3 // 8
     assert b["ln_quant_plan"] == 28 * C
     assert b["kv_quant"] == 2 * (kv * 2 + kv * 3 // 8)
+    assert b["kv_quant_cluster_ordered"] == kv * 2 + kv * 3 // 8
     assert b["dequant_act"] == T * C * 3 // 8 + T * C * 2
     assert b["dequant_kv"] == 2 * (kv * 3 // 8 + kv * 2)
     assert b["kv_append"] == 2 * (8 * 96 * 128 * 2 + 8 * 96 * 128 * 3 // 8)
@@ -70,10 +71,11 @@ def test_stage_accounting_per_workload():
     N = 3 * C
     assert b["linear_prepare"] == N * C // 2 + N * C * 2 + 8 * N and b["reordered_linear"] == 0
     assert bench.stage_flops(W.WORKLOADS["opt175b-12288"]) == {"reordered_linear": 2 * 2048 * C * N}
-    assert sum(l for _, _, l in st) == 29  # 2 + 4 + 6 + 1 + 1 + 1 + 3 + 3 + 1 + 1 + 1 + 1 + 2 + 1 + 1
+    assert sum(l for _, _, l in st) == 30  # 2 + 4 + 6 + 1 + 1 + 1 + 3 + 3 + 1 + 1 + 1 + 1 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["kv-4096"])
-    assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "dequant_kv", "kv_append", "kv_decode_attention"]
-    assert sum(l for _, _, l in st) == 4 + 4 + 1 + 2 + 1 + 1
+    assert [s[0] for s in st] == ["kv_calib", "kmeans", "kv_quant", "kv_quant_cluster_ordered", "dequant_kv", "kv_append",
+                                  "kv_decode_attention"]
+    assert sum(l for _, _, l in st) == 4 + 4 + 1 + 1 + 2 + 1 + 1
     st = bench.stage_list(W.WORKLOADS["tiny-768"])
     assert [s[0] for s in st] == ["calib_ln", "kmeans", "ln_quant_plan", "ln_reorder_quant", "ln_reorder_quant_unplanned",
                                   "explicit_reorder_baseline", "dynamic_ranges", "linear_prepare", "reordered_linear",

@@ -91,6 +91,9 @@ def test_kv_repeats():
     vq = torch.empty_like(kq)
     args = (ck["labels"], ck["scale"], ck["zero"], cv["labels"], cv["scale"], cv["zero"], bits)
     assert _same_every_time(lambda: rptq.rptq_kv_quant(k, v, *args, k_codes=kq, v_codes=vq)) == 0
+    kco = torch.empty((B, S, H * D * bits // 8), dtype=torch.uint8, device=DEV)
+    assert _same_every_time(lambda: (rptq.rptq_kv_quant_cluster_ordered(k, ck["R"], ck["col_cluster"], ck["scale"],
+                                                                        ck["zero"], bits, codes=kco),)) == 0
     out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=DEV)
     assert _same_every_time(lambda: (rptq.rptq_dequant(kq, ck["labels"], ck["scale"], ck["zero"], bits,
                                                        layout=rptq.RPTQ_LAYOUT_BHSD, out=out),)) == 0
