@@ -577,8 +577,8 @@ __device__ __forceinline__ uint32_t kvo_code(float x, const KvoCluster &k)
     return kv_code_ieee<QMAX>(x, k.s, k.z);
 }
 
-template <typename T, int BITS>
-__global__ void __launch_bounds__(KVO_THREADS)
+template <typename T, int BITS, int GPT, int NT>
+__global__ void __launch_bounds__(NT)
     kv_quant_reordered_kernel(const T *__restrict__ kv, int H, int64_t S, int D, int64_t units,
                               const int32_t *__restrict__ R, const int32_t *__restrict__ col_cluster,
                               const float *__restrict__ scale, const int32_t *__restrict__ zero, int g,
@@ -594,11 +594,11 @@ __global__ void __launch_bounds__(KVO_THREADS)
     KvoCluster *cl = reinterpret_cast<KvoCluster *>(kvo_smem + ((size_t)C * 6 + 15) / 16 * 16);  // [g]
     uint32_t *cbuf = reinterpret_cast<uint32_t *>(cl + g);     // [C] 4 tokens' codes per stored column
 
-    for (int c = tid; c < C; c += KVO_THREADS) {
+    for (int c = tid; c < C; c += NT) {
         posw[c] = 0;
         kcl[c] = 0;
     }
-    for (int k = tid; k < g; k += KVO_THREADS) {
+    for (int k = tid; k < g; k += NT) {
         const float sv = scale[k];
         const int z = zero[k];
         KvoCluster e;
@@ -613,7 +613,7 @@ __global__ void __launch_bounds__(KVO_THREADS)
         cl[k] = e;
     }
     __syncthreads();
-    for (int j = tid; j < C; j += KVO_THREADS) {
+    for (int j = tid; j < C; j += NT) {
         const int c = R[j];
         int k = col_cluster[j];
         if (k < 0 || k >= g) {
@@ -631,26 +631,46 @@ __global__ void __launch_bounds__(KVO_THREADS)
 
     const int64_t NQ = (S + 3) / 4, pitch = (int64_t)C * BITS / 8;
     const int NG8 = C / 8, NU = C / 32;
+    // the rows of unit u: one bulk L2 prefetch per head (4 consecutive rows of a (b, h) block)
+    auto prefetch_unit = [&](int64_t u) {
+        if (u >= units) return;
+        const int64_t b = u / NQ, s0 = (u - b * NQ) * 4;
+        const int nt = (int)min((int64_t)4, S - s0);
+        for (int h = tid; h < H; h += NT)
+            prefetch_l2(kv + ((b * H + h) * S + s0) * D, (uint32_t)(nt * D * (int)sizeof(T)));
+    };
+    prefetch_unit(blockIdx.x);
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t b = u / NQ, s0 = (u - b * NQ) * 4;
         const int nt = (int)min((int64_t)4, S - s0);
-        for (int i = tid; i < NG8; i += KVO_THREADS) {
+        prefetch_unit(u + gridDim.x);
+        // every row load of the thread's groups first (GPT groups of 8 channels, 4 tokens each)
+        uint4 xv[GPT][4][8 / VEC];
+#pragma unroll
+        for (int gi = 0; gi < GPT; ++gi) {
+            const int i = tid + gi * NT;
             const int c0 = 8 * i, h = c0 / D, d0 = c0 - h * D;
             const T *row = kv + ((b * H + h) * S + s0) * D + d0;
-            uint4 xv[4][8 / VEC];
 #pragma unroll
             for (int t = 0; t < 4; ++t)
 #pragma unroll
                 for (int v = 0; v < 8 / VEC; ++v)
-                    xv[t][v] = t < nt ? __ldg(reinterpret_cast<const uint4 *>(row + (int64_t)t * D) + v)
-                                      : make_uint4(0u, 0u, 0u, 0u);
+                    xv[gi][t][v] = (i < NG8 && t < nt) ? __ldg(reinterpret_cast<const uint4 *>(row + (int64_t)t * D) + v)
+                                                      : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int gi = 0; gi < GPT; ++gi) {
+            const int i = tid + gi * NT;
+            if (i >= NG8) continue;
+            const int c0 = 8 * i;
+            const uint4 (&xg)[4][8 / VEC] = xv[gi];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 const KvoCluster k0 = cl[kcl[c0 + e]], k1 = cl[kcl[c0 + e + 1]];
                 uint32_t w0 = 0, w1 = 0;
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
-                    const f32x2 x2 = pair_of<T>(xv[t][e / VEC], (e % VEC) / 2);
+                    const f32x2 x2 = pair_of<T>(xg[t][e / VEC], (e % VEC) / 2);
                     w0 |= kvo_code<BITS>(lo2(x2), k0) << (8 * t);
                     w1 |= kvo_code<BITS>(hi2(x2), k1) << (8 * t);
                 }
@@ -659,7 +679,7 @@ __global__ void __launch_bounds__(KVO_THREADS)
             }
         }
         __syncthreads();
-        for (int pu = tid; pu < NU; pu += KVO_THREADS) {
+        for (int pu = tid; pu < NU; pu += NT) {
             uint32_t o[4][4];  // [group m of 8 stored columns][token]
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
@@ -703,25 +723,39 @@ cudaError_t launch_kv_quant_reordered(const KvReorderedArgs &a)
     if (units == 0) return cudaSuccess;
     const int C = a.H * a.D;
     const size_t smem = kvo_smem_bytes(C, a.g);
+    // wide rows (C > 8192) take 1024-thread CTAs (one per SM, by shared memory) so that every SM
+    // keeps 32 warps; narrower ones 256-thread CTAs, several per SM; groups of 8 channels per
+    // thread rounded up to a compiled count
+    const bool wide = C > 8192;
+    const int nt = wide ? 1024 : KVO_THREADS;
+    const int gpt = (C / 8 + nt - 1) / nt;
+    auto pick = [&](auto k1, auto k2, auto k4, auto k8, auto w2) {
+        return wide ? (const void *)w2
+                    : gpt <= 1 ? (const void *)k1 : gpt <= 2 ? (const void *)k2 : gpt <= 4 ? (const void *)k4 : (const void *)k8;
+    };
+#define KVO_PICK(T_, B_)                                                                                     \
+    pick(kv_quant_reordered_kernel<T_, B_, 1, KVO_THREADS>, kv_quant_reordered_kernel<T_, B_, 2, KVO_THREADS>, \
+         kv_quant_reordered_kernel<T_, B_, 4, KVO_THREADS>, kv_quant_reordered_kernel<T_, B_, 8, KVO_THREADS>, \
+         kv_quant_reordered_kernel<T_, B_, 2, 1024>)
     const void *kern = nullptr;
     if (a.dtype == 0)
-        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<float, 4> : (const void *)kv_quant_reordered_kernel<float, 3>;
+        kern = a.bits == 4 ? KVO_PICK(float, 4) : KVO_PICK(float, 3);
     else if (a.dtype == 1)
-        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<__half, 4> : (const void *)kv_quant_reordered_kernel<__half, 3>;
+        kern = a.bits == 4 ? KVO_PICK(__half, 4) : KVO_PICK(__half, 3);
     else
-        kern = a.bits == 4 ? (const void *)kv_quant_reordered_kernel<__nv_bfloat16, 4>
-                           : (const void *)kv_quant_reordered_kernel<__nv_bfloat16, 3>;
+        kern = a.bits == 4 ? KVO_PICK(__nv_bfloat16, 4) : KVO_PICK(__nv_bfloat16, 3);
+#undef KVO_PICK
     cudaError_t e = kernel_smem(kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 1;
-    e = kernel_occupancy(&per_sm, kern, KVO_THREADS, smem);
+    e = kernel_occupancy(&per_sm, kern, nt, smem);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<int64_t>(units, (int64_t)a.num_sms * std::max(1, per_sm));
     int H = a.H, D = a.D, g = a.g;
     int64_t S = a.S, U = units;
     void *args[] = {(void *)&a.kv, (void *)&H, (void *)&S, (void *)&D, (void *)&U, (void *)&a.R,
                     (void *)&a.col_cluster, (void *)&a.scale, (void *)&a.zero, (void *)&g, (void *)&a.codes, (void *)&a.err};
-    return cudaLaunchKernel(kern, dim3((unsigned)grid), dim3(KVO_THREADS), args, smem, a.stream);
+    return cudaLaunchKernel(kern, dim3((unsigned)grid), dim3(nt), args, smem, a.stream);
 }
 
 }  // namespace rptq
