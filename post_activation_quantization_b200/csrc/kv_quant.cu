@@ -552,29 +552,31 @@ extern "C" int rptq_testing_kv_quotient(const float *x, int64_t n, float s, floa
 namespace rptq {
 namespace {
 constexpr int KVO_THREADS = 256;
-struct KvoCluster {
-    float ns, r, s;    // -s 2^24, RN(1/s) 2^-24, s
-    int32_t lo, hi, z;  // clamp of the rounded bit pattern: MAGIC_BITS - z .. + qmax
-    int32_t fast, pad;
+// per cluster, 16 bytes (one shared-memory load per channel): -s 2^24, RN(1/s) 2^-24 and the
+// clamp of the rounded bit pattern, MAGIC_BITS - z .. + qmax; s and z for the IEEE path
+struct KvoFast {
+    float ns, r;
+    int32_t lo, hi;
+};
+struct KvoSlow {
+    float s;
+    int32_t z;
 };
 __host__ __device__ inline size_t kvo_smem_bytes(int C, int g)
 {
-    return ((size_t)C * 6 + 15) / 16 * 16 + (size_t)g * sizeof(KvoCluster) + (size_t)C * 4;
+    return (size_t)C * 4 + ((size_t)g * (sizeof(KvoFast) + sizeof(KvoSlow)) + 15) / 16 * 16 + (size_t)C * 4;
 }
 }  // namespace
 
-template <int BITS>
-__device__ __forceinline__ uint32_t kvo_code(float x, const KvoCluster &k)
+// The code of x in a cluster whose scale and zero point take the fast quotient (kv_fast_scale,
+// |z| < 2^21): the same operations as kv_quant_row's fast path
+__device__ __forceinline__ uint32_t kvo_code(float x, const KvoFast &k)
 {
-    constexpr int QMAX = (1 << BITS) - 1;
-    if (k.fast) {
-        const float q0 = x * k.r;
-        const float qq = __fmaf_rn(__fmaf_rn(q0, k.ns, x), k.r, q0);  // RN(x / (s 2^24))
-        const float b = __fmaf_rn(qq, KV_QSCALE, MAGIC_RINT);           // 1.5*2^23 + rint(x / s)
-        const int32_t l = min(max((int32_t)__float_as_uint(b), k.lo), k.hi);
-        return (uint32_t)(l - k.lo);
-    }
-    return kv_code_ieee<QMAX>(x, k.s, k.z);
+    const float q0 = x * k.r;
+    const float qq = __fmaf_rn(__fmaf_rn(q0, k.ns, x), k.r, q0);  // RN(x / (s 2^24))
+    const float b = __fmaf_rn(qq, KV_QSCALE, MAGIC_RINT);           // 1.5*2^23 + rint(x / s)
+    const int32_t l = min(max((int32_t)__float_as_uint(b), k.lo), k.hi);
+    return (uint32_t)(l - k.lo);
 }
 
 template <typename T, int BITS, int GPT, int NT>
@@ -589,30 +591,29 @@ __global__ void __launch_bounds__(NT)
     constexpr int QMAX = (1 << BITS) - 1;
     extern __shared__ __align__(16) uint8_t kvo_smem[];
     const int C = H * D, tid = threadIdx.x;
-    uint32_t *posw = reinterpret_cast<uint32_t *>(kvo_smem);  // [C] word index of channel c's stored column
-    uint16_t *kcl = reinterpret_cast<uint16_t *>(posw + C);    // [C] cluster of channel c
-    KvoCluster *cl = reinterpret_cast<KvoCluster *>(kvo_smem + ((size_t)C * 6 + 15) / 16 * 16);  // [g]
-    uint32_t *cbuf = reinterpret_cast<uint32_t *>(cl + g);     // [C] 4 tokens' codes per stored column
+    // [C] per channel c: its stored column j (bits 0-15) and cluster (bits 16-24)
+    uint32_t *tab = reinterpret_cast<uint32_t *>(kvo_smem);
+    KvoFast *clf = reinterpret_cast<KvoFast *>(tab + C);  // [g]
+    KvoSlow *cls = reinterpret_cast<KvoSlow *>(clf + g);                                    // [g]
+    // [C] 4 tokens' codes per stored column (16-byte aligned: read 4 words at a time)
+    uint32_t *cbuf = reinterpret_cast<uint32_t *>((reinterpret_cast<uintptr_t>(cls + g) + 15) & ~(uintptr_t)15);
 
-    for (int c = tid; c < C; c += NT) {
-        posw[c] = 0;
-        kcl[c] = 0;
-    }
+    for (int c = tid; c < C; c += NT) tab[c] = 0;
+    bool fast = true;
     for (int k = tid; k < g; k += NT) {
         const float sv = scale[k];
         const int z = zero[k];
-        KvoCluster e;
+        KvoFast e;
         e.ns = -(sv * KV_QSCALE);
         e.r = __frcp_rn(sv) * KV_QSCALE_INV;
-        e.s = sv;
-        e.z = z;
         e.lo = (int32_t)(MAGIC_BITS - (uint32_t)z);
         e.hi = (int32_t)(MAGIC_BITS + (uint32_t)QMAX - (uint32_t)z);
-        e.fast = (z > -(1 << 21)) && (z < (1 << 21)) && kv_fast_scale(sv);
-        e.pad = 0;
-        cl[k] = e;
+        clf[k] = e;
+        cls[k] = KvoSlow{sv, z};
+        fast &= (z > -(1 << 21)) && (z < (1 << 21)) && kv_fast_scale(sv);
     }
-    __syncthreads();
+    // every cluster takes the fast quotient, or every element the IEEE division (the same codes)
+    const bool all_fast = __syncthreads_and(fast) != 0;
     for (int j = tid; j < C; j += NT) {
         const int c = R[j];
         int k = col_cluster[j];
@@ -624,8 +625,7 @@ __global__ void __launch_bounds__(NT)
             raise_error(err, RPTQ_DEVERR_REORDER);
             continue;
         }
-        posw[c] = (uint32_t)j;
-        kcl[c] = (uint16_t)k;
+        tab[c] = (uint32_t)j | ((uint32_t)k << 16);
     }
     __syncthreads();
 
@@ -664,18 +664,31 @@ __global__ void __launch_bounds__(NT)
             if (i >= NG8) continue;
             const int c0 = 8 * i;
             const uint4 (&xg)[4][8 / VEC] = xv[gi];
+            const uint4 ta = *reinterpret_cast<const uint4 *>(tab + c0), tb = *reinterpret_cast<const uint4 *>(tab + c0 + 4);
+            const uint32_t te[8] = {ta.x, ta.y, ta.z, ta.w, tb.x, tb.y, tb.z, tb.w};
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
-                const KvoCluster k0 = cl[kcl[c0 + e]], k1 = cl[kcl[c0 + e + 1]];
+                const int ka = (int)(te[e] >> 16), kb = (int)(te[e + 1] >> 16);
                 uint32_t w0 = 0, w1 = 0;
+                if (all_fast) {
+                    const KvoFast k0 = clf[ka], k1 = clf[kb];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const f32x2 x2 = pair_of<T>(xg[t][e / VEC], (e % VEC) / 2);
-                    w0 |= kvo_code<BITS>(lo2(x2), k0) << (8 * t);
-                    w1 |= kvo_code<BITS>(hi2(x2), k1) << (8 * t);
+                    for (int t = 0; t < 4; ++t) {
+                        const f32x2 x2 = pair_of<T>(xg[t][e / VEC], (e % VEC) / 2);
+                        w0 |= kvo_code(lo2(x2), k0) << (8 * t);
+                        w1 |= kvo_code(hi2(x2), k1) << (8 * t);
+                    }
+                } else {
+                    const KvoSlow k0 = cls[ka], k1 = cls[kb];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const f32x2 x2 = pair_of<T>(xg[t][e / VEC], (e % VEC) / 2);
+                        w0 |= kv_code_ieee<QMAX>(lo2(x2), k0.s, k0.z) << (8 * t);
+                        w1 |= kv_code_ieee<QMAX>(hi2(x2), k1.s, k1.z) << (8 * t);
+                    }
                 }
-                cbuf[posw[c0 + e]] = w0;
-                cbuf[posw[c0 + e + 1]] = w1;
+                cbuf[te[e] & 0xFFFFu] = w0;
+                cbuf[te[e + 1] & 0xFFFFu] = w1;
             }
         }
         __syncthreads();

@@ -73,6 +73,19 @@ def test_cluster_ordered_cache_matches_oracle_and_kept_layout(B, H, S, D, dtype,
     assert np.array_equal(to_np(deq), want)
 
 
+def test_huge_zero_point_takes_the_ieee_division():
+    """A zero point beyond 2^21 leaves the fast quotient's range: every element then takes the IEEE
+    division and the definition directly; the codes still equal the oracle's exactly."""
+    B, H, S, D, g, bits = 2, 4, 9, 32, 6, 4
+    kv, kv32, cal, p = _case(B, H, S, D, "bf16", g, bits, 23)
+    z = cal["zero"].copy()
+    z[1] = (1 << 22) + 5  # every channel of cluster 1 clamps to 15 (or 0 for very negative x)
+    ref = oracle.kv_quant_cluster_ordered(kv32, cal["R"], cal["col_cluster"], cal["scale"], z, bits)
+    got = rptq.rptq_kv_quant_cluster_ordered(kv.to(DEV), p["R"], p["col_cluster"], p["scale"],
+                                             torch.from_numpy(z).to(DEV), bits)
+    assert np.array_equal(to_np(got), ref)
+
+
 def test_refusals_and_empty():
     kv, kv32, cal, p = _case(1, 2, 8, 16, "bf16", 4, 3, 5)  # C = 32
     args = (p["R"], p["col_cluster"], p["scale"], p["zero"])
