@@ -564,7 +564,7 @@ struct KvoSlow {
 };
 __host__ __device__ inline size_t kvo_smem_bytes(int C, int g)
 {
-    return (size_t)C * 4 + ((size_t)g * (sizeof(KvoFast) + sizeof(KvoSlow)) + 15) / 16 * 16 + (size_t)C * 4;
+    return (size_t)C * 4 + ((size_t)g * (sizeof(KvoFast) + sizeof(KvoSlow)) + 15) / 16 * 16 + (size_t)C * 8;
 }
 }  // namespace
 
@@ -595,8 +595,9 @@ __global__ void __launch_bounds__(NT)
     uint32_t *tab = reinterpret_cast<uint32_t *>(kvo_smem);
     KvoFast *clf = reinterpret_cast<KvoFast *>(tab + C);  // [g]
     KvoSlow *cls = reinterpret_cast<KvoSlow *>(clf + g);                                    // [g]
-    // [C] 4 tokens' codes per stored column (16-byte aligned: read 4 words at a time)
-    uint32_t *cbuf = reinterpret_cast<uint32_t *>((reinterpret_cast<uintptr_t>(cls + g) + 15) & ~(uintptr_t)15);
+    // two code buffers used by turns, [C] words each: 4 tokens' codes per stored column (16-byte
+    // aligned: read 4 words at a time); with two, one barrier per quad suffices
+    uint32_t *cbuf2 = reinterpret_cast<uint32_t *>((reinterpret_cast<uintptr_t>(cls + g) + 15) & ~(uintptr_t)15);
 
     for (int c = tid; c < C; c += NT) tab[c] = 0;
     bool fast = true;
@@ -640,9 +641,11 @@ __global__ void __launch_bounds__(NT)
             prefetch_l2(kv + ((b * H + h) * S + s0) * D, (uint32_t)(nt * D * (int)sizeof(T)));
     };
     prefetch_unit(blockIdx.x);
-    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    int par = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, par ^= 1) {
         const int64_t b = u / NQ, s0 = (u - b * NQ) * 4;
         const int nt = (int)min((int64_t)4, S - s0);
+        uint32_t *cbuf = cbuf2 + (size_t)par * C;
         prefetch_unit(u + gridDim.x);
         // every row load of the thread's groups first (GPT groups of 8 channels, 4 tokens each)
         uint4 xv[GPT][4][8 / VEC];
@@ -719,7 +722,8 @@ __global__ void __launch_bounds__(NT)
                 }
             }
         }
-        __syncthreads();  // the code buffer is refilled by the next quad
+        // no barrier: the next quad fills the other buffer, and the barrier after its scatter
+        // comes before this buffer is filled again
     }
 }
 
