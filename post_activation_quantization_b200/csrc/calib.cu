@@ -382,6 +382,12 @@ __global__ void __launch_bounds__(512, 1)
         pipe.advance();
     }
     if (lq == 0) return;  // this CTA saw no rows
+    // The CTA's extremes pass through shared memory so that the atomics of a warp cover 32
+    // consecutive channels (from registers, a thread's VEC consecutive channels would spread
+    // them VEC words apart over VEC times as many lines).  The ring is idle here: every row
+    // copied into it has been read, and its 4 or more rows of C values hold the 2 C floats.
+    __syncthreads();
+    float *shi = reinterpret_cast<float *>(smem), *slo = shi + C;
 #pragma unroll
     for (int k = 0; k < CPT; ++k) {
         const int ch = tid + k * NT;
@@ -390,11 +396,14 @@ __global__ void __launch_bounds__(512, 1)
         for (int e = 0; e < VEC; ++e) {
             const int c = ch * VEC + e;
             const float gm = gamma[c], bt = beta[c];
-            const float hi = fmaf(gm >= 0.f ? tmax[k][e] : tmin[k][e], gm, bt);
-            const float lo = fmaf(gm >= 0.f ? tmin[k][e] : tmax[k][e], gm, bt);
-            atomic_max_f32(ch_max + c, hi);
-            atomic_min_f32(ch_min + c, lo);
+            shi[c] = fmaf(gm >= 0.f ? tmax[k][e] : tmin[k][e], gm, bt);
+            slo[c] = fmaf(gm >= 0.f ? tmin[k][e] : tmax[k][e], gm, bt);
         }
+    }
+    __syncthreads();
+    for (int c = tid; c < C; c += NT) {
+        atomic_max_f32(ch_max + c, shi[c]);
+        atomic_min_f32(ch_min + c, slo[c]);
     }
 }
 
