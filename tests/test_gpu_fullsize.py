@@ -141,3 +141,79 @@ def test_kv_full_size(name):
                                 cal["scale"], cal["zero"], kvw.bits)
             ref[sel] = oracle.pack(q, kvw.bits)
         compare_codes(to_np(got.reshape(nrow, -1)[ri]), ref, D, kvw.bits, f"{name} kv")
+
+
+@pytest.mark.parametrize("name", ["opt66b-9216", "opt175b-12288"])
+def test_dequant_and_dynamic_ranges_full_size(name):
+    """The rows-layout dequantization of the whole batch's codes into the batch's dtype (the call
+    the benchmark times), bit-exact on sampled rows against oracle.dequant of the same codes; and
+    the dynamic ranges of the whole batch: rptq_cluster_params of the GPU's LayerNorm statistics
+    bit-exact against oracle.cluster_params of the same statistics (the statistics themselves are
+    covered by the calibration tests above)."""
+    w = WORKLOADS[name]
+    m, gamma, beta, x, cal = _act_setup(w)
+    p = dev_params(cal)
+    gd, bd = gamma.to(DEV), beta.to(DEV)
+    codes, _ = rptq.rptq_ln_reorder_quant(x, gd, bd, p["R"], p["col_cluster"], p["scale"], p["zero"], w.bits,
+                                          eps=w.eps)
+    out = torch.empty((w.T, w.C), dtype=x.dtype, device=DEV)
+    rptq.rptq_dequant(codes, p["col_cluster"], p["scale"], p["zero"], w.bits, out=out)
+    torch.cuda.synchronize()
+    rows = np.unique(np.concatenate([[0, w.T - 1], np.random.default_rng(w.seed + 1).choice(w.T, 256, False)]))
+    ri = torch.from_numpy(rows).to(DEV)
+    q = oracle.unpack(to_np(codes[ri]), w.C, w.bits)
+    ref = torch.from_numpy(oracle.dequant(q, cal["col_cluster"], cal["scale"], cal["zero"])).to(x.dtype)
+    assert torch.equal(out[ri].cpu(), ref), name
+    mx, mn = rptq.rptq_calib_minmax(x, gd, bd, w.eps)
+    s, z = rptq.rptq_cluster_params(mx, mn, p["labels"], w.g, w.bits)
+    rs, rz = oracle.cluster_params(to_np(mx), to_np(mn), cal["labels"], w.g, w.bits)
+    assert np.array_equal(to_np(s).view(np.uint32), rs.view(np.uint32)) and np.array_equal(to_np(z), rz), name
+    del x, out, codes
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", KVW)
+def test_kv_cluster_order_and_dequant_full_size(name):
+    """The K cache at full size stored in cluster order (rptq_kv_quant_cluster_ordered, as the
+    benchmark launches it), sampled token rows against oracle.kv_quant_cluster_ordered of the
+    same tokens; and the kept-layout codes of K and V read back by rptq_dequant's [B, H, S, D]
+    layout, sampled rows bit-exact against oracle.kv_dequant."""
+    w, kvw, (k, v) = _kv_setup(name)
+    B, H, S, D, bits = kvw.B, kvw.H, kvw.S, kvw.D, kvw.bits
+    C = H * D
+    rng = np.random.default_rng(w.seed + 2)
+    cals = []
+    for t in (k, v):
+        tok = t.permute(0, 2, 1, 3).reshape(B * S, C)[:2048].cpu()
+        omx, omn = oracle.minmax(tok)
+        cals.append(oracle.calibrate(omx, omn, kvw.g, kvw.iters, bits))
+    pk, pv = dev_params(cals[0]), dev_params(cals[1])
+    co = rptq.rptq_kv_quant_cluster_ordered(k, pk["R"], pk["col_cluster"], pk["scale"], pk["zero"], bits)
+    torch.cuda.synchronize()
+    tok = np.unique(np.concatenate([[0, B * S - 1], rng.choice(B * S, 384, replace=False)]))
+    bi, si = torch.from_numpy(tok // S).to(DEV), torch.from_numpy(tok % S).to(DEV)
+    sub = k[bi, :, si, :].unsqueeze(2).cpu()  # [n, H, 1, D]: every sampled token as its own batch row
+    ref = oracle.kv_quant_cluster_ordered(sub, cals[0]["R"], cals[0]["col_cluster"], cals[0]["scale"],
+                                          cals[0]["zero"], bits)
+    compare_codes(to_np(co[bi, si]), ref.reshape(len(tok), -1), C, bits, f"{name} k cluster order")
+    del co
+    kq, vq = rptq.rptq_kv_quant(k, v, pk["labels"], pk["scale"], pk["zero"], pv["labels"], pv["scale"],
+                                pv["zero"], bits)
+    nrow = B * H * S
+    rows = np.unique(np.concatenate([[0, nrow - 1], rng.choice(nrow, 1024, replace=False)]))
+    ri = torch.from_numpy(rows).to(DEV)
+    for codes, cal, pd, t in ((kq, cals[0], pk, k), (vq, cals[1], pv, v)):
+        out = torch.empty((B, H, S, D), dtype=t.dtype, device=DEV)
+        rptq.rptq_dequant(codes, pd["labels"], pd["scale"], pd["zero"], bits, layout=rptq.RPTQ_LAYOUT_BHSD, out=out)
+        torch.cuda.synchronize()
+        sel = codes.reshape(nrow, -1)[ri].cpu().numpy()
+        hh = (rows // S) % H
+        want = np.empty((len(rows), D), np.float32)
+        for h in np.unique(hh):
+            m_ = hh == h
+            want[m_] = oracle.kv_dequant(sel[m_].reshape(1, 1, -1, D * bits // 8), D,
+                                         cal["labels"][h * D:(h + 1) * D], cal["scale"], cal["zero"],
+                                         bits).reshape(-1, D)
+        assert torch.equal(out.reshape(nrow, D)[ri].cpu(), torch.from_numpy(want).to(t.dtype)), name
+    del k, v, kq, vq
+    torch.cuda.empty_cache()

@@ -49,6 +49,8 @@ def _case(B, H, S, D, dtype, g, bits, seed):
     (2, 96, 64, 128, "bf16", 64, 3),  # the OPT-175B cache width
     (1, 3, 2, 256, "bf16", 12, 4),    # fewer tokens than one quad
     (2, 5, 19, 96, "f16", 10, 3),     # D = 96 (not a power of two), C = 480
+    (1, 128, 9, 128, "bf16", 512, 4), # the largest width (16384 channels) and cluster count
+    (1, 64, 6, 256, "f32", 100, 3),   # 16384 channels of fp32
 ])
 def test_cluster_ordered_cache_matches_oracle_and_kept_layout(B, H, S, D, dtype, g, bits):
     C = H * D
