@@ -217,3 +217,51 @@ def test_kv_cluster_order_and_dequant_full_size(name):
         assert torch.equal(out.reshape(nrow, D)[ri].cpu(), torch.from_numpy(want).to(t.dtype)), name
     del k, v, kq, vq
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", KVW)
+def test_kv_decode_step_full_size(name):
+    """The decode step as the benchmark launches it on the full caches: one new token appended
+    at position S - 1 of the packed K and V caches, then attention of one query per (b, h) over
+    all S positions.  The appended rows against oracle.kv_quant of the new token (codes bar, on
+    every (b, h)); the attention of the first and last batch entries (all heads) against
+    oracle.kv_decode_attention within the bound derived from the kernel's fp32 evaluation order."""
+    from tests.test_gpu_kv_decode import _attn_bound
+    w, kvw, (k, v) = _kv_setup(name)
+    B, H, S, D, bits = kvw.B, kvw.H, kvw.S, kvw.D, kvw.bits
+    C = H * D
+    cals = []
+    for t in (k, v):
+        tok = t.permute(0, 2, 1, 3).reshape(B * S, C)[:2048].cpu()
+        omx, omn = oracle.minmax(tok)
+        cals.append(oracle.calibrate(omx, omn, kvw.g, kvw.iters, bits))
+    pk, pv = dev_params(cals[0]), dev_params(cals[1])
+    kq, vq = rptq.rptq_kv_quant(k, v, pk["labels"], pk["scale"], pk["zero"], pv["labels"], pv["scale"],
+                                pv["zero"], bits)
+    del k, v
+    mk = synthetic.channel_model(kvw.channels, w.seed, kvw.outlier_frac, kvw.outlier_factor, tag=1)
+    mv = synthetic.channel_model(kvw.channels, w.seed, kvw.outlier_frac, kvw.outlier_factor, tag=2)
+    knew = synthetic.kv_cache(B, H, 1, D, mk, w.seed + 1, "k", dtype=kvw.dtype, device=DEV)
+    vnew = synthetic.kv_cache(B, H, 1, D, mv, w.seed + 1, "v", dtype=kvw.dtype, device=DEV)
+    rptq.rptq_kv_append(knew, vnew, pk["labels"], pk["scale"], pk["zero"], pv["labels"], pv["scale"], pv["zero"],
+                        bits, k_cache=kq, v_cache=vq, s_begin=S - 1)
+    for new, cal, cache in ((knew, cals[0], kq), (vnew, cals[1], vq)):
+        ref = oracle.kv_quant(new.cpu(), cal["labels"], cal["scale"], cal["zero"], bits)
+        compare_codes(to_np(cache[:, :, S - 1:S]), ref, D, bits, f"{name} appended row")
+    gq = torch.Generator(device=DEV)
+    gq.manual_seed(w.seed * 31)
+    q = torch.randn((B, H, D), generator=gq, device=DEV, dtype=torch.float32) * 0.05
+    out = rptq.rptq_kv_decode_attention(q, kq, vq, S, pk["labels"], pk["scale"], pk["zero"], pv["labels"],
+                                        pv["scale"], pv["zero"], bits)
+    torch.cuda.synchronize()
+    bsel = torch.tensor([0, B - 1], device=DEV)
+    qs, kc, vc = to_np(q[bsel]), kq[bsel].cpu().numpy(), vq[bsel].cpu().numpy()
+    ref, _ = oracle.kv_decode_attention(qs, kc, vc, S, D, cals[0]["labels"], cals[0]["scale"], cals[0]["zero"],
+                                        cals[1]["labels"], cals[1]["scale"], cals[1]["zero"], bits)
+    Kd = oracle.kv_dequant(kc, D, cals[0]["labels"], cals[0]["scale"], cals[0]["zero"], bits)
+    Vd = oracle.kv_dequant(vc, D, cals[1]["labels"], cals[1]["scale"], cals[1]["zero"], bits)
+    tol = _attn_bound(qs, Kd, Vd, S, D, 1.0 / np.sqrt(D))
+    err = np.abs(to_np(out[bsel]).astype(np.float64) - ref)
+    assert (err <= tol).all(), f"{name}: worst excess {(err - tol).max():.3e}"
+    del kq, vq
+    torch.cuda.empty_cache()
