@@ -270,14 +270,18 @@ __device__ __forceinline__ int checked_cluster(const int32_t *cluster, int c, in
 }
 
 // Rows layout, C % 256 == 0: CTA = WR warps, warp w owns spans w + WR*i (i < NSPAN) of every row.
-template <typename T, int BITS, int NSPAN>
+// SPLIT: the row's spans are split into `parts` column ranges of WR * NSPAN spans, CTA b taking
+// range b % parts of every (gridDim / parts)-th row, so that rows too wide for one CTA of one
+// span per warp still get several resident CTAs per SM.
+template <typename T, int BITS, int NSPAN, bool SPLIT>
 __global__ void __launch_bounds__(NSPAN <= 2 ? 1024 : 512)
     dequant_rows_span(const uint8_t *__restrict__ codes, int64_t rows, int C, const int32_t *__restrict__ cluster,
                       const float *__restrict__ scale, const int32_t *__restrict__ zero, int g, T *__restrict__ out,
-                      int *err)
+                      int *err, int parts)
 {
     constexpr int U = 4;  // rows in flight
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, WR = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, WR = blockDim.x >> 5;
+    const int w = (threadIdx.x >> 5) + (SPLIT ? (int)(blockIdx.x % parts) * WR * NSPAN : 0);
     const int64_t pitch = (int64_t)C * BITS / 8;
     float sc[NSPAN][8], nzf[NSPAN][8];
     bool exact = true;
@@ -294,8 +298,8 @@ __global__ void __launch_bounds__(NSPAN <= 2 ? 1024 : 512)
             nzf[i][e] = -(float)((1 << 23) + (ok ? z : 0));
         }
     exact = __all_sync(FULL, exact);  // the shuffles below need the whole warp on one path
-    const int64_t step = gridDim.x;
-    for (int64_t r0 = blockIdx.x; r0 < rows; r0 += U * step) {
+    const int64_t step = SPLIT ? gridDim.x / parts : gridDim.x;
+    for (int64_t r0 = SPLIT ? blockIdx.x / parts : blockIdx.x; r0 < rows; r0 += U * step) {
         uint32_t wv[U][NSPAN];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -580,18 +584,13 @@ static cudaError_t launch_dq_t(const DequantArgs &a)
     return cudaGetLastError();
 }
 
-template <typename T, int BITS, int NSPAN>
-static cudaError_t launch_rows_span(const DequantArgs &a, int WR)
+template <typename T, int BITS, int NSPAN, bool SPLIT>
+static cudaError_t launch_rows_span(const DequantArgs &a, int WR, int parts, int per_sm)
 {
     const int threads = WR * 32;
-    int per_sm = 1;
-    if (kernel_occupancy(&per_sm, (const void *)dequant_rows_span<T, BITS, NSPAN>, threads, 0) !=
-            cudaSuccess ||
-        per_sm < 1)
-        per_sm = 1;
-    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(a.n0, (int64_t)a.num_sms * per_sm));
-    dequant_rows_span<T, BITS, NSPAN><<<(unsigned)grid, threads, 0, a.stream>>>(
-        a.codes, a.n0, a.n1, a.cluster, a.scale, a.zero, a.g, (T *)a.out, a.err);
+    const int64_t ctas = std::max<int64_t>(1, std::min<int64_t>(a.n0, (int64_t)a.num_sms * per_sm / parts));
+    dequant_rows_span<T, BITS, NSPAN, SPLIT><<<(unsigned)(ctas * parts), threads, 0, a.stream>>>(
+        a.codes, a.n0, a.n1, a.cluster, a.scale, a.zero, a.g, (T *)a.out, a.err, parts);
     return cudaGetLastError();
 }
 
@@ -639,12 +638,37 @@ static cudaError_t launch_dq_b(const DequantArgs &a)
         }
     } else if (aligned && a.n1 % 256 == 0) {
         const int spans = a.n1 / 256;  // 256-channel spans per row, at most 64
-        // fewest spans per thread (most warps) that keep the CTA within 1024 (NSPAN <= 2) or
-        // 512 threads
-        if (spans <= 32) return launch_rows_span<T, BITS, 1>(a, spans);
-        if (spans % 2 == 0) return launch_rows_span<T, BITS, 2>(a, spans / 2);
-        if (spans % 3 == 0 && spans / 3 <= 16) return launch_rows_span<T, BITS, 3>(a, spans / 3);
-        if (spans % 4 == 0 && spans / 4 <= 16) return launch_rows_span<T, BITS, 4>(a, spans / 4);
+        // a CTA takes spans / parts spans of a row, NSPAN per warp: the first split (fewest
+        // parts, then fewest spans per warp) that keeps at least 24 warps resident on an SM,
+        // else the split with the most
+        const void *whole[5] = {nullptr, (const void *)dequant_rows_span<T, BITS, 1, false>,
+                                (const void *)dequant_rows_span<T, BITS, 2, false>,
+                                (const void *)dequant_rows_span<T, BITS, 3, false>,
+                                (const void *)dequant_rows_span<T, BITS, 4, false>};
+        const void *split[3] = {nullptr, (const void *)dequant_rows_span<T, BITS, 1, true>,
+                                (const void *)dequant_rows_span<T, BITS, 2, true>};
+        int bp = 0, bn = 0, bwarps = 0, bper = 0;
+        for (int parts = 1; parts <= 4; ++parts)
+            for (int n = 1; n <= (parts == 1 ? 4 : 2); ++n) {
+                if (spans % (parts * n) != 0) continue;
+                const int wr = spans / (parts * n);
+                if (wr * 32 > (n <= 2 ? 1024 : 512) || wr < std::min(4, spans)) continue;
+                int per_sm = 0;
+                if (kernel_occupancy(&per_sm, parts == 1 ? whole[n] : split[n], wr * 32, 0) != cudaSuccess) per_sm = 0;
+                if (per_sm * wr > bwarps && bwarps < 24) {
+                    bp = parts, bn = n, bwarps = per_sm * wr, bper = per_sm;
+                }
+            }
+        if (bn) {
+            const int wr = spans / (bp * bn);
+            if (bp > 1)
+                return bn == 1 ? launch_rows_span<T, BITS, 1, true>(a, wr, bp, bper)
+                               : launch_rows_span<T, BITS, 2, true>(a, wr, bp, bper);
+            if (bn == 1) return launch_rows_span<T, BITS, 1, false>(a, wr, 1, bper);
+            if (bn == 2) return launch_rows_span<T, BITS, 2, false>(a, wr, 1, bper);
+            if (bn == 3) return launch_rows_span<T, BITS, 3, false>(a, wr, 1, bper);
+            return launch_rows_span<T, BITS, 4, false>(a, wr, 1, bper);
+        }
     }
     const int width = a.layout == RPTQ_LAYOUT_BHSD ? a.D : a.n1;
     if (width % 32 == 0) return launch_dq_t<T, BITS, 32>(a);

@@ -272,7 +272,9 @@ def test_kv_quant(dtype, B, H, S, D, g, bits):
 # ---------------------------------------------------------------- dequantization
 @pytest.mark.parametrize("out_dtype", [torch.float32, torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("rows,C,bits", [(37, 768, 4), (5, 4096, 3), (3, 72, 3), (2, 40, 4), (9, 12288, 3),
-                                         (6, 12288, 4), (11, 9216, 3), (4, 256, 3), (3, 16384, 4)])
+                                         (6, 12288, 4), (11, 9216, 3), (4, 256, 3), (3, 16384, 4),
+                                         # rows split over several CTAs (column ranges), one row among them
+                                         (7, 5120, 4), (1, 9216, 3)])
 def test_dequant_rows_bit_exact(out_dtype, rows, C, bits):
     rng = np.random.default_rng(rows * C)
     g = 9
