@@ -226,10 +226,14 @@ __global__ void __launch_bounds__(256)
 
 // Ring form for 16-bit caches whose shape passes kv_ring_shape_ok (stages of kv_stream.cuh): the
 // eight pieces of a stage that a thread reads all hold its channel group, so it keeps one packed
-// running max / min; when the head changes (and at the end) the lanes sharing a channel group
-// are folded by shuffles and the result goes to the outputs with the same integer atomics.
+// running max / min.  When the head changes (and at the end) every thread of the CTA flushes:
+// the lanes sharing a channel group are folded by shuffles, the warps through a D-wide shared
+// buffer (fmx / fmn, integer atomics, exact and order-independent), and the CTA's result goes to
+// the outputs with the same integer atomics, one per channel and 32 consecutive channels per warp.
+// fmx / fmn hold -inf / +inf on entry and again on return.
 template <typename T>
-__device__ __forceinline__ void kv_calib_flush(const RawAcc<T> &acc, int h, int D, float *ch_max, float *ch_min)
+__device__ __forceinline__ void kv_calib_flush(const RawAcc<T> &acc, int h, int D, float *fmx, float *fmn,
+                                               float *ch_max, float *ch_min)
 {
     const int lane = threadIdx.x & 31, npr = D >> 3, col = threadIdx.x & (npr - 1);
     float m[8], n[8];
@@ -247,10 +251,21 @@ __device__ __forceinline__ void kv_calib_flush(const RawAcc<T> &acc, int h, int 
     if (lane < npr || npr >= 32)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            atomic_max_f32(ch_max + h * D + col * 8 + e, m[e]);
-            atomic_min_f32(ch_min + h * D + col * 8 + e, n[e]);
+            atomic_max_f32(fmx + col * 8 + e, m[e]);
+            atomic_min_f32(fmn + col * 8 + e, n[e]);
         }
+    __syncthreads();
+    for (int d = threadIdx.x; d < D; d += blockDim.x) {
+        atomic_max_f32(ch_max + h * D + d, fmx[d]);
+        atomic_min_f32(ch_min + h * D + d, fmn[d]);
+        fmx[d] = -INFINITY;
+        fmn[d] = INFINITY;
+    }
+    __syncthreads();  // the buffer is reset before any thread's next flush
 }
+
+constexpr int KVR_BAR_BYTES = 32;  // the ring's KVR_NS mbarriers, rounded up to 16 bytes
+static_assert(8 * KVR_NS <= KVR_BAR_BYTES, "ring barriers");
 
 template <typename T>
 __global__ void __launch_bounds__(KVR_THREADS, 2)
@@ -260,6 +275,7 @@ __global__ void __launch_bounds__(KVR_THREADS, 2)
     __shared__ int s_abort;
     uint8_t *ring = smem;
     const uint32_t bar0 = smem_u32(smem + (size_t)KVR_NS * KVR_STAGE);
+    float *fmx = reinterpret_cast<float *>(smem + (size_t)KVR_NS * KVR_STAGE + KVR_BAR_BYTES), *fmn = fmx + D;
     const int tid = threadIdx.x;
     const int64_t total = (int64_t)B * H * SPB;
     const int64_t j0 = total * blockIdx.x / gridDim.x, j1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -279,6 +295,10 @@ __global__ void __launch_bounds__(KVR_THREADS, 2)
         prod.set(j0, total, B, SPB);
         for (int s = 0; s < KVR_NS && s < n; ++s) issue((uint32_t)s);
     }
+    for (int d = tid; d < D; d += KVR_THREADS) {
+        fmx[d] = -INFINITY;
+        fmn[d] = INFINITY;
+    }
     __syncthreads();
     KvStagePos cur;
     cur.set(j0, total, B, SPB);
@@ -288,7 +308,7 @@ __global__ void __launch_bounds__(KVR_THREADS, 2)
     uint32_t slot = 0, phase = 0;
     for (int i = 0; i < n; ++i) {
         if (cur.h != acc_h) {  // the same in every thread
-            kv_calib_flush<T>(acc, acc_h, D, ch_max, ch_min);
+            kv_calib_flush<T>(acc, acc_h, D, fmx, fmn, ch_max, ch_min);
             acc.init();
             acc_h = cur.h;
         }
@@ -311,7 +331,7 @@ __global__ void __launch_bounds__(KVR_THREADS, 2)
             phase ^= 1u;
         }
     }
-    kv_calib_flush<T>(acc, acc_h, D, ch_max, ch_min);
+    kv_calib_flush<T>(acc, acc_h, D, fmx, fmn, ch_max, ch_min);
 }
 
 // ---- LayerNorm mode ------------------------------------------------------------------------
@@ -600,7 +620,8 @@ static cudaError_t launch_kv_calib_ring(const KvCalibArgs &a)
 {
     const int SPB = (int)(a.S / kv_ring_rows(a.D));
     auto kern = kv_calib_ring<T>;
-    const size_t smem = (size_t)KVR_NS * KVR_STAGE + 8 * KVR_NS;
+    // the stage ring, its barriers and the CTA's D-wide max / min fold buffer
+    const size_t smem = (size_t)KVR_NS * KVR_STAGE + KVR_BAR_BYTES + 8 * (size_t)a.D;
     cudaError_t e = kernel_smem((const void *)kern, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

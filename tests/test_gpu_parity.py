@@ -217,7 +217,9 @@ def test_ln_reorder_is_ln_then_gather():
                                      # whole 32 KB stages (16-bit): the streaming-ring kernel; the
                                      # last case has more stages than CTAs, so CTAs cross heads
                                      (2, 3, 128, 128), (1, 2, 2048, 8), (2, 5, 512, 32), (1, 2, 8, 2048),
-                                     (2, 4, 16384, 128)])
+                                     (2, 4, 16384, 128),
+                                     # channel groups spanning two warps (D = 512); many short heads
+                                     (2, 2, 64, 512), (3, 6, 256, 64)])
 def test_kv_calib_bit_exact(dtype, B, H, S, D):
     m = synthetic.channel_model(H * D, S, tag=1)
     kv = synthetic.kv_cache(B, H, S, D, m, S, "k", dtype=dtype)
