@@ -203,7 +203,7 @@ class Step:
         return stage_list(self.w)
 
     def repeat_calls(self):
-        """The benchmark spec's two kernels as single calls on the step's full-size buffers (for the
+        """The two headline kernels as single calls on the step's full-size buffers (for the
         back-to-back measurement): the planned fused LN-reorder-quant and the K/V quantizer."""
         r, w, k = self.r, self.w, self.kvw
         calls = {}
@@ -531,7 +531,7 @@ def run_rptq(args):
             step.run({n: ev[n][i] for n in ev})
     t1.record()
     torch.cuda.synchronize()
-    # the benchmark spec's kernels once more, launched back to back (inside the clock record)
+    # the two headline kernels once more, launched back to back (inside the clock record)
     b2b = {n: back_to_back_ms(c, mode == "graph") for n, c in step.repeat_calls().items()}
     if clk:
         clk.end()
